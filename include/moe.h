@@ -1,0 +1,207 @@
+/*
+ * moe.h -- C ABI of the B200 latent-MoE decode block (libmoe_b200.so).
+ *
+ * The block, per token b of a decode batch (B = 1..128 tokens):
+ *
+ *   logits = x . W_r                 router scores          } one weight-streaming pass
+ *   z      = x . W_in                latent input projection} over the same x
+ *   ids, w = top-k of the scores     softmax, or sigmoid + per-expert selection bias;
+ *                                    weights renormalised over the k chosen experts
+ *   y_j    = SwiGLU expert ids[j] on z, MXFP4 weights (e2m1 elements, e8m0 scale per 32)
+ *   out    = (sum_j w_j y_j) . W_out + SwiGLU_shared(x) . W_sd
+ *
+ * Sources of the operation:
+ *   - router scoring and the latent input projection computed together as one
+ *     matmul; the shared expert on its own stream, overlapping routing and the
+ *     selected experts: page "Hyper Optimizing Kimi K3 in vLLM: Moving Fast and
+ *     Responsibly", section 从算子之间找时间 ("finding time between operators");
+ *   - the MXFP4 top-k finalize (weighted combine) fused into the latent-tail
+ *     kernel, saving one launch and one intermediate write + re-read: page
+ *     "Kimi K3 在 vLLM 中的性能优化", section 延迟 MXFP4 最终化 ("deferred MXFP4
+ *     finalize");
+ *   - decode batch 1-64 and the 16 x 8 speculative-verify shape: page 1 intro
+ *     and page "Kimi K3 vLLM 优化：NVIDIA 解码速度提升 1.68×", section
+ *     上游测试实际展示了什么.
+ *   MXFP4 encodings follow the OCP Microscaling (MX) v1.0 specification.
+ *
+ * Conventions for every call:
+ *   - Status codes are returned; nothing throws across the ABI.  Invalid
+ *     arguments are detected on the host before anything is launched.
+ *   - "device pointer" means memory of the plan's device; "host pointer" means
+ *     ordinary or pinned host memory.
+ *   - Streams are passed as void* and are cudaStream_t values (NULL = legacy
+ *     default stream).
+ *   - A plan is used by one host thread and one stream at a time.
+ *   - There is no CPU fallback: without a usable sm_100 device every call that
+ *     needs the GPU returns MOE_ERR_UNSUPPORTED or MOE_ERR_CUDA.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, B out of range */
+  MOE_ERR_UNSUPPORTED = 2, /* shape or device this library does not implement */
+  MOE_ERR_NOT_LOADED = 3,  /* moe_forward before moe_load_weights succeeded */
+  MOE_ERR_OOM = 4,         /* a device or host allocation failed (plan create / load only) */
+  MOE_ERR_CUDA = 5,        /* a CUDA runtime call failed; the plan should be destroyed */
+  MOE_ERR_TIMEOUT = 6,     /* a device-side bounded wait gave up (reported by moe_sync_status) */
+  MOE_ERR_RANGE = 7        /* weights hold an encoding the block rejects (e8m0 NaN byte 0xFF) */
+} moe_status;
+
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
+
+/* Layer shape and routing rule, fixed at plan creation. */
+typedef struct moe_config {
+  int32_t hidden;       /* H: multiple of 32 */
+  int32_t latent;       /* L: multiple of 32 */
+  int32_t num_experts;  /* E: 1..1024 */
+  int32_t top_k;        /* k: 1..min(E, 16) */
+  int32_t expert_inter; /* I: multiple of 32 */
+  int32_t shared_inter; /* I_s: multiple of 32, or 0 for no shared expert */
+  int32_t max_tokens;   /* largest B a forward may pass: 1..128 */
+  int32_t score_fn;     /* MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID */
+  int32_t renormalize;  /* 1: combine weights divided by their sum over the k chosen */
+  float routed_scale;   /* factor applied to every combine weight (1.0 = none) */
+  int32_t shared_sms;   /* CTAs given to the side-stream shared expert, 0 = automatic */
+} moe_config;
+
+/*
+ * Weights in canonical layout, all DEVICE pointers, row-major, 16-byte aligned.
+ * bf16 tensors are in "x . W" orientation [in][out]; MXFP4 tensors are
+ * output-row-major with K (the reduction index) contiguous:
+ *   router_w   bf16 [H][E]
+ *   router_bias f32 [E]       selection bias (sigmoid scoring only); may be NULL
+ *   w_in       bf16 [H][L]
+ *   w_out      bf16 [L][H]
+ *   gu_codes   u8   [E][2I][L/2]   rows 0..I-1 gate, rows I..2I-1 up;
+ *                                  element 2t in the low nibble of byte t
+ *   gu_scales  u8   [E][2I][L/32]  e8m0, value 2^(s-127); 0xFF (NaN) rejected
+ *   dn_codes   u8   [E][L][I/2]
+ *   dn_scales  u8   [E][L][I/32]
+ *   sh_gate    bf16 [H][I_s]   (ignored when I_s == 0)
+ *   sh_up      bf16 [H][I_s]
+ *   sh_down    bf16 [I_s][H]
+ * The caller keeps ownership and may free them once moe_load_weights returns.
+ */
+typedef struct moe_weights {
+  const void *router_w;
+  const float *router_bias;
+  const void *w_in;
+  const void *w_out;
+  const uint8_t *gu_codes;
+  const uint8_t *gu_scales;
+  const uint8_t *dn_codes;
+  const uint8_t *dn_scales;
+  const void *sh_gate;
+  const void *sh_up;
+  const void *sh_down;
+} moe_weights;
+
+typedef struct moe_plan_s *moe_plan;
+
+/* What a plan chose, for logging and for checking that the fast path runs. */
+typedef struct moe_plan_info {
+  int32_t device;
+  int32_t num_sms;
+  int32_t main_ctas;        /* CTAs of the main-stream kernels while the side stream runs */
+  int32_t shared_ctas;      /* CTAs of the side-stream shared-expert kernel */
+  int64_t packed_bytes;     /* library-owned packed weights */
+  int64_t workspace_bytes;  /* library-owned activations, routing metadata, partial sums */
+  int64_t dense_weight_bytes;      /* bf16 bytes one forward streams regardless of routing */
+  int64_t expert_weight_bytes;     /* MXFP4 bytes of one expert (gate/up + down, codes + scales) */
+  int32_t kernels_per_forward;     /* launches one moe_forward makes */
+} moe_plan_info;
+
+/*
+ * Create a plan on `device`: checks the shape, allocates packed-weight storage,
+ * workspace, a side stream and events.  *out receives the plan.
+ * Errors: INVALID_ARG (null, bad shape), UNSUPPORTED (no sm_100 device, shape
+ * beyond the limits above), OOM, CUDA.
+ */
+MOE_API moe_status moe_plan_create(const moe_config *cfg, int device, moe_plan *out);
+
+/*
+ * Pack canonical weights (device pointers, see moe_weights) into the plan's
+ * kernel layouts.  Runs kernels on `stream` and synchronises it before
+ * returning.  Rejects e8m0 byte 0xFF with MOE_ERR_RANGE (plan stays unloaded).
+ */
+MOE_API moe_status moe_load_weights(moe_plan p, const moe_weights *w, void *stream);
+
+/*
+ * out[B][H] (bf16, device) = block(x[B][H] bf16, device).  B = num_tokens,
+ * 1..max_tokens.  x and out must be 16-byte aligned and must not overlap.
+ * Asynchronous on `stream`: allocates nothing, does no host synchronisation,
+ * may be captured into a CUDA graph.  Internally forks the shared expert onto
+ * the plan's side stream and joins it back before returning control of
+ * `stream`.  Errors: INVALID_ARG, NOT_LOADED, CUDA (launch failure).
+ */
+MOE_API moe_status moe_forward(moe_plan p, const void *x, int32_t num_tokens, void *out, void *stream);
+
+/*
+ * Same block with HOST buffers: copies x_host to a plan-owned device buffer,
+ * runs moe_forward and copies the result to out_host, all enqueued on
+ * `stream`.  With pinned host memory the call is asynchronous; the caller
+ * synchronises `stream` before reading out_host.
+ */
+MOE_API moe_status moe_forward_host(moe_plan p, const void *x_host, int32_t num_tokens, void *out_host,
+                            void *stream);
+
+/*
+ * Copy the routing of the most recent forward to host memory (synchronises
+ * the device): ids_host[B][k] int32 in key-descending order, w_host[B][k]
+ * float combine weights.  Either pointer may be NULL.
+ */
+MOE_API moe_status moe_last_routing(moe_plan p, int32_t *ids_host, float *w_host, int32_t num_tokens);
+
+/* Intermediates of the most recent forward, decoded to float32 (synchronises). */
+enum {
+  MOE_DBG_LOGITS = 0, /* [B][E] router logits */
+  MOE_DBG_Z = 1,      /* [B][L] latent activations as stored for the experts */
+  MOE_DBG_H = 2,      /* [B][k][I] expert SwiGLU outputs as stored for the down projection */
+  MOE_DBG_Y = 3,      /* [B][k][L] expert outputs (before the weighted combine) */
+  MOE_DBG_HS = 4      /* [B][I_s] shared-expert SwiGLU output */
+};
+MOE_API moe_status moe_debug_fetch(moe_plan p, int32_t what, int32_t num_tokens, float *host, int64_t count);
+
+/* Synchronise the plan's streams and report a device-side error word
+ * (MOE_ERR_TIMEOUT if a bounded wait gave up), then clear it. */
+MOE_API moe_status moe_sync_status(moe_plan p);
+
+MOE_API moe_status moe_get_plan_info(moe_plan p, moe_plan_info *info);
+
+/*
+ * Per-kernel timing, for measurement only.  While enabled, moe_forward brackets
+ * each of its kernels with CUDA events on the stream that kernel runs on and
+ * waits for them before returning (so profiled forwards are synchronous and
+ * must not be captured into a graph).  moe_get_profile writes the accumulated
+ * milliseconds per kernel in launch-kind order {router+latent, shared gate/up,
+ * expert gate/up, expert down, latent tail} to ms[0..4] and the number of
+ * profiled forwards to *count, then clears both.
+ */
+MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
+MOE_API moe_status moe_get_profile(moe_plan p, float *ms, int32_t *count);
+
+/* Release everything the plan owns.  NULL is ignored. */
+MOE_API void moe_plan_destroy(moe_plan p);
+
+/* Static string for a status code. */
+MOE_API const char *moe_status_str(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

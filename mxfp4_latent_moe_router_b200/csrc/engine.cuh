@@ -1,0 +1,94 @@
+// engine.cuh -- kernel parameters shared by the launchers and the kernels.
+#pragma once
+#include <cstdint>
+
+#include "layout.cuh"
+
+namespace moe {
+
+enum Kind : int {
+  KIND_RL = 0,    // router logits + latent projection (+ top-k by the last router row block)
+  KIND_SGU = 1,   // shared expert gate/up + SwiGLU (side stream)
+  KIND_EGU = 2,   // routed experts gate/up + SwiGLU, MXFP4
+  KIND_EDN = 3,   // routed experts down projection, MXFP4
+  KIND_TAIL = 4,  // weighted combine + W_out, plus shared down projection -> out
+  KIND_COUNT = 5
+};
+
+// Per-kernel scheduling state in device memory, zero between launches: the
+// piece cursor is reset by the last CTA to leave.
+struct Ctl {
+  int cursor;
+  int exits;
+  int pad[30];
+};
+
+// error word bits
+enum : int {
+  ERR_WAIT_FULL = 0,
+  ERR_WAIT_EMPTY = 1,
+  ERR_NAN_SCALE = 2,
+};
+
+struct VExpert {  // one token group of one routed expert
+  int expert, start, count, pad;
+};
+
+struct Params {
+  int H, L, E, topk, I, Is;
+  int B;  // tokens of this forward
+  int score_fn, renorm;
+  float routed_scale;
+
+  // iteration space: virtual matrices x row blocks x pieces
+  int RB;             // row blocks per virtual matrix
+  int C;              // K chunks per row block
+  int PPR;            // pieces per row block (0: computed on the device, EGU/EDN)
+  int target_pieces;  // EGU/EDN: aim for at least this many pieces
+  int C_lat;          // TAIL: chunks covering L; chunks >= C_lat cover I_s
+  int RB_router;      // RL: row blocks holding router rows
+  int tg;             // tokens per group (EGU/EDN/TAIL)
+  int KL;             // K extent of the chunked dimension (for ragged last chunk)
+  int KS;             // TAIL: K extent of the shared part (I_s)
+
+  // shared memory geometry (bytes)
+  int nstages, stage_bytes, act_off, act_stride, scratch_off, stage_off;
+
+  const uint8_t* wt;       // packed tiles
+  long long matrix_bytes;  // EGU/EDN: bytes of one expert's tiles
+
+  const uint16_t* x;   // [B][H] bf16
+  const float* bias;   // [E] or null
+  float* logits;       // [maxB][E]
+  uint8_t* z_mx;       // [B][ceil(L/256)][544]
+  float* h_s;          // [ceil(Is/64)][B][64]
+  uint8_t* h_mx;       // [ceil(I/256)][B*k][544] in expert-sorted slot order
+  float* y;            // [ceil(L/64)][B*k][64]
+  uint16_t* out;       // [B][H] bf16
+  int ld_slots;        // B*k (row count of h_mx / y chunk planes)
+
+  int* ids;            // [B][k]
+  float* wts;          // [B][k]
+  int* slots_sorted;   // [B*k]
+  VExpert* ve;         // virtual experts
+  int* nve;
+  int ve_max;
+
+  Ctl* ctl;
+  int* counters;   // finalize tickets per (virtual matrix, row block)
+  int* router_done;
+  float* partials;
+  int* err;
+};
+
+// Host-side launcher (defined in moe_kernels.cu).
+int launch_kind(int kind, int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
+int max_smem_optin();
+int set_smem_limits(size_t bytes);
+
+int launch_pack_dense(const void* src, int K, int N, int layout, int RB, int C, int rows_valid,
+                      uint8_t* dst, void* stream, const void* src2, int K2, int C_first);
+int launch_pack_mx(const uint8_t* codes, const uint8_t* scales, int E, int rows, int K,
+                   int layout, int RB, int C, uint8_t* dst, int* err, void* stream);
+
+}  // namespace moe

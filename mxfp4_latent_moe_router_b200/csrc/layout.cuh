@@ -1,0 +1,56 @@
+// layout.cuh -- packed weight tiles and activation records of the B200 path.
+//
+// Every weight matrix is cut into row blocks of 128 output rows (8 warp tiles
+// of 16 rows) and, along K, into chunks; one (row block, chunk) tile is one
+// contiguous run of bytes that a single bulk copy moves into shared memory.
+// Inside a tile the elements sit in the order in which the lanes of an
+// m16n8k16 MMA hold them, so each lane fetches its A fragments with 16-byte
+// shared-memory loads and no shuffles.
+//
+// K permutation.  Within every 32-wide block of K, lane (g = lane/4, t =
+// lane%4) covers the 8 physical columns 8t..8t+7: k16 step 0 takes 8t+{0,1}
+// (fragment k 2t,2t+1) and 8t+{2,3} (fragment k 2t+8,2t+9), step 1 takes
+// 8t+{4,5} and 8t+{6,7}.  The same map is applied to the activations, which
+// therefore stay in natural row-major order: lane (g,t) reads 16 bytes of
+// token g at columns 32*blk + 8t .. +7.  Each MMA still sums over one 32-wide
+// block only, so MX block scales apply after every pair of k16 steps.
+#pragma once
+#include <cstdint>
+
+namespace moe {
+
+constexpr int kRowsPerBlock = 128;  // rows of one packed row block
+constexpr int kWarpRows = 16;       // rows of one warp tile
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+
+// bf16 tiles: 128 rows x 64 K = 16 KB.  Order: [warp 8][blk 2][step 2][lane 32][16 B]
+// with the 16 bytes = 4 A registers (a01 a23 a45 a67) of that k16 step.
+constexpr int kDenseChunkK = 64;
+constexpr int kDenseTileBytes = kRowsPerBlock * kDenseChunkK * 2;
+
+// MXFP4 tiles: 128 rows x 256 K.  Codes [warp 8][blk pair 4][lane 32][16 B]:
+// bytes 0..7 belong to the even block of the pair, 8..15 to the odd one, and
+// inside a block byte r (0..7) is A register r%4 of k16 step r/4 as an e2m1
+// pair (low nibble = lower k).  Scales follow: [warp 8][g 8][16 B] with bytes
+// 0..7 = row g, blocks 0..7 and bytes 8..15 = row g+8, blocks 0..7.
+constexpr int kMxChunkK = 256;
+constexpr int kMxCodeBytes = kRowsPerBlock * kMxChunkK / 2;  // 16384
+constexpr int kMxScaleBytes = kRowsPerBlock * kMxChunkK / 32;  // 1024
+constexpr int kMxTileBytes = kMxCodeBytes + kMxScaleBytes;    // 17408
+
+// Activation record for the MXFP4 kernels ("f16 MX"): per (row, 256-wide chunk)
+// 256 f16 values scaled by a power of two per 32-block, then the 8 float
+// scales that undo it.  544 bytes, 16-byte multiple.
+constexpr int kActRecBytes = kMxChunkK * 2 + 8 * 4;
+
+// fragment map: lane (g,t), k16 step s, register q (0..3), half e (0..1) ->
+// (row within the 16-row warp tile, physical k within the 32-block)
+__host__ __device__ constexpr int frag_row(int g, int q) { return (q & 1) ? g + 8 : g; }
+__host__ __device__ constexpr int frag_k(int t, int s, int q, int e) {
+  return 8 * t + 4 * s + ((q & 2) ? 2 : 0) + e;
+}
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace moe

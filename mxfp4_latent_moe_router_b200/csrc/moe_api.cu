@@ -1,0 +1,808 @@
+// moe_api.cu -- the C ABI declared in include/moe.h.
+//
+// A plan owns: packed weights, the per-forward workspace (activations, routing
+// tables, split-K partial sums, scheduling counters), a side stream and two
+// events.  moe_forward only enqueues work; all memory exists from
+// moe_plan_create on.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "engine.cuh"
+#include "layout.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kScratchOff = 1024;
+constexpr int kScratchBytes = 20480;
+constexpr int kStageOff = kScratchOff + kScratchBytes;
+constexpr int kHdr = 128;
+constexpr int kTailTg = 16;
+constexpr int kExpertTg = 32;
+constexpr int kBigSmem = 227 * 1024;
+constexpr int kSmallSmem = 113 * 1024;
+
+struct KindGeom {
+  int RB = 0, C = 0, KL = 0;
+  size_t tile_bytes = 0;
+  size_t weight_bytes = 0;  // packed (per expert for EGU/EDN)
+};
+
+struct DevBuf {
+  void* p = nullptr;
+  size_t n = 0;
+};
+
+}  // namespace
+
+struct moe_plan_s {
+  moe_config cfg{};
+  int device = 0;
+  int num_sms = 0;
+  bool loaded = false;
+  int last_B = 0;
+
+  KindGeom g[KIND_COUNT];
+  int RB_router = 0, C_lat = 0, tail_tg = kTailTg, ve_max = 0;
+
+  std::vector<void*> allocs;
+  size_t packed_bytes = 0, workspace_bytes = 0;
+
+  uint8_t* w_rl = nullptr;
+  uint8_t* w_sgu = nullptr;
+  uint8_t* w_egu = nullptr;
+  uint8_t* w_edn = nullptr;
+  uint8_t* w_tail = nullptr;
+  float* bias = nullptr;
+
+  float* logits = nullptr;
+  uint8_t* z_mx = nullptr;
+  float* h_s = nullptr;
+  uint8_t* h_mx = nullptr;
+  float* y = nullptr;
+  int* ids = nullptr;
+  float* wts = nullptr;
+  int* slots_sorted = nullptr;
+  VExpert* ve = nullptr;
+  int* nve = nullptr;
+  Ctl* ctl = nullptr;  // [KIND_COUNT]
+  int* counters[KIND_COUNT] = {};
+  int* router_done = nullptr;
+  float* partials[KIND_COUNT] = {};
+  size_t partial_cap[KIND_COUNT] = {};  // floats
+  int* err = nullptr;
+  uint16_t* x_stage = nullptr;
+  uint16_t* out_stage = nullptr;
+
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+
+  bool profiling = false;
+  cudaEvent_t ev_prof[KIND_COUNT][2] = {};
+  double prof_ms[KIND_COUNT] = {};
+  int prof_count = 0;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+int pow2_at_least(int v) {
+  int r = 1;
+  while (r < v) r <<= 1;
+  return r;
+}
+
+moe_status alloc(moe_plan p, void** out, size_t bytes, bool packed) {
+  void* d = nullptr;
+  if (bytes == 0) bytes = 16;
+  if (getenv("MOE_FAIL_ALLOC_AFTER")) {  // fault injection for the OOM path (host side only)
+    static int left = -1;
+    if (left < 0) left = atoi(getenv("MOE_FAIL_ALLOC_AFTER"));
+    if (left-- == 0) return MOE_ERR_OOM;
+  }
+  cudaError_t e = cudaMalloc(&d, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA;
+  }
+  p->allocs.push_back(d);
+  (packed ? p->packed_bytes : p->workspace_bytes) += bytes;
+  *out = d;
+  return MOE_OK;
+}
+
+bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
+
+// token geometry of one forward
+struct FwdGeom {
+  int nt_rl, nt_e, nt_tail, tail_tg;
+  int main_grid, side_grid, tail_grid;
+};
+
+FwdGeom fwd_geom(const moe_plan_s* p, int B) {
+  FwdGeom f;
+  f.nt_rl = pow2_at_least((B + 7) / 8);
+  f.nt_e = pow2_at_least((std::min(B, kExpertTg) + 7) / 8);
+  f.tail_tg = p->tail_tg;
+  f.nt_tail = pow2_at_least((std::min(B, p->tail_tg) + 7) / 8);
+  const moe_config& c = p->cfg;
+  int side = 0;
+  if (c.shared_inter > 0) {
+    if (c.shared_sms > 0) {
+      side = c.shared_sms;
+    } else {
+      // share the SMs in proportion to the bytes each stream has to move
+      const double E = c.num_experts, k = c.top_k;
+      const double distinct = E * (1.0 - std::pow(1.0 - k / E, (double)B));
+      const double sgu = 2.0 * c.hidden * 2.0 * c.shared_inter;
+      const double rl = 2.0 * c.hidden * (double)(c.num_experts + c.latent);
+      const double ex = distinct * (double)(p->g[KIND_EGU].weight_bytes + p->g[KIND_EDN].weight_bytes);
+      side = (int)std::lround(p->num_sms * sgu / (sgu + rl + ex));
+    }
+    side = std::max(4, std::min(side, p->num_sms / 2));
+  }
+  f.side_grid = side;
+  f.main_grid = p->num_sms - side;
+  f.tail_grid = p->num_sms;
+  return f;
+}
+
+struct SmemGeom {
+  int stage_bytes, nstages, act_off, act_stride;
+  size_t total;
+};
+
+SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk) {
+  SmemGeom s;
+  int act = 0;
+  s.act_stride = 0;
+  if (kind == KIND_RL || kind == KIND_SGU) {
+    s.act_stride = 192;
+    act = 8 * nt * s.act_stride;
+  } else if (kind == KIND_EGU || kind == KIND_EDN) {
+    s.act_stride = 576;
+    act = 8 * nt * s.act_stride;
+  } else {
+    act = tail_tg_eff * std::max(1, topk) * 256;
+  }
+  const int tile = (kind == KIND_EGU || kind == KIND_EDN) ? kMxTileBytes : kDenseTileBytes;
+  s.act_off = kHdr + tile;
+  s.stage_bytes = ((kHdr + tile + act) + 127) / 128 * 128;
+  const int budget = s.stage_bytes <= 24 * 1024 ? kSmallSmem : kBigSmem;
+  s.nstages = std::max(2, std::min(8, (budget - kStageOff) / s.stage_bytes));
+  s.total = (size_t)kStageOff + (size_t)s.nstages * s.stage_bytes;
+  return s;
+}
+
+int target_pieces(int grid, int nt) { return grid * std::max(2, 8 / nt); }
+
+Params base_params(const moe_plan_s* p, int B) {
+  Params q;
+  std::memset(&q, 0, sizeof(q));
+  const moe_config& c = p->cfg;
+  q.H = c.hidden;
+  q.L = c.latent;
+  q.E = c.num_experts;
+  q.topk = c.top_k;
+  q.I = c.expert_inter;
+  q.Is = c.shared_inter;
+  q.B = B;
+  q.score_fn = c.score_fn;
+  q.renorm = c.renormalize;
+  q.routed_scale = c.routed_scale;
+  q.bias = p->bias;
+  q.logits = p->logits;
+  q.z_mx = p->z_mx;
+  q.h_s = p->h_s;
+  q.h_mx = p->h_mx;
+  q.y = p->y;
+  q.ld_slots = B * c.top_k;
+  q.ids = p->ids;
+  q.wts = p->wts;
+  q.slots_sorted = p->slots_sorted;
+  q.ve = p->ve;
+  q.nve = p->nve;
+  q.ve_max = p->ve_max;
+  q.router_done = p->router_done;
+  q.err = p->err;
+  q.RB_router = p->RB_router;
+  q.C_lat = p->C_lat;
+  q.KS = c.shared_inter;
+  q.scratch_off = kScratchOff;
+  q.stage_off = kStageOff;
+  return q;
+}
+
+void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
+  q.RB = p->g[kind].RB;
+  q.C = p->g[kind].C;
+  q.KL = p->g[kind].KL;
+  q.ctl = p->ctl + kind;
+  q.counters = p->counters[kind];
+  q.partials = p->partials[kind];
+  q.nstages = s.nstages;
+  q.stage_bytes = s.stage_bytes;
+  q.act_off = s.act_off;
+  q.act_stride = s.act_stride;
+  q.matrix_bytes = (long long)p->g[kind].weight_bytes;
+  switch (kind) {
+    case KIND_RL: q.wt = p->w_rl; q.tg = kExpertTg; break;  // top-k groups expert tokens
+    case KIND_SGU: q.wt = p->w_sgu; break;
+    case KIND_EGU: q.wt = p->w_egu; q.tg = kExpertTg; break;
+    case KIND_EDN: q.wt = p->w_edn; q.tg = kExpertTg; break;
+    default: q.wt = p->w_tail; q.tg = p->tail_tg; break;
+  }
+}
+
+int ppr_for(int target, int rb, int C) {
+  int v = (target + rb - 1) / rb;
+  return std::max(1, std::min(C, v));
+}
+
+// largest number of partial-sum floats a kind can need for B <= maxB
+size_t partial_floats(const moe_plan_s* p, int kind) {
+  size_t best = 0;
+  for (int B = 1; B <= p->cfg.max_tokens; ++B) {
+    FwdGeom f = fwd_geom(p, B);
+    size_t pieces = 0;
+    int nt = 1;
+    const KindGeom& g = p->g[kind];
+    if (kind == KIND_RL) {
+      nt = f.nt_rl;
+      pieces = (size_t)g.RB * ppr_for(target_pieces(f.main_grid, nt), g.RB, g.C);
+    } else if (kind == KIND_SGU) {
+      nt = f.nt_rl;
+      if (!p->cfg.shared_inter) continue;
+      pieces = (size_t)g.RB * ppr_for(target_pieces(f.side_grid, nt), g.RB, g.C);
+    } else if (kind == KIND_TAIL) {
+      nt = f.nt_tail;
+      const int passes = (B + p->tail_tg - 1) / p->tail_tg;
+      pieces = (size_t)passes * g.RB * ppr_for(target_pieces(f.tail_grid, nt), g.RB * passes, g.C);
+    } else {
+      nt = f.nt_e;
+      // PPR > 1 only while (virtual experts x row blocks) < target, so the
+      // pieces that need partial storage stay below 2 x target
+      pieces = 2 * (size_t)target_pieces(f.main_grid, nt) + g.RB;
+    }
+    best = std::max(best, pieces * (size_t)nt * 1024);
+  }
+  return best;
+}
+
+#define TRY(x)                          \
+  do {                                  \
+    moe_status _s = (x);                \
+    if (_s != MOE_OK) return _s;        \
+  } while (0)
+#define CUDA_TRY(x)                      \
+  do {                                   \
+    if ((x) != cudaSuccess) {            \
+      cudaGetLastError();                \
+      return MOE_ERR_CUDA;               \
+    }                                    \
+  } while (0)
+
+moe_status check_cfg(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->latent <= 0 || c->num_experts <= 0 || c->expert_inter <= 0 ||
+      c->shared_inter < 0 || c->top_k <= 0 || c->max_tokens <= 0 || c->shared_sms < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->hidden % 32 || c->latent % 32 || c->expert_inter % 32 || c->shared_inter % 32)
+    return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->num_experts) return MOE_ERR_INVALID_ARG;
+  if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (!(c->routed_scale == c->routed_scale)) return MOE_ERR_INVALID_ARG;
+  if (c->num_experts > 1024 || c->top_k > 16 || c->max_tokens > 128) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
+  p->cfg = *cfg;
+  p->device = device;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return MOE_ERR_UNSUPPORTED;
+  }
+  cudaDeviceProp prop;
+  CUDA_TRY(cudaGetDeviceProperties(&prop, device));
+  if (prop.major != 10) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
+  p->num_sms = prop.multiProcessorCount;
+  if (set_smem_limits(kBigSmem) != 0) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+
+  const moe_config& c = *cfg;
+  const int H = c.hidden, L = c.latent, E = c.num_experts, I = c.expert_inter, Is = c.shared_inter;
+  p->RB_router = ceil_div(E, kRowsPerBlock);
+  KindGeom& rl = p->g[KIND_RL];
+  rl.RB = p->RB_router + ceil_div(L, kRowsPerBlock);
+  rl.C = ceil_div(H, kDenseChunkK);
+  rl.KL = H;
+  rl.weight_bytes = (size_t)rl.RB * rl.C * kDenseTileBytes;
+  KindGeom& sg = p->g[KIND_SGU];
+  sg.RB = ceil_div(Is, 64);
+  sg.C = ceil_div(H, kDenseChunkK);
+  sg.KL = H;
+  sg.weight_bytes = (size_t)sg.RB * sg.C * kDenseTileBytes;
+  KindGeom& eg = p->g[KIND_EGU];
+  eg.RB = ceil_div(I, 64);
+  eg.C = ceil_div(L, kMxChunkK);
+  eg.KL = L;
+  eg.weight_bytes = (size_t)eg.RB * eg.C * kMxTileBytes;
+  KindGeom& ed = p->g[KIND_EDN];
+  ed.RB = ceil_div(L, kRowsPerBlock);
+  ed.C = ceil_div(I, kMxChunkK);
+  ed.KL = I;
+  ed.weight_bytes = (size_t)ed.RB * ed.C * kMxTileBytes;
+  KindGeom& tl = p->g[KIND_TAIL];
+  p->C_lat = ceil_div(L, kDenseChunkK);
+  tl.RB = ceil_div(H, kRowsPerBlock);
+  tl.C = p->C_lat + ceil_div(Is, kDenseChunkK);
+  tl.KL = L;
+  tl.weight_bytes = (size_t)tl.RB * tl.C * kDenseTileBytes;
+  p->tail_tg = std::max(1, std::min(kTailTg, 128 / c.top_k));
+
+  const int maxB = c.max_tokens, K = c.top_k;
+  const int slots = maxB * K;
+  p->ve_max = std::min(E, slots) + ceil_div(slots, kExpertTg) + 1;
+
+  void* v;
+  TRY(alloc(p, &v, rl.weight_bytes, true));
+  p->w_rl = (uint8_t*)v;
+  if (Is > 0) {
+    TRY(alloc(p, &v, sg.weight_bytes, true));
+    p->w_sgu = (uint8_t*)v;
+  }
+  TRY(alloc(p, &v, (size_t)E * eg.weight_bytes, true));
+  p->w_egu = (uint8_t*)v;
+  TRY(alloc(p, &v, (size_t)E * ed.weight_bytes, true));
+  p->w_edn = (uint8_t*)v;
+  TRY(alloc(p, &v, tl.weight_bytes, true));
+  p->w_tail = (uint8_t*)v;
+  TRY(alloc(p, &v, sizeof(float) * E, true));
+  p->bias = (float*)v;
+
+  TRY(alloc(p, &v, sizeof(float) * maxB * E, false));
+  p->logits = (float*)v;
+  TRY(alloc(p, &v, (size_t)maxB * ceil_div(L, kMxChunkK) * kActRecBytes, false));
+  p->z_mx = (uint8_t*)v;
+  TRY(alloc(p, &v, sizeof(float) * (size_t)ceil_div(std::max(Is, 1), 64) * maxB * 64, false));
+  p->h_s = (float*)v;
+  TRY(alloc(p, &v, (size_t)ceil_div(I, kMxChunkK) * slots * kActRecBytes, false));
+  p->h_mx = (uint8_t*)v;
+  TRY(alloc(p, &v, sizeof(float) * (size_t)ceil_div(L, 64) * slots * 64, false));
+  p->y = (float*)v;
+  TRY(alloc(p, &v, sizeof(int) * slots, false));
+  p->ids = (int*)v;
+  TRY(alloc(p, &v, sizeof(float) * slots, false));
+  p->wts = (float*)v;
+  TRY(alloc(p, &v, sizeof(int) * slots, false));
+  p->slots_sorted = (int*)v;
+  TRY(alloc(p, &v, sizeof(VExpert) * p->ve_max, false));
+  p->ve = (VExpert*)v;
+  // small control block: nve, router_done, err, Ctl[KIND_COUNT]
+  TRY(alloc(p, &v, 1024 + sizeof(Ctl) * KIND_COUNT, false));
+  p->nve = (int*)v;
+  p->router_done = p->nve + 1;
+  p->err = p->nve + 2;
+  p->ctl = reinterpret_cast<Ctl*>((uint8_t*)v + 1024);
+  CUDA_TRY(cudaMemset(v, 0, 1024 + sizeof(Ctl) * KIND_COUNT));
+  const int cnt_n[KIND_COUNT] = {rl.RB, std::max(sg.RB, 1), p->ve_max * eg.RB, p->ve_max * ed.RB,
+                                 ceil_div(maxB, 1) * tl.RB};
+  for (int k = 0; k < KIND_COUNT; ++k) {
+    TRY(alloc(p, &v, sizeof(int) * cnt_n[k], false));
+    p->counters[k] = (int*)v;
+    CUDA_TRY(cudaMemset(v, 0, sizeof(int) * cnt_n[k]));
+    p->partial_cap[k] = partial_floats(p, k);
+    TRY(alloc(p, &v, sizeof(float) * std::max<size_t>(p->partial_cap[k], 4), false));
+    p->partials[k] = (float*)v;
+  }
+  TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
+  p->x_stage = (uint16_t*)v;
+  TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
+  p->out_stage = (uint16_t*)v;
+
+  CUDA_TRY(cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking));
+  CUDA_TRY(cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming));
+  CUDA_TRY(cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming));
+  for (int k = 0; k < KIND_COUNT; ++k)
+    for (int j = 0; j < 2; ++j) CUDA_TRY(cudaEventCreate(&p->ev_prof[k][j]));
+  CUDA_TRY(cudaDeviceSynchronize());
+  if (getenv("MOE_LOG")) {
+    fprintf(stderr,
+            "[moe] plan dev=%d sms=%d H=%d L=%d E=%d k=%d I=%d Is=%d maxB=%d packed=%.1fMB "
+            "workspace=%.1fMB\n",
+            device, p->num_sms, H, L, E, K, I, Is, maxB, p->packed_bytes / 1e6,
+            p->workspace_bytes / 1e6);
+  }
+  return MOE_OK;
+}
+
+void destroy_impl(moe_plan p) {
+  if (!p) return;
+  DeviceGuard g(p->device);
+  cudaDeviceSynchronize();
+  for (void* a : p->allocs) cudaFree(a);
+  if (p->side) cudaStreamDestroy(p->side);
+  if (p->ev_fork) cudaEventDestroy(p->ev_fork);
+  if (p->ev_join) cudaEventDestroy(p->ev_join);
+  for (int k = 0; k < KIND_COUNT; ++k)
+    for (int j = 0; j < 2; ++j)
+      if (p->ev_prof[k][j]) cudaEventDestroy(p->ev_prof[k][j]);
+  cudaGetLastError();
+  delete p;
+}
+
+moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStream_t s) {
+  const moe_config& c = p->cfg;
+  const FwdGeom f = fwd_geom(p, B);
+  const int tail_tg_eff = std::min(B, p->tail_tg);
+  const bool shared = c.shared_inter > 0;
+  Params base = base_params(p, B);
+  base.x = (const uint16_t*)x;
+  base.out = (uint16_t*)out;
+
+  if (shared) {
+    CUDA_TRY(cudaEventRecord(p->ev_fork, s));
+    CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_fork, 0));
+    Params q = base;
+    const SmemGeom sm = smem_geom(KIND_SGU, f.nt_rl, tail_tg_eff, c.top_k);
+    set_kind(q, p, KIND_SGU, sm);
+    q.PPR = ppr_for(target_pieces(f.side_grid, f.nt_rl), q.RB, q.C);
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_SGU][0], p->side));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_SGU, f.nt_rl, q, f.side_grid, sm.total, p->side, false));
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_SGU][1], p->side));
+    CUDA_TRY(cudaEventRecord(p->ev_join, p->side));
+  }
+  {
+    Params q = base;
+    const SmemGeom sm = smem_geom(KIND_RL, f.nt_rl, tail_tg_eff, c.top_k);
+    set_kind(q, p, KIND_RL, sm);
+    q.PPR = ppr_for(target_pieces(f.main_grid, f.nt_rl), q.RB, q.C);
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_RL][0], s));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_RL, f.nt_rl, q, f.main_grid, sm.total, s, true));
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_RL][1], s));
+  }
+  {
+    Params q = base;
+    const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k);
+    set_kind(q, p, KIND_EGU, sm);
+    q.target_pieces = target_pieces(f.main_grid, f.nt_e);
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][0], s));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.main_grid, sm.total, s, true));
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
+  }
+  {
+    Params q = base;
+    const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k);
+    set_kind(q, p, KIND_EDN, sm);
+    q.target_pieces = target_pieces(f.main_grid, f.nt_e);
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][0], s));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.main_grid, sm.total, s, true));
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
+  }
+  if (shared) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));
+  {
+    Params q = base;
+    const SmemGeom sm = smem_geom(KIND_TAIL, f.nt_tail, tail_tg_eff, c.top_k);
+    set_kind(q, p, KIND_TAIL, sm);
+    const int passes = (B + p->tail_tg - 1) / p->tail_tg;
+    q.PPR = ppr_for(target_pieces(f.tail_grid, f.nt_tail), q.RB * passes, q.C);
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, true));
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][1], s));
+  }
+  p->last_B = B;
+  if (p->profiling) {
+    for (int k = 0; k < KIND_COUNT; ++k) {
+      if (k == KIND_SGU && !shared) continue;
+      CUDA_TRY(cudaEventSynchronize(p->ev_prof[k][1]));
+      float ms = 0.f;
+      CUDA_TRY(cudaEventElapsedTime(&ms, p->ev_prof[k][0], p->ev_prof[k][1]));
+      p->prof_ms[k] += ms;
+    }
+    ++p->prof_count;
+  }
+  return MOE_OK;
+}
+
+float half_to_float(uint16_t h) {
+  const uint32_t sign = (h >> 15) & 1, ex = (h >> 10) & 0x1F, man = h & 0x3FF;
+  float v;
+  if (ex == 0)
+    v = std::ldexp((float)man, -24);
+  else if (ex == 31)
+    v = man ? NAN : INFINITY;
+  else
+    v = std::ldexp((float)(man | 0x400), (int)ex - 25);
+  return sign ? -v : v;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_str(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case MOE_ERR_NOT_LOADED: return "weights not loaded";
+    case MOE_ERR_OOM: return "out of memory";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_RANGE: return "weights hold a rejected encoding (e8m0 NaN)";
+  }
+  return "unknown status";
+}
+
+moe_status moe_plan_create(const moe_config* cfg, int device, moe_plan* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  moe_plan p = new (std::nothrow) moe_plan_s();
+  if (!p) return MOE_ERR_OOM;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    delete p;
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (device < 0 || device >= ndev) {
+    delete p;
+    return MOE_ERR_INVALID_ARG;
+  }
+  {
+    DeviceGuard g(device);
+    st = create_impl(cfg, device, p);
+  }
+  if (st != MOE_OK) {
+    destroy_impl(p);
+    return st;
+  }
+  *out = p;
+  return MOE_OK;
+}
+
+void moe_plan_destroy(moe_plan p) { destroy_impl(p); }
+
+moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
+  if (!p || !w) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = p->cfg;
+  const void* need[] = {w->router_w, w->w_in, w->w_out, w->gu_codes, w->gu_scales, w->dn_codes,
+                        w->dn_scales};
+  for (const void* q : need)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (c.shared_inter > 0) {
+    const void* sh[] = {w->sh_gate, w->sh_up, w->sh_down};
+    for (const void* q : sh)
+      if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  }
+  DeviceGuard g(p->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  p->loaded = false;
+  const int H = c.hidden, L = c.latent, E = c.num_experts, I = c.expert_inter, Is = c.shared_inter;
+  CUDA_TRY(cudaMemsetAsync(p->err, 0, sizeof(int), s));
+  // RL: router rows then latent rows, both from [H][N] tensors
+  const KindGeom& rl = p->g[KIND_RL];
+  CUDA_TRY((cudaError_t)launch_pack_dense(w->router_w, H, E, 0, p->RB_router, rl.C, E, p->w_rl, s,
+                                          nullptr, 0, 0));
+  CUDA_TRY((cudaError_t)launch_pack_dense(
+      w->w_in, H, L, 0, rl.RB - p->RB_router, rl.C, L,
+      p->w_rl + (size_t)p->RB_router * rl.C * kDenseTileBytes, s, nullptr, 0, 0));
+  if (Is > 0) {
+    const KindGeom& sg = p->g[KIND_SGU];
+    CUDA_TRY((cudaError_t)launch_pack_dense(w->sh_gate, H, Is, 1, sg.RB, sg.C, Is, p->w_sgu, s,
+                                            w->sh_up, 0, 0));
+  }
+  const KindGeom& tl = p->g[KIND_TAIL];
+  CUDA_TRY((cudaError_t)launch_pack_dense(w->w_out, L, H, 2, tl.RB, tl.C, H, p->w_tail, s,
+                                          Is > 0 ? w->sh_down : w->w_out, Is, p->C_lat));
+  const KindGeom& eg = p->g[KIND_EGU];
+  CUDA_TRY((cudaError_t)launch_pack_mx(w->gu_codes, w->gu_scales, E, 2 * I, L, 1, eg.RB, eg.C,
+                                       p->w_egu, p->err, s));
+  const KindGeom& ed = p->g[KIND_EDN];
+  CUDA_TRY((cudaError_t)launch_pack_mx(w->dn_codes, w->dn_scales, E, L, I, 0, ed.RB, ed.C,
+                                       p->w_edn, p->err, s));
+  if (w->router_bias && c.score_fn == MOE_SCORE_SIGMOID) {
+    if (!aligned16(w->router_bias)) return MOE_ERR_INVALID_ARG;
+    CUDA_TRY(cudaMemcpyAsync(p->bias, w->router_bias, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
+  } else {
+    CUDA_TRY(cudaMemsetAsync(p->bias, 0, sizeof(float) * E, s));
+  }
+  int err = 0;
+  CUDA_TRY(cudaMemcpyAsync(&err, p->err, sizeof(int), cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  if (err & (1 << ERR_NAN_SCALE)) {
+    CUDA_TRY(cudaMemset(p->err, 0, sizeof(int)));
+    return MOE_ERR_RANGE;
+  }
+  p->loaded = true;
+  return MOE_OK;
+}
+
+moe_status moe_forward(moe_plan p, const void* x, int32_t num_tokens, void* out, void* stream) {
+  if (!p || !x || !out) return MOE_ERR_INVALID_ARG;
+  if (num_tokens < 1 || num_tokens > p->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)num_tokens * p->cfg.hidden * 2;
+  const uint8_t* xa = (const uint8_t*)x;
+  const uint8_t* oa = (const uint8_t*)out;
+  if (xa < oa + bytes && oa < xa + bytes) return MOE_ERR_INVALID_ARG;
+  if (!p->loaded) return MOE_ERR_NOT_LOADED;
+  DeviceGuard g(p->device);
+  return enqueue_forward(p, x, num_tokens, out, (cudaStream_t)stream);
+}
+
+moe_status moe_forward_host(moe_plan p, const void* x_host, int32_t num_tokens, void* out_host,
+                            void* stream) {
+  if (!p || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if (num_tokens < 1 || num_tokens > p->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (!p->loaded) return MOE_ERR_NOT_LOADED;
+  DeviceGuard g(p->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t bytes = (size_t)num_tokens * p->cfg.hidden * 2;
+  CUDA_TRY(cudaMemcpyAsync(p->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s));
+  TRY(enqueue_forward(p, p->x_stage, num_tokens, p->out_stage, s));
+  CUDA_TRY(cudaMemcpyAsync(out_host, p->out_stage, bytes, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+moe_status moe_sync_status(moe_plan p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  int err = 0;
+  CUDA_TRY(cudaMemcpy(&err, p->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (err) {
+    CUDA_TRY(cudaMemset(p->err, 0, sizeof(int)));
+    if (err & ((1 << ERR_WAIT_FULL) | (1 << ERR_WAIT_EMPTY))) return MOE_ERR_TIMEOUT;
+    return MOE_ERR_RANGE;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_last_routing(moe_plan p, int32_t* ids_host, float* w_host, int32_t num_tokens) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (num_tokens < 1 || num_tokens > p->last_B) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  const size_t n = (size_t)num_tokens * p->cfg.top_k;
+  if (ids_host) CUDA_TRY(cudaMemcpy(ids_host, p->ids, n * sizeof(int), cudaMemcpyDeviceToHost));
+  if (w_host) CUDA_TRY(cudaMemcpy(w_host, p->wts, n * sizeof(float), cudaMemcpyDeviceToHost));
+  return MOE_OK;
+}
+
+moe_status moe_debug_fetch(moe_plan p, int32_t what, int32_t num_tokens, float* host,
+                           int64_t count) {
+  if (!p || !host) return MOE_ERR_INVALID_ARG;
+  const int B = p->last_B;
+  if (B < 1 || num_tokens != B) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = p->cfg;
+  const int L = c.latent, E = c.num_experts, K = c.top_k, I = c.expert_inter, Is = c.shared_inter;
+  DeviceGuard g(p->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  const int slots = B * K;
+  switch (what) {
+    case MOE_DBG_LOGITS: {
+      if (count != (int64_t)B * E) return MOE_ERR_INVALID_ARG;
+      CUDA_TRY(cudaMemcpy(host, p->logits, sizeof(float) * B * E, cudaMemcpyDeviceToHost));
+      return MOE_OK;
+    }
+    case MOE_DBG_Z: {
+      if (count != (int64_t)B * L) return MOE_ERR_INVALID_ARG;
+      const int cz = ceil_div(L, kMxChunkK);
+      std::vector<uint8_t> raw((size_t)B * cz * kActRecBytes);
+      CUDA_TRY(cudaMemcpy(raw.data(), p->z_mx, raw.size(), cudaMemcpyDeviceToHost));
+      for (int b = 0; b < B; ++b)
+        for (int l = 0; l < L; ++l) {
+          const uint8_t* rec = raw.data() + ((size_t)b * cz + l / kMxChunkK) * kActRecBytes;
+          uint16_t hv;
+          float sc;
+          std::memcpy(&hv, rec + (l % kMxChunkK) * 2, 2);
+          std::memcpy(&sc, rec + 512 + 4 * ((l % kMxChunkK) / 32), 4);
+          host[(size_t)b * L + l] = half_to_float(hv) * sc;
+        }
+      return MOE_OK;
+    }
+    case MOE_DBG_H: {
+      if (count != (int64_t)slots * I) return MOE_ERR_INVALID_ARG;
+      const int ci = ceil_div(I, kMxChunkK);
+      std::vector<uint8_t> raw((size_t)ci * slots * kActRecBytes);
+      std::vector<int> sorted(slots);
+      CUDA_TRY(cudaMemcpy(raw.data(), p->h_mx, raw.size(), cudaMemcpyDeviceToHost));
+      CUDA_TRY(cudaMemcpy(sorted.data(), p->slots_sorted, sizeof(int) * slots, cudaMemcpyDeviceToHost));
+      for (int pos = 0; pos < slots; ++pos) {
+        const int slot = sorted[pos];
+        if (slot < 0 || slot >= slots) return MOE_ERR_RANGE;
+        for (int i = 0; i < I; ++i) {
+          const uint8_t* rec = raw.data() + ((size_t)(i / kMxChunkK) * slots + pos) * kActRecBytes;
+          uint16_t hv;
+          float sc;
+          std::memcpy(&hv, rec + (i % kMxChunkK) * 2, 2);
+          std::memcpy(&sc, rec + 512 + 4 * ((i % kMxChunkK) / 32), 4);
+          host[(size_t)slot * I + i] = half_to_float(hv) * sc;
+        }
+      }
+      return MOE_OK;
+    }
+    case MOE_DBG_Y: {
+      if (count != (int64_t)slots * L) return MOE_ERR_INVALID_ARG;
+      const int cy = ceil_div(L, 64);
+      std::vector<float> raw((size_t)cy * slots * 64);
+      CUDA_TRY(cudaMemcpy(raw.data(), p->y, raw.size() * sizeof(float), cudaMemcpyDeviceToHost));
+      for (int s = 0; s < slots; ++s)
+        for (int l = 0; l < L; ++l) host[(size_t)s * L + l] = raw[((size_t)(l / 64) * slots + s) * 64 + l % 64];
+      return MOE_OK;
+    }
+    case MOE_DBG_HS: {
+      if (Is == 0 || count != (int64_t)B * Is) return MOE_ERR_INVALID_ARG;
+      const int cs = ceil_div(Is, 64);
+      std::vector<float> raw((size_t)cs * B * 64);
+      CUDA_TRY(cudaMemcpy(raw.data(), p->h_s, raw.size() * sizeof(float), cudaMemcpyDeviceToHost));
+      for (int b = 0; b < B; ++b)
+        for (int i = 0; i < Is; ++i) host[(size_t)b * Is + i] = raw[((size_t)(i / 64) * B + b) * 64 + i % 64];
+      return MOE_OK;
+    }
+    default: return MOE_ERR_INVALID_ARG;
+  }
+}
+
+moe_status moe_get_plan_info(moe_plan p, moe_plan_info* info) {
+  if (!p || !info) return MOE_ERR_INVALID_ARG;
+  const FwdGeom f = fwd_geom(p, p->cfg.max_tokens);
+  info->device = p->device;
+  info->num_sms = p->num_sms;
+  info->main_ctas = f.main_grid;
+  info->shared_ctas = f.side_grid;
+  info->packed_bytes = (int64_t)p->packed_bytes;
+  info->workspace_bytes = (int64_t)p->workspace_bytes;
+  const moe_config& c = p->cfg;
+  info->dense_weight_bytes =
+      2LL * c.hidden * (c.num_experts + c.latent) + 2LL * c.latent * c.hidden +
+      6LL * c.hidden * c.shared_inter;
+  info->expert_weight_bytes =
+      (3LL * c.expert_inter * c.latent) / 2 + (3LL * c.expert_inter * c.latent) / 32;
+  info->kernels_per_forward = c.shared_inter > 0 ? 5 : 4;
+  return MOE_OK;
+}
+
+moe_status moe_set_profiling(moe_plan p, int32_t enable) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  p->profiling = enable != 0;
+  return MOE_OK;
+}
+
+moe_status moe_get_profile(moe_plan p, float* ms, int32_t* count) {
+  if (!p || !ms || !count) return MOE_ERR_INVALID_ARG;
+  for (int k = 0; k < KIND_COUNT; ++k) {
+    ms[k] = (float)p->prof_ms[k];
+    p->prof_ms[k] = 0.0;
+  }
+  *count = p->prof_count;
+  p->prof_count = 0;
+  return MOE_OK;
+}
+
+}  // extern "C"

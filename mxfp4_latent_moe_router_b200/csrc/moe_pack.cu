@@ -1,0 +1,168 @@
+// moe_pack.cu -- one-time repacking of canonical weights into MMA-fragment tiles.
+//
+// Canonical inputs (see include/moe.h): bf16 tensors in "x . W" orientation
+// [K][N]; MXFP4 tensors output-row-major [rows][K/2] codes + [rows][K/32]
+// e8m0 scales.  Outputs are the tile layouts described in layout.cuh.
+#include <cuda_runtime.h>
+
+#include "engine.cuh"
+#include "layout.cuh"
+
+namespace moe {
+
+// dense layouts
+enum : int { DENSE_PLAIN = 0, DENSE_GATE_UP = 1, DENSE_TWO_K = 2 };
+// MXFP4 layouts
+enum : int { MX_PLAIN = 0, MX_GATE_UP = 1 };
+
+__global__ void pack_dense_kernel(const uint16_t* __restrict__ src, int K, int N, int layout,
+                                  int RB, int C, uint8_t* __restrict__ dst,
+                                  const uint16_t* __restrict__ src2, int K2, int C_first) {
+  const long long units = (long long)RB * C * 1024;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const int lane = u & 31, s = (u >> 5) & 1, b = (u >> 6) & 1, w = (u >> 7) & 7;
+    const long long tile = u >> 10;
+    const int rb = (int)(tile / C), c = (int)(tile % C);
+    const int g = lane >> 2, t = lane & 3;
+    uint16_t v[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = frag_row(g, q);  // row within the warp tile
+        const int kk = 32 * b + frag_k(t, s, q, e);
+        const uint16_t* m = src;
+        int col = -1, k = -1, kmax = K;
+        if (layout == DENSE_PLAIN) {
+          col = rb * kRowsPerBlock + 16 * w + r;
+          k = c * kDenseChunkK + kk;
+        } else if (layout == DENSE_GATE_UP) {
+          col = 64 * rb + 8 * w + (r & 7);
+          if (r >= 8) m = src2;
+          k = c * kDenseChunkK + kk;
+        } else {  // DENSE_TWO_K: rows = output columns n, K = [src rows ; src2 rows]
+          col = rb * kRowsPerBlock + 16 * w + r;
+          if (c < C_first) {
+            k = c * kDenseChunkK + kk;
+          } else {
+            m = src2;
+            kmax = K2;
+            k = (c - C_first) * kDenseChunkK + kk;
+          }
+        }
+        uint16_t val = 0;
+        if (col < N && k < kmax) val = m[(long long)k * N + col];
+        v[2 * q + e] = val;
+      }
+    }
+    uint4 o;
+    o.x = v[0] | ((uint32_t)v[1] << 16);
+    o.y = v[2] | ((uint32_t)v[3] << 16);
+    o.z = v[4] | ((uint32_t)v[5] << 16);
+    o.w = v[6] | ((uint32_t)v[7] << 16);
+    // [warp][blk][step][lane][16 B]
+    uint8_t* d = dst + tile * kDenseTileBytes + (((w * 2 + b) * 2 + s) * 32 + lane) * 16;
+    *reinterpret_cast<uint4*>(d) = o;
+  }
+}
+
+__device__ __forceinline__ int mx_src_row(int layout, int rb, int row_in_block, int rows_half,
+                                          int rows, bool& valid) {
+  if (layout == MX_GATE_UP) {
+    const int w = row_in_block >> 4, r = row_in_block & 15;
+    const int h = 64 * rb + 8 * w + (r & 7);  // SwiGLU output index
+    valid = h < rows_half;
+    return (r < 8) ? h : rows_half + h;
+  }
+  const int row = rb * kRowsPerBlock + row_in_block;
+  valid = row < rows;
+  return row;
+}
+
+__global__ void pack_mx_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                               int E, int rows, int K, int layout, int RB, int C,
+                               uint8_t* __restrict__ dst, int* err) {
+  const int rows_half = rows / 2;  // gate/up: I
+  const long long per_tile = 1024 + 64;
+  const long long units = (long long)E * RB * C * per_tile;
+  const int kb_total = K / 32;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const long long tile = u / per_tile;
+    const int v = (int)(u % per_tile);
+    const int e = (int)(tile / ((long long)RB * C));
+    const int rem = (int)(tile % ((long long)RB * C));
+    const int rb = rem / C, c = rem % C;
+    const uint8_t* ce = codes + (long long)e * rows * (K / 2);
+    const uint8_t* se = scales + (long long)e * rows * kb_total;
+    uint8_t* tdst = dst + tile * kMxTileBytes;
+    uint8_t out[16];
+    if (v < 1024) {
+      const int lane = v & 31, bp = (v >> 5) & 3, w = v >> 7;
+      const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int b = 2 * bp + (j >> 3), r = j & 7, s = r >> 2, q = r & 3;
+        const int row_in_block = 16 * w + frag_row(g, q);
+        const int k0 = c * kMxChunkK + 32 * b + frag_k(t, s, q, 0);  // even
+        bool valid;
+        const int sr = mx_src_row(layout, rb, row_in_block, rows_half, rows, valid);
+        out[j] = (valid && k0 < K) ? ce[(long long)sr * (K / 2) + k0 / 2] : 0;
+      }
+      uint4 o;
+      o.x = out[0] | (out[1] << 8) | (out[2] << 16) | ((uint32_t)out[3] << 24);
+      o.y = out[4] | (out[5] << 8) | (out[6] << 16) | ((uint32_t)out[7] << 24);
+      o.z = out[8] | (out[9] << 8) | (out[10] << 16) | ((uint32_t)out[11] << 24);
+      o.w = out[12] | (out[13] << 8) | (out[14] << 16) | ((uint32_t)out[15] << 24);
+      *reinterpret_cast<uint4*>(tdst + (w * 4 + bp) * 512 + lane * 16) = o;
+    } else {
+      const int idx = v - 1024, w = idx >> 3, g = idx & 7;
+      int bad = 0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int row_in_block = 16 * w + g + ((j >= 8) ? 8 : 0);
+        const int blk = c * 8 + (j & 7);
+        bool valid;
+        const int sr = mx_src_row(layout, rb, row_in_block, rows_half, rows, valid);
+        uint8_t sv = 127;
+        if (valid && blk < kb_total) {
+          sv = se[(long long)sr * kb_total + blk];
+          if (sv == 0xFF) bad = 1;
+        }
+        out[j] = sv;
+      }
+      if (bad) atomicOr(err, 1 << ERR_NAN_SCALE);
+      uint4 o;
+      o.x = out[0] | (out[1] << 8) | (out[2] << 16) | ((uint32_t)out[3] << 24);
+      o.y = out[4] | (out[5] << 8) | (out[6] << 16) | ((uint32_t)out[7] << 24);
+      o.z = out[8] | (out[9] << 8) | (out[10] << 16) | ((uint32_t)out[11] << 24);
+      o.w = out[12] | (out[13] << 8) | (out[14] << 16) | ((uint32_t)out[15] << 24);
+      *reinterpret_cast<uint4*>(tdst + kMxCodeBytes + (w * 8 + g) * 16) = o;
+    }
+  }
+}
+
+int launch_pack_dense(const void* src, int K, int N, int layout, int RB, int C, int /*rows_valid*/,
+                      uint8_t* dst, void* stream, const void* src2, int K2, int C_first) {
+  const long long units = (long long)RB * C * 1024;
+  const int threads = 256;
+  const int blocks = (int)((units + threads - 1) / threads < 65535 * 8 ? (units + threads - 1) / threads
+                                                                         : 65535 * 8);
+  pack_dense_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
+      (const uint16_t*)src, K, N, layout, RB, C, dst, (const uint16_t*)src2, K2, C_first);
+  return (int)cudaGetLastError();
+}
+
+int launch_pack_mx(const uint8_t* codes, const uint8_t* scales, int E, int rows, int K, int layout,
+                   int RB, int C, uint8_t* dst, int* err, void* stream) {
+  const long long units = (long long)E * RB * C * (1024 + 64);
+  const int threads = 256;
+  long long nb = (units + threads - 1) / threads;
+  if (nb > 65535LL * 16) nb = 65535LL * 16;
+  pack_mx_kernel<<<(int)nb, threads, 0, (cudaStream_t)stream>>>(codes, scales, E, rows, K, layout,
+                                                                 RB, C, dst, err);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,259 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Each step of the block is checked on its own (router logits and top-k, latent
+z, expert SwiGLU h, expert outputs y, shared-expert h_s) and the block output
+against the oracle's fp64 result: top-k ids exact (up to reported near ties),
+combine weights to 1e-5, floating outputs within max-rel 2e-2 / mean-rel 2e-3.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import mxfp4_latent_moe_router_b200 as moe  # noqa: E402
+from mxfp4_latent_moe_router_b200 import synth  # noqa: E402
+from helpers import assert_close, bf16_to_f32, check_routing  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+class GpuBlock:
+    def __init__(self, shape, w, max_tokens, shared_sms=0):
+        self.shape = shape
+        self.w = w
+        self.plan = moe.MoePlan(moe.config_from_shape(shape, max_tokens=max_tokens,
+                                                      shared_sms=shared_sms))
+        self.dev_w = moe.weights_to_device(w)
+        self.plan.load(self.dev_w)
+        torch.cuda.synchronize()
+
+    def run(self, x_bits: np.ndarray):
+        x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+        out = torch.empty_like(x)
+        self.plan.forward(x, out)
+        torch.cuda.synchronize()
+        assert self.plan.sync_status() == 0
+        return out.cpu().numpy().view(np.uint16)
+
+    def fetch_all(self, B):
+        r = {"logits": self.plan.fetch(moe.MOE_DBG_LOGITS, B),
+             "z": self.plan.fetch(moe.MOE_DBG_Z, B),
+             "h": self.plan.fetch(moe.MOE_DBG_H, B),
+             "y": self.plan.fetch(moe.MOE_DBG_Y, B)}
+        if self.shape.shared_inter:
+            r["h_s"] = self.plan.fetch(moe.MOE_DBG_HS, B)
+        r["ids"], r["w"] = self.plan.routing(B)
+        return r
+
+
+def _slot_order(gpu_ids, orc_ids):
+    """Map GPU slot j of token b to the oracle's slot of the same expert."""
+    perm = np.zeros_like(gpu_ids)
+    for b in range(gpu_ids.shape[0]):
+        pos = {e: j for j, e in enumerate(orc_ids[b].tolist())}
+        perm[b] = [pos.get(e, -1) for e in gpu_ids[b].tolist()]
+    return perm
+
+
+def full_check(blk: GpuBlock, x, tokens=None, intermediates=True):
+    shape, w = blk.shape, blk.w
+    out = blk.run(x)
+    B = x.shape[0]
+    sel = np.arange(B) if tokens is None else np.asarray(tokens)
+    orc = oracle.forward(shape, w, x[sel], intermediates=intermediates)
+    g = blk.fetch_all(B)
+    near = check_routing(shape, w, x[sel], g["ids"][sel], g["w"][sel], g["logits"][sel], orc)
+    if intermediates:
+        assert_close(g["z"][sel], orc["z"], "z (latent)")
+        if shape.shared_inter:
+            assert_close(g["h_s"][sel], orc["h_s"], "h_s (shared SwiGLU)")
+        ok = [i for i, b in enumerate(sel) if b not in near]
+        perm = _slot_order(g["ids"][sel], orc["ids"])
+        for i in ok:
+            hg = g["h"][sel[i]]
+            yg = g["y"][sel[i]]
+            ho = orc["h"][i][perm[i]]
+            yo = orc["y"][i][perm[i]]
+            assert_close(hg, ho, "h (expert SwiGLU) token %d" % sel[i])
+            assert_close(yg, yo, "y (expert out) token %d" % sel[i])
+    ok_rows = [i for i, b in enumerate(sel) if b not in near]
+    res = assert_close(bf16_to_f32(out[sel][ok_rows]), orc["out"][ok_rows], "out")
+    return out, res, near
+
+
+# ---------------------------------------------------------------------------
+# small shapes: several tiles, ragged tails, every branch
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    shape = synth.SHAPES["tiny"]
+    return shape, synth.make_weights(shape)
+
+
+def test_tiny_single_token(tiny):
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=1)
+    full_check(blk, synth.make_x(shape))
+
+
+@pytest.mark.parametrize("B", [2, 13, 16])
+def test_tiny_ragged_batches(tiny, B):
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=16)
+    full_check(blk, synth.make_x(shape, tokens=B, step=B))
+
+
+@pytest.mark.parametrize("score_fn,k,Is", [(synth.SCORE_SIGMOID, 3, 32), (synth.SCORE_SOFTMAX, 1, 64),
+                                           (synth.SCORE_SIGMOID, 4, 0)])
+def test_ragged_shapes(score_fn, k, Is):
+    # H=96 (dense chunks 64+32), L=96 and I=96 (MXFP4 chunks of 3 blocks), E=10
+    # (router rows padded), I_s=32 or none
+    shape = synth.custom_shape("ragged", 5, 96, 96, 10, k, 96, Is, score_fn, seed=21 + k,
+                               scale_exp_lo=-5, scale_exp_hi=-2)
+    w = synth.make_weights(shape)
+    blk = GpuBlock(shape, w, max_tokens=40)
+    full_check(blk, synth.make_x(shape))
+    full_check(blk, synth.make_x(shape, tokens=37, step=3))
+
+
+def test_zero_input_gives_exact_zero(tiny):
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=4)
+    x = np.zeros((3, shape.hidden), np.uint16)
+    out = blk.run(x)
+    assert np.all(out == 0)
+    ids, wts = blk.plan.routing(3)
+    assert ids.tolist() == [[0, 1]] * 3
+    np.testing.assert_allclose(wts, 0.5, rtol=0, atol=1e-7)
+
+
+def test_back_to_back_forwards_read_their_own_inputs(tiny):
+    """Two forwards on one stream with different x: a read hoisted above a
+    dependency wait would pick up the other step's activations."""
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=8)
+    xa = synth.make_x(shape, tokens=8, step=100)
+    xb = synth.make_x(shape, tokens=8, step=101)
+    ta = torch.from_numpy(xa.view(np.int16)).cuda()
+    tb = torch.from_numpy(xb.view(np.int16)).cuda()
+    oa, ob = torch.empty_like(ta), torch.empty_like(tb)
+    for _ in range(3):
+        blk.plan.forward(ta, oa)
+        blk.plan.forward(tb, ob)
+    torch.cuda.synchronize()
+    for x, o in ((xa, oa), (xb, ob)):
+        ref = oracle.forward(shape, w, x, intermediates=False)
+        assert_close(bf16_to_f32(o.cpu().numpy().view(np.uint16)), ref["out"], "out")
+
+
+def test_deterministic_and_graph_replay(tiny):
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=8)
+    x = torch.from_numpy(synth.make_x(shape, tokens=8, step=7).view(np.int16)).cuda()
+    o1, o2, o3 = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+    blk.plan.forward(x, o1)
+    blk.plan.forward(x, o2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        blk.plan.forward(x, o3, stream=s)  # warm-up outside capture
+        s.synchronize()
+        o3.zero_()
+        with torch.cuda.graph(g, stream=s):
+            blk.plan.forward(x, o3, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o3)
+
+
+def test_host_buffer_entry_point(tiny):
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=4)
+    x = synth.make_x(shape, tokens=4, step=9)
+    dev = blk.run(x)
+    xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    blk.plan.forward_host(xh, oh)
+    torch.cuda.synchronize()
+    assert np.array_equal(oh.numpy().view(np.uint16), dev)
+
+
+def test_argument_errors(tiny):
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=4)
+    x = torch.zeros((4, shape.hidden), dtype=torch.int16, device="cuda")
+    out = torch.empty_like(x)
+    h = blk.plan.handle
+    assert moe.moe_forward(h, x, 0, out) == 1
+    assert moe.moe_forward(h, x, 5, out) == 1
+    assert moe.moe_forward(h, x, 4, x) == 1                      # aliasing
+    xb = torch.zeros(4 * shape.hidden + 8, dtype=torch.int16, device="cuda")
+    assert moe.moe_forward(h, xb[1:], 4, out) == 1               # misaligned
+    fresh = moe.MoePlan(moe.config_from_shape(shape, max_tokens=4))
+    assert moe.moe_forward(fresh.handle, x, 4, out) == 3         # not loaded
+    bad = dict(w)
+    bad["gu_scales"] = w["gu_scales"].copy()
+    bad["gu_scales"][3, 5, 1] = 0xFF
+    with pytest.raises(moe.MoeError) as ei:
+        fresh.load(moe.weights_to_device(bad))
+    assert ei.value.status == 7
+    assert moe.moe_forward(fresh.handle, x, 4, out) == 3
+
+
+# ---------------------------------------------------------------------------
+# full-size decode shapes (H=7168, L=2048, E=384, k=8, I=2048, I_s=2048)
+
+
+@pytest.fixture(scope="module")
+def full_weights():
+    shape = synth.SHAPES["b1"]
+    return synth.make_weights(shape)
+
+
+@pytest.fixture(scope="module")
+def full_block(full_weights):
+    shape = synth.SHAPES["b1"]
+    blk = GpuBlock(shape, full_weights, max_tokens=128)
+    yield blk
+    blk.plan.close()
+
+
+def test_b1_full_size(full_block):
+    shape = synth.SHAPES["b1"]
+    _, (mx, mn), near = full_check(full_block, synth.make_x(shape))
+    print("b1: max_rel %.3g mean_rel %.3g near-ties %s" % (mx, mn, near))
+
+
+@pytest.mark.parametrize("name,sample", [("b8", None), ("b64", [0, 9, 31, 63]),
+                                         ("b128", [0, 5, 64, 127])])
+def test_batched_full_size(full_block, full_weights, name, sample):
+    shape = synth.SHAPES[name]
+    w = full_weights
+    if shape.routing == "zipf":
+        # the speculative-verify shape: skewed popularity through the bias
+        w = dict(full_weights)
+        w["router_bias"] = synth.make_weights(synth.custom_shape(
+            "bias-only", 1, 32, 32, shape.num_experts, 1, 32, 0, synth.SCORE_SIGMOID,
+            routing="zipf", seed=shape.seed))["router_bias"]
+        blk = GpuBlock(shape, w, max_tokens=128)
+    else:
+        blk = full_block
+    x = synth.make_x(shape)
+    out = blk.run(x)
+    # routing of every token, with the cheap router-only oracle
+    r = oracle.route(shape, w, x)
+    ids, wts = blk.plan.routing(x.shape[0])
+    logits = blk.plan.fetch(moe.MOE_DBG_LOGITS, x.shape[0])
+    near = check_routing(shape, w, x, ids, wts, logits, r)
+    # whole block on sampled tokens
+    sel = np.arange(x.shape[0]) if sample is None else np.array(sample)
+    sel = np.array([b for b in sel if b not in near])
+    orc = oracle.forward(shape, w, x[sel], intermediates=False)
+    assert_close(bf16_to_f32(out[sel]), orc["out"], name + " out")
+    distinct = len(np.unique(ids))
+    print("%s: distinct experts %d, near ties %s" % (name, distinct, near))
