@@ -36,7 +36,6 @@ sys.path.insert(0, ROOT)
 
 METRIC = "latent-MoE layer µs/step and weight-stream GB/s vs HBM peak, B=1–64"
 UNIT = "us/step"
-INSTANCES = 4
 INPUT_POOL = 4
 
 
@@ -54,6 +53,18 @@ def _workload_desc(shape):
             % (shape.name, shape.tokens, shape.hidden, shape.latent, shape.num_experts, shape.top_k,
                "softmax" if shape.score_fn == 0 else "sigmoid+bias", shape.expert_inter,
                shape.shared_inter))
+
+
+def max_over_ranks(v: float) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return v
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def _dist():
@@ -225,6 +236,7 @@ def run_ours(args):
 
     shape = synth.SHAPES[args.workload]
     B = shape.tokens
+    INSTANCES = args.instances
     stream = torch.cuda.Stream()
     plans, host_w0 = [], None
     for inst in range(INSTANCES):
@@ -285,11 +297,7 @@ def run_ours(args):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    ms_total = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
     us_step = ms_total * 1e3 / args.steps
     del g
 
@@ -357,11 +365,7 @@ def run_ours(args):
             plans[k % INSTANCES].forward_host(xh[k % INPUT_POOL], oh[k % INPUT_POOL], stream=stream)
         f1.record(stream)
     stream.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
     e2e_us = e2e_ms * 1e3 / args.steps
 
     # CPU oracle baseline (rank 0, one GPU only)
@@ -417,6 +421,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="b1", choices=["tiny", "b1", "b8", "b64", "b128"])
     ap.add_argument("--shared-sms", type=int, default=0)
+    ap.add_argument("--instances", type=int, default=4,
+                    help="resident weight instances rotated per step (4 keeps every step out of L2)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     args = ap.parse_args()

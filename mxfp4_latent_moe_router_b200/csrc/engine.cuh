@@ -53,6 +53,7 @@ struct Params {
 
   // shared memory geometry (bytes)
   int nstages, stage_bytes, act_off, act_stride, scratch_off, stage_off;
+  int table_off;  // EGU/EDN: shared-memory copy of the routing tables
 
   const uint8_t* wt;       // packed tiles
   long long matrix_bytes;  // EGU/EDN: bytes of one expert's tiles

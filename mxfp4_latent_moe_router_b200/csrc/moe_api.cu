@@ -85,6 +85,12 @@ struct moe_plan_s {
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 
+  // tuning knobs read once at plan creation (environment): pieces each CTA
+  // should get on average, and whether kernels chain with programmatic
+  // dependent launch
+  int pieces_per_cta = 8;
+  bool use_pdl = true;
+
   bool profiling = false;
   cudaEvent_t ev_prof[KIND_COUNT][2] = {};
   double prof_ms[KIND_COUNT] = {};
@@ -166,12 +172,17 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
 }
 
 struct SmemGeom {
-  int stage_bytes, nstages, act_off, act_stride;
+  int stage_bytes, nstages, act_off, act_stride, table_bytes, stage_off;
   size_t total;
 };
 
-SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk) {
+SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int slots) {
   SmemGeom s;
+  // routing tables (virtual experts + expert-sorted slots) for the expert kernels
+  s.table_bytes = 0;
+  if (kind == KIND_EGU || kind == KIND_EDN)
+    s.table_bytes = ((ve_max * (int)sizeof(VExpert) + slots * 4) + 127) / 128 * 128;
+  const int stage_off = kStageOff + s.table_bytes;
   int act = 0;
   s.act_stride = 0;
   if (kind == KIND_RL || kind == KIND_SGU) {
@@ -187,12 +198,14 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk) {
   s.act_off = kHdr + tile;
   s.stage_bytes = ((kHdr + tile + act) + 127) / 128 * 128;
   const int budget = s.stage_bytes <= 24 * 1024 ? kSmallSmem : kBigSmem;
-  s.nstages = std::max(2, std::min(8, (budget - kStageOff) / s.stage_bytes));
-  s.total = (size_t)kStageOff + (size_t)s.nstages * s.stage_bytes;
+  s.nstages = std::max(2, std::min(8, (budget - stage_off) / s.stage_bytes));
+  s.stage_off = stage_off;
+  s.total = (size_t)stage_off + (size_t)s.nstages * s.stage_bytes;
   return s;
 }
 
-int target_pieces(int grid, int nt) { return grid * std::max(2, 8 / nt); }
+int g_pieces_per_cta = 8;  // set from the plan before any geometry call
+int target_pieces(int grid, int nt) { return grid * std::max(1, g_pieces_per_cta / nt); }
 
 Params base_params(const moe_plan_s* p, int B) {
   Params q;
@@ -227,7 +240,6 @@ Params base_params(const moe_plan_s* p, int B) {
   q.C_lat = p->C_lat;
   q.KS = c.shared_inter;
   q.scratch_off = kScratchOff;
-  q.stage_off = kStageOff;
   return q;
 }
 
@@ -242,6 +254,8 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   q.stage_bytes = s.stage_bytes;
   q.act_off = s.act_off;
   q.act_stride = s.act_stride;
+  q.table_off = kStageOff;
+  q.stage_off = s.stage_off;
   q.matrix_bytes = (long long)p->g[kind].weight_bytes;
   switch (kind) {
     case KIND_RL: q.wt = p->w_rl; q.tg = kExpertTg; break;  // top-k groups expert tokens
@@ -326,6 +340,9 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   CUDA_TRY(cudaGetDeviceProperties(&prop, device));
   if (prop.major != 10) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
   p->num_sms = prop.multiProcessorCount;
+  if (const char* e = getenv("MOE_PIECES_PER_CTA")) p->pieces_per_cta = std::max(1, atoi(e));
+  if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
+  g_pieces_per_cta = p->pieces_per_cta;
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -455,6 +472,7 @@ void destroy_impl(moe_plan p) {
 
 moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStream_t s) {
   const moe_config& c = p->cfg;
+  g_pieces_per_cta = p->pieces_per_cta;
   const FwdGeom f = fwd_geom(p, B);
   const int tail_tg_eff = std::min(B, p->tail_tg);
   const bool shared = c.shared_inter > 0;
@@ -466,7 +484,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     CUDA_TRY(cudaEventRecord(p->ev_fork, s));
     CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_fork, 0));
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_SGU, f.nt_rl, tail_tg_eff, c.top_k);
+    const SmemGeom sm = smem_geom(KIND_SGU, f.nt_rl, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_SGU, sm);
     q.PPR = ppr_for(target_pieces(f.side_grid, f.nt_rl), q.RB, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_SGU][0], p->side));
@@ -476,40 +494,40 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_RL, f.nt_rl, tail_tg_eff, c.top_k);
+    const SmemGeom sm = smem_geom(KIND_RL, f.nt_rl, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_RL, sm);
     q.PPR = ppr_for(target_pieces(f.main_grid, f.nt_rl), q.RB, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_RL][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_RL, f.nt_rl, q, f.main_grid, sm.total, s, true));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_RL, f.nt_rl, q, f.main_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_RL][1], s));
   }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k);
+    const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EGU, sm);
     q.target_pieces = target_pieces(f.main_grid, f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.main_grid, sm.total, s, true));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.main_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
   }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k);
+    const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EDN, sm);
     q.target_pieces = target_pieces(f.main_grid, f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.main_grid, sm.total, s, true));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.main_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
   }
   if (shared) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_TAIL, f.nt_tail, tail_tg_eff, c.top_k);
+    const SmemGeom sm = smem_geom(KIND_TAIL, f.nt_tail, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_TAIL, sm);
     const int passes = (B + p->tail_tg - 1) / p->tail_tg;
     q.PPR = ppr_for(target_pieces(f.tail_grid, f.nt_tail), q.RB * passes, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, true));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][1], s));
   }
   p->last_B = B;

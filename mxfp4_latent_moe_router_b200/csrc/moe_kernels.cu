@@ -128,7 +128,8 @@ __device__ __forceinline__ int chunk_blocks(const Params& p, int c) {
 
 template <int KIND>
 __device__ __forceinline__ void fill_header(const Params& p, const Space& sp, int piece, int c,
-                                            int c_first, int c_last, Hdr& h) {
+                                            int c_first, int c_last, Hdr& h,
+                                            const VExpert* ve_tab) {
   const int per_v = p.RB * sp.ppr;
   const int v = piece / per_v;
   const int rem = piece - v * per_v;
@@ -148,7 +149,7 @@ __device__ __forceinline__ void fill_header(const Params& p, const Space& sp, in
     h.tok0 = v * p.tg;
     h.ntok = min(p.tg, p.B - h.tok0);
   } else {
-    const VExpert ve = p.ve[v];
+    const VExpert ve = ve_tab[v];
     h.expert = ve.expert;
     h.tok0 = ve.start;
     h.ntok = ve.count;
@@ -176,7 +177,7 @@ __device__ __forceinline__ const uint8_t* weight_src(const Params& p, const Hdr&
 // Issue this stage's activation copies (all 32 producer lanes).
 template <int KIND>
 __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t* act, uint64_t* bar,
-                                          int lane) {
+                                          int lane, const int* slot_tab) {
   if (KIND == KIND_RL || KIND == KIND_SGU) {
     const int bytes = h.nb * 64;
     for (int r = lane; r < h.ntok; r += 32)
@@ -184,7 +185,7 @@ __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t
   } else if (KIND == KIND_EGU) {
     const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
     for (int r = lane; r < h.ntok; r += 32) {
-      const int slot = p.slots_sorted[h.tok0 + r];
+      const int slot = slot_tab[h.tok0 + r];
       const int tok = slot / p.topk;
       bulk_g2s(act + r * p.act_stride, p.z_mx + ((long long)tok * cz + h.chunk) * kActRecBytes,
                kActRecBytes, bar);
@@ -207,8 +208,8 @@ __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t
 }
 
 template <int KIND>
-__device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint64_t* full,
-                         uint64_t* empty, int lane) {
+__device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t* tables,
+                         uint64_t* full, uint64_t* empty, int lane) {
   int stage = 0;
   uint32_t ephase = 1;  // empty barriers start "released"
   Space sp;
@@ -220,21 +221,29 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint64_
     waited = true;
   }
   sp = make_space<KIND>(p);
+  // routing tables in shared memory: the per-stage lookups then cost no
+  // global round trip (they are visible to the consumers through the first
+  // full-barrier completion)
+  VExpert* ve_tab = reinterpret_cast<VExpert*>(tables);
+  int* slot_tab = reinterpret_cast<int*>(tables + (size_t)p.ve_max * sizeof(VExpert));
+  if (KindTraits<KIND>::kDynamicSpace) {
+    const int nve = *reinterpret_cast<volatile int*>(p.nve);
+    for (int i = lane; i < nve; i += 32) ve_tab[i] = p.ve[i];
+    for (int i = lane; i < p.ld_slots; i += 32) slot_tab[i] = p.slots_sorted[i];
+    __syncwarp();
+  }
 
-  auto grab = [&]() -> int {
-    int v = 0;
-    if (lane == 0) v = atomicAdd(&ctl->cursor, 1);
-    return __shfl_sync(0xffffffffu, v, 0);
-  };
-
-  int piece = grab();
+  // lane 0 keeps one cursor grab in flight; its result is read one piece later
+  int grabbed = 0;
+  if (lane == 0) grabbed = atomicAdd(&ctl->cursor, 1);
+  int piece = __shfl_sync(0xffffffffu, grabbed, 0);
+  if (lane == 0) grabbed = atomicAdd(&ctl->cursor, 1);
   while (true) {
     if (piece >= sp.total) break;
     const int per_v = p.RB * sp.ppr;
     const int pr = (piece % per_v) % sp.ppr;
     const int c_first = (int)((long long)pr * p.C / sp.ppr);
     const int c_last = (int)((long long)(pr + 1) * p.C / sp.ppr);
-    const int next_piece = grab();
     for (int c = c_first; c < c_last; ++c) {
       // before the dependency resolves, fill at most one ring of weight-only stages
       if (!waited && prefetched == p.nstages) {
@@ -244,13 +253,13 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint64_
         for (int s = 0; s < prefetched; ++s) {
           uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
           const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
-          issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane);
+          issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
         }
       }
       if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY)) return;
       uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
       Hdr h;
-      fill_header<KIND>(p, sp, piece, c, c_first, c_last, h);
+      fill_header<KIND>(p, sp, piece, c, c_first, c_last, h, ve_tab);
       if (lane == 0) {
         *reinterpret_cast<Hdr*>(sb) = h;
         mbar_arrive_expect_tx(&full[stage], KindTraits<KIND>::kTileBytes + h.act_bytes);
@@ -258,7 +267,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint64_
       }
       __syncwarp();
       if (waited)
-        issue_act<KIND>(p, h, sb + p.act_off, &full[stage], lane);
+        issue_act<KIND>(p, h, sb + p.act_off, &full[stage], lane, slot_tab);
       else
         ++prefetched;
       if (++stage == p.nstages) {
@@ -266,7 +275,8 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint64_
         ephase ^= 1;
       }
     }
-    piece = next_piece;
+    piece = __shfl_sync(0xffffffffu, grabbed, 0);
+    if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1);
   }
   if (!waited) {
     pdl_wait();
@@ -274,7 +284,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint64_
     for (int s = 0; s < prefetched; ++s) {
       uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
       const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
-      issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane);
+      issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
     }
   }
   // end marker
@@ -506,7 +516,7 @@ __device__ void route_tokens(const Params& p, uint8_t* scratch, int tid, int war
 
 template <int KIND, int NT>
 __device__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
-                         int* sm_flag, int tid, int warp, int lane) {
+                         int* sm_flag, const int* slot_tab, int tid, int warp, int lane) {
   const int g = lane >> 2, tig = lane & 3;
   if (KIND == KIND_RL) {
     if (h.rb < p.RB_router) {
@@ -582,7 +592,7 @@ __device__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uin
         const int l = h.rb * kRowsPerBlock + 16 * warp + ((q & 2) ? g + 8 : g);
         const int col = 8 * t + 2 * tig + (q & 1);
         if (col < h.ntok && l < p.L) {
-          const int slot = p.slots_sorted[h.tok0 + col];
+          const int slot = slot_tab[h.tok0 + col];
           p.y[((long long)(l >> 6) * p.ld_slots + slot) * 64 + (l & 63)] = acc[t][q];
         }
       }
@@ -633,7 +643,7 @@ __device__ void route_tokens(const Params& p, uint8_t* scratch, int tid, int war
       key[j] = -INFINITY;
       src[j] = 0.f;
       if (e < E) {
-        const float l = ld_cg(p.logits + (long long)b * E + e);
+        const float l = __ldcg(p.logits + (long long)b * E + e);
         if (p.score_fn == 1) {
           const float s = 1.0f / (1.0f + expf(-l));
           src[j] = s;
@@ -756,15 +766,79 @@ __device__ void route_tokens(const Params& p, uint8_t* scratch, int tid, int war
 // ---------------------------------------------------------------------------
 // consumer warps
 
+// Split-K partial sums: [piece][token column][128 rows] floats, only the
+// columns that hold tokens are written.
+template <int NT>
+__device__ __forceinline__ void write_partial(const Params& p, int piece, int ntok,
+                                              const float (&acc)[NT][4], int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  float* base = p.partials + (long long)piece * (NT * 8 * kRowsPerBlock);
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = 8 * t + 2 * tig + (q & 1);
+      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+      if (col < ntok) base[col * kRowsPerBlock + row] = acc[t][q];
+    }
+}
+
+// Sum the row block's pieces in piece order (the same order whatever CTA ran
+// them, so the result is deterministic).
+template <int NT>
+__device__ __forceinline__ void sum_partials(const Params& p, const Hdr& h, float (&acc)[NT][4],
+                                             int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  const long long first = (long long)(h.v * p.RB + h.rb) * h.ppr;
+  const long long stride = NT * 8 * kRowsPerBlock;
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = 8 * t + 2 * tig + (q & 1);
+      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+      float sum = 0.f;
+      if (col < h.ntok) {
+        const float* src = p.partials + first * stride + col * kRowsPerBlock + row;
+        int pr = 0;
+        for (; pr + 8 <= h.ppr; pr += 8) {
+          float v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (pr + u) * stride);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) sum += v[u];
+        }
+        for (; pr < h.ppr; ++pr) sum += __ldcg(src + pr * stride);
+      }
+      acc[t][q] = sum;
+    }
+}
+
+template <int KIND, int NT>
+__device__ void finalize(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
+                         int* sm_flag, const int* slot_tab, int tid, int warp, int lane) {
+  sum_partials<NT>(p, h, acc, warp, lane);
+  if (tid == 0) p.counters[h.v * p.RB + h.rb] = 0;  // ready for the next launch
+  epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+}
+
 template <int KIND, int NT>
 __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, uint64_t* empty,
-                         uint8_t* scratch, int* sm_flag, int warp, int lane) {
+                         uint8_t* scratch, int* sm_flag, const int* slot_tab, int warp, int lane) {
   const int tid = warp * 32 + lane;
   int stage = 0;
   uint32_t phase = 0;
   int nbuf = 0;
   float acc[NT][4];
   zero_acc(acc);
+  // A piece whose ticket (finalize counter) is still in flight: thread 0
+  // issues the atomic after the piece's partials are written and reads its
+  // result only at the next piece end, so nobody waits on the round trip.
+  bool pend = false;
+  Hdr pend_h;
+  int ticket = 0;
+  int* tflag = sm_flag + 4;  // two alternating slots
+  int tslot = 0;
   // activations, routing tables and partial sums of the previous kernel are
   // read only after the dependency has resolved; the next kernel may then be
   // scheduled (it cannot overtake this one's own predecessor)
@@ -796,40 +870,24 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
     if (!(h.flags & HDR_LAST)) continue;
 
     if (h.ppr == 1) {
-      epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, tid, warp, lane);
+      epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
       continue;
     }
-    // split-K: publish this piece's partial sums, the last piece of the row
-    // block adds all of them in piece order
-    float4* part = reinterpret_cast<float4*>(p.partials + (long long)h.piece * NT * 1024);
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-      part[(t * kConsumerWarps + warp) * 32 + lane] =
-          make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
-    __threadfence();
+    write_partial<NT>(p, h.piece, h.ntok, acc, warp, lane);
+    if (tid == 0 && pend) tflag[tslot] = (ticket == pend_h.ppr - 1);
+    named_sync(1, kConsumerThreads);  // every warp's partials precede thread 0's release
+    const bool fin = pend && tflag[tslot] != 0;
+    if (tid == 0) ticket = atom_add_acqrel(p.counters + h.v * p.RB + h.rb, 1);
+    const Hdr prev = pend_h;
+    pend_h = h;
+    pend = true;
+    tslot ^= 1;
+    if (fin) finalize<KIND, NT>(p, prev, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+  }
+  if (pend) {
+    if (tid == 0) tflag[tslot] = (ticket == pend_h.ppr - 1);
     named_sync(1, kConsumerThreads);
-    int* ctr = p.counters + h.v * p.RB + h.rb;
-    if (tid == 0) *sm_flag = (atomicAdd(ctr, 1) == h.ppr - 1);
-    named_sync(1, kConsumerThreads);
-    const bool last = *sm_flag != 0;
-    named_sync(1, kConsumerThreads);
-    if (!last) continue;
-    __threadfence();
-    zero_acc(acc);
-    const long long first = (long long)(h.v * p.RB + h.rb) * h.ppr;
-    for (int pr = 0; pr < h.ppr; ++pr) {
-      const float* src = p.partials + (first + pr) * NT * 1024;
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const float* q = src + ((t * kConsumerWarps + warp) * 32 + lane) * 4;
-        acc[t][0] += ld_cg(q + 0);
-        acc[t][1] += ld_cg(q + 1);
-        acc[t][2] += ld_cg(q + 2);
-        acc[t][3] += ld_cg(q + 3);
-      }
-    }
-    if (tid == 0) *ctr = 0;
-    epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, tid, warp, lane);
+    if (tflag[tslot] != 0) finalize<KIND, NT>(p, pend_h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
   }
 }
 
@@ -839,13 +897,16 @@ template <int KIND, int NT>
 __global__ void __launch_bounds__(kThreads, (NT <= 4 ? 2 : 1))
     moe_kernel(const __grid_constant__ Params p) {
   // shared memory: [0,128) full barriers, [128,256) empty barriers,
-  // [256,512) flags, [scratch_off, stage_off) scratch, [stage_off, ...) ring
+  // [256,512) flags, [scratch_off, ...) scratch, [table_off, ...) routing
+  // tables (expert kernels), [stage_off, ...) ring
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
   int* sm_flag = reinterpret_cast<int*>(smem + 256);
   uint8_t* scratch = smem + p.scratch_off;
   uint8_t* stages = smem + p.stage_off;
+  uint8_t* tables = smem + p.table_off;
+  const int* slot_tab = reinterpret_cast<const int*>(tables + (size_t)p.ve_max * sizeof(VExpert));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Ctl* ctl = p.ctl;
   if (threadIdx.x == 0) {
@@ -857,9 +918,9 @@ __global__ void __launch_bounds__(kThreads, (NT <= 4 ? 2 : 1))
   }
   __syncthreads();
   if (warp == kConsumerWarps) {
-    producer<KIND>(p, ctl, stages, full, empty, lane);
+    producer<KIND>(p, ctl, stages, tables, full, empty, lane);
   } else {
-    consumer<KIND, NT>(p, stages, full, empty, scratch, sm_flag, warp, lane);
+    consumer<KIND, NT>(p, stages, full, empty, scratch, sm_flag, slot_tab, warp, lane);
   }
   __syncthreads();
   if (threadIdx.x == 0) {

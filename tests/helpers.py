@@ -33,39 +33,49 @@ def assert_close(got, ref, what, max_rel=MAX_REL, mean_rel=MEAN_REL):
 
 
 def logit_tolerance(shape, w, x):
-    """Bound on the fp32 router logits: 2^-16 of the sum of |x_h W_he| (per token, expert)."""
+    """Bound on the fp32 router logits: 2^-14 of the sum of |x_h W_he|, about the
+    worst-case rounding of the few hundred fp32 additions behind each logit."""
     xf = np.abs(bf16_to_f32(x).astype(np.float64))
     Wr = np.abs(bf16_to_f32(w["router_w"]).astype(np.float64).reshape(shape.hidden, shape.num_experts))
-    return (xf @ Wr) * 2.0 ** -16 + 1e-30
+    return (xf @ Wr) * 2.0 ** -14 + 1e-30
+
+
+def _keys(shape, w, logits):
+    lg = np.asarray(logits, np.float64)
+    if shape.score_fn == synth.SCORE_SIGMOID:
+        return 1 / (1 + np.exp(-lg)) + (0 if w["router_bias"] is None else w["router_bias"].astype(np.float64))
+    return lg  # softmax ranks by logit (monotone in the probability)
 
 
 def check_routing(shape, w, x, gpu_ids, gpu_w, gpu_logits, orc):
-    """Top-k parity: exact where the oracle's selection margin exceeds what the
-    GPU's fp32 keys can move; elsewhere the GPU's choice must be the top-k of
-    its own logits under the same rule (reported as a near tie)."""
+    """Top-k parity.
+
+    The GPU's logits must sit within the fp32 rounding bound of the oracle's.
+    If every selection key moved by at most d, any gap wider than 2d keeps its
+    order, so for tokens whose oracle margin (k-th minus (k+1)-th key) exceeds
+    twice the measured key deviation (plus the fp32 rounding of the key
+    itself) the ids must match exactly.  Closer calls are reported as near
+    ties and checked for validity: the GPU's ids must be the top-k of its own
+    logits under the same rule."""
     B, k, E = x.shape[0], shape.top_k, shape.num_experts
     tol = logit_tolerance(shape, w, x)
     dl = np.abs(gpu_logits.astype(np.float64) - orc["logits"])
     assert np.all(dl <= tol), "router logits off by %.3g (tolerance %.3g)" % (
         float(np.max(dl - tol)), float(tol.max()))
-    # key error bound: sigmoid is 1/4-Lipschitz, softmax keys are logits here
-    key_err = 0.25 * tol.max(1) if shape.score_fn == synth.SCORE_SIGMOID else tol.max(1)
+    kg = _keys(shape, w, gpu_logits)
+    ko = _keys(shape, w, orc["logits"])
+    dev = np.max(np.abs(kg - ko), axis=1) + 2.0 ** -22 * (np.max(np.abs(ko), axis=1) + 1.0)
     near = []
     for b in range(B):
-        if orc["margin"][b] > 2 * key_err[b] + 1e-6:
+        if orc["margin"][b] > 2 * dev[b]:
             assert sorted(gpu_ids[b].tolist()) == sorted(orc["ids"][b].tolist()), (
-                "token %d: ids %s vs oracle %s (margin %.3g)" % (b, gpu_ids[b], orc["ids"][b], orc["margin"][b]))
-            # combine weights follow the oracle's key order
+                "token %d: ids %s vs oracle %s (margin %.3g, key deviation %.3g)" % (
+                    b, gpu_ids[b], orc["ids"][b], orc["margin"][b], dev[b]))
             order = {e: j for j, e in enumerate(orc["ids"][b].tolist())}
             wo = np.array([orc["weights"][b][order[e]] for e in gpu_ids[b].tolist()])
             np.testing.assert_allclose(gpu_w[b], wo, rtol=1e-5, atol=1e-7)
         else:
             near.append(b)
-            lg = gpu_logits[b].astype(np.float64)
-            if shape.score_fn == synth.SCORE_SIGMOID:
-                key = 1 / (1 + np.exp(-lg)) + (0 if w["router_bias"] is None else w["router_bias"])
-            else:
-                key = lg
-            order = sorted(range(E), key=lambda e: (-key[e], e))[:k]
+            order = sorted(range(E), key=lambda e: (-kg[b][e], e))[:k]
             assert sorted(order) == sorted(gpu_ids[b].tolist()), "near-tie token %d invalid" % b
     return near
