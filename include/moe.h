@@ -194,6 +194,36 @@ MOE_API moe_status moe_get_plan_info(moe_plan p, moe_plan_info *info);
 MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
 MOE_API moe_status moe_get_profile(moe_plan p, float *ms, int32_t *count);
 
+/*
+ * Router scores and top-k for callers that cannot allocate device memory.
+ * The source pages have no counterpart to this call; it exists for code that
+ * runs where no allocation may happen (a fixed up-front memory budget, a
+ * custom allocator that must account for every byte, a thread that may not
+ * call cudaMalloc) and therefore cannot create a plan.
+ *
+ * Computes the routing step of moe_forward for B = num_tokens tokens on the
+ * CURRENT device: logits = x . router_w, scores (softmax, or sigmoid plus the
+ * selection bias), top-k with ties to the lower index, combine weights
+ * renormalised when `renormalize`, times routed_scale.
+ *   x         device bf16 [B][hidden]
+ *   router_w  device bf16 [hidden][num_experts] (canonical, unpacked)
+ *   router_bias device f32 [num_experts] or NULL (used for sigmoid scoring only)
+ *   ids       device int32 [B][top_k] out, key-descending
+ *   weights   device f32   [B][top_k] out
+ * Allocates nothing: its only scratch is a 512 KB array in the library's
+ * device memory (statically sized, present on every GPU that loads the
+ * library until the process exits).  The first call on a device looks up that
+ * array's device address; make that first call before any stream capture.
+ * Every call shares the array, so calls whose kernels overlap on the GPU
+ * (different streams, or different host threads) race; serialise them.
+ * Limits: B <= 128, num_experts <= 1024, top_k <= 16, else MOE_ERR_UNSUPPORTED.
+ * Asynchronous on `stream`.
+ */
+MOE_API moe_status moe_route_noalloc(const void *x, const void *router_w, const float *router_bias,
+                                     int32_t num_tokens, int32_t hidden, int32_t num_experts,
+                                     int32_t top_k, int32_t score_fn, int32_t renormalize,
+                                     float routed_scale, int32_t *ids, float *weights, void *stream);
+
 /* Release everything the plan owns.  NULL is ignored. */
 MOE_API void moe_plan_destroy(moe_plan p);
 

@@ -25,7 +25,8 @@ MOE_DBG_LOGITS, MOE_DBG_Z, MOE_DBG_H, MOE_DBG_Y, MOE_DBG_HS = range(5)
 # every entry point include/moe.h declares
 ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forward_host",
                "moe_last_routing", "moe_debug_fetch", "moe_sync_status", "moe_get_plan_info",
-               "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile"]
+               "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile",
+               "moe_route_noalloc"]
 KERNEL_NAMES = ["router_latent", "shared_gate_up", "expert_gate_up", "expert_down", "latent_tail"]
 
 
@@ -80,6 +81,9 @@ def load_library():
     lib.moe_get_plan_info.argtypes = [P, ctypes.POINTER(moe_plan_info)]
     lib.moe_plan_destroy.argtypes = [P]
     lib.moe_plan_destroy.restype = None
+    lib.moe_route_noalloc.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_float, P, P, P]
     lib.moe_set_profiling.argtypes = [P, ctypes.c_int32]
     lib.moe_get_profile.argtypes = [P, P, P]
     lib.moe_status_str.argtypes = [ctypes.c_int]
@@ -168,6 +172,16 @@ def moe_get_profile(plan: int):
     n = ctypes.c_int32()
     _check(load_library().moe_get_profile(plan, ms, ctypes.byref(n)), "moe_get_profile")
     return dict(zip(KERNEL_NAMES, list(ms))), n.value
+
+
+def moe_route_noalloc(x, router_w, router_bias, num_tokens: int, hidden: int, num_experts: int,
+                      top_k: int, score_fn: int, renormalize: int, routed_scale: float, ids, weights,
+                      stream=None) -> int:
+    """Router + top-k without any allocation (device tensors in, device tensors out)."""
+    return load_library().moe_route_noalloc(_ptr(x), _ptr(router_w), _ptr(router_bias), num_tokens,
+                                            hidden, num_experts, top_k, score_fn, renormalize,
+                                            routed_scale, _ptr(ids), _ptr(weights),
+                                            _stream_ptr(stream))
 
 
 def moe_plan_destroy(plan: int) -> None:

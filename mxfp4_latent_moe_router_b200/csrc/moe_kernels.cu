@@ -41,6 +41,7 @@
 #include "engine.cuh"
 #include "layout.cuh"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -611,16 +612,8 @@ __device__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uin
 }
 
 // ---------------------------------------------------------------------------
-// top-k routing and per-expert token lists (one CTA, 256 threads)
-//
-// Scores: softmax ranks experts by logit (the same order as by probability);
-// sigmoid ranks by sigmoid(logit) + bias.  Ties go to the lower expert index.
-// Combine weights come from the unbiased score, renormalised over the chosen
-// experts when requested, times routed_scale.
-
-__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
-  return ka > kb || (ka == kb && ia < ib);
-}
+// top-k routing and per-expert token lists (one CTA, 256 threads); the
+// per-token selection is warp_topk (topk.cuh).
 
 __device__ void route_tokens(const Params& p, uint8_t* scratch, int tid, int warp, int lane) {
   const int E = p.E, K = p.topk, B = p.B;
@@ -633,81 +626,14 @@ __device__ void route_tokens(const Params& p, uint8_t* scratch, int tid, int war
     fill[i] = 0;
   }
   named_sync(1, kConsumerThreads);
-  constexpr int EPL = 32;  // E <= 1024
   for (int b = warp; b < B; b += kConsumerWarps) {
-    float key[EPL], src[EPL];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      key[j] = -INFINITY;
-      src[j] = 0.f;
-      if (e < E) {
-        const float l = __ldcg(p.logits + (long long)b * E + e);
-        if (p.score_fn == 1) {
-          const float s = 1.0f / (1.0f + expf(-l));
-          src[j] = s;
-          key[j] = s + (p.bias ? p.bias[e] : 0.f);
-        } else {
-          src[j] = l;
-          key[j] = l;
-          mx = fmaxf(mx, l);
-        }
-      }
-    }
-    float den = 1.f;
-    if (p.score_fn == 0) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j)
-        if (lane + 32 * j < E) sum += expf(src[j] - mx);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      den = sum;
-    }
-    int sel_id = 0;
-    float sel_src = 0.f, tot = 0.f;
-    for (int r = 0; r < K; ++r) {
-      float bk = -INFINITY, bs = 0.f;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && better(key[j], e, bk, bi)) {
-          bk = key[j];
-          bi = e;
-          bs = src[j];
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        if (better(ok, oi, bk, bi)) {
-          bk = ok;
-          bi = oi;
-          bs = os;
-        }
-      }
-      if (bi < 0 || bi >= E) bi = 0;  // only reachable with NaN logits; keeps indices in range
-      // remove the winner
-#pragma unroll
-      for (int j = 0; j < EPL; ++j)
-        if (lane + 32 * j == bi) key[j] = -INFINITY;
-      const float sv = (p.score_fn == 0) ? expf(bs - mx) / den : bs;
-      tot += sv;
-      if (lane == r) {
-        sel_id = bi;
-        sel_src = sv;
-      }
-    }
+    int sel_id;
+    float sel_w;
+    warp_topk(p.logits + (long long)b * E, E, K, p.score_fn, p.bias, p.renorm, p.routed_scale, lane,
+              sel_id, sel_w);
     if (lane < K) {
-      const float wv = (p.renorm ? sel_src / tot : sel_src) * p.routed_scale;
       p.ids[b * K + lane] = sel_id;
-      p.wts[b * K + lane] = wv;
+      p.wts[b * K + lane] = sel_w;
       ids_s[b * K + lane] = sel_id;
       atomicAdd(&cnt[sel_id], 1);
     }
