@@ -192,6 +192,20 @@ MOE_API moe_status moe_get_plan_info(moe_plan p, moe_plan_info *info);
  * profiled forwards to *count, then clears both.
  */
 MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
+
+/*
+ * Per-CTA timeline of the most recent forward, for measurement only; exists
+ * when the plan was created with the environment variable MOE_TRACE set
+ * (else MOE_ERR_UNSUPPORTED).  host receives count = 5 * num_sms * 24 uint64:
+ * for kernel kind k (launch order as in moe_get_profile) and CTA c, the 24
+ * values at (k * num_sms + c) * 24 are {start ns, end ns, pieces, finalizes,
+ * top-k start ns, top-k end ns, first stage ready ns, finalize ns, consumer
+ * cycles waiting for data, computing, closing pieces, producer cycles waiting
+ * for a free stage, issuing, stages issued, 0, 0} (ns from globaltimer,
+ * cycles from clock64); value 14 is the SM the CTA ran on.
+ * Synchronises the device.
+ */
+MOE_API moe_status moe_debug_trace(moe_plan p, uint64_t *host, int64_t count);
 MOE_API moe_status moe_get_profile(moe_plan p, float *ms, int32_t *count);
 
 /*

@@ -26,7 +26,7 @@ MOE_DBG_LOGITS, MOE_DBG_Z, MOE_DBG_H, MOE_DBG_Y, MOE_DBG_HS = range(5)
 ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forward_host",
                "moe_last_routing", "moe_debug_fetch", "moe_sync_status", "moe_get_plan_info",
                "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile",
-               "moe_route_noalloc"]
+               "moe_route_noalloc", "moe_debug_trace"]
 KERNEL_NAMES = ["router_latent", "shared_gate_up", "expert_gate_up", "expert_down", "latent_tail"]
 
 
@@ -85,6 +85,7 @@ def load_library():
                                       ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                       ctypes.c_float, P, P, P]
     lib.moe_set_profiling.argtypes = [P, ctypes.c_int32]
+    lib.moe_debug_trace.argtypes = [P, P, ctypes.c_int64]
     lib.moe_get_profile.argtypes = [P, P, P]
     lib.moe_status_str.argtypes = [ctypes.c_int]
     lib.moe_status_str.restype = ctypes.c_char_p
@@ -182,6 +183,14 @@ def moe_route_noalloc(x, router_w, router_bias, num_tokens: int, hidden: int, nu
                                             hidden, num_experts, top_k, score_fn, renormalize,
                                             routed_scale, _ptr(ids), _ptr(weights),
                                             _stream_ptr(stream))
+
+
+def moe_debug_trace(plan: int, num_sms: int):
+    """Per-CTA timeline of the last forward: uint64 array [5 kinds][num_sms][24]."""
+    import numpy as np
+    a = np.zeros((5, num_sms, 24), np.uint64)
+    _check(load_library().moe_debug_trace(plan, a.ctypes.data, a.size), "moe_debug_trace")
+    return a
 
 
 def moe_plan_destroy(plan: int) -> None:

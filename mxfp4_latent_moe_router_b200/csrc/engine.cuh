@@ -54,6 +54,9 @@ struct Params {
   // shared memory geometry (bytes)
   int nstages, stage_bytes, act_off, act_stride, scratch_off, stage_off;
   int table_off;  // EGU/EDN: shared-memory copy of the routing tables
+  // TAIL with few tokens: the whole activation [c ; h_s] of every token is
+  // formed once per CTA in shared memory (bf16 hi + lo per value); 0 = off
+  int res_off, res_stride, res_k;
 
   const uint8_t* wt;       // packed tiles
   long long matrix_bytes;  // EGU/EDN: bytes of one expert's tiles
@@ -76,6 +79,9 @@ struct Params {
   int ve_max;
 
   Ctl* ctl;
+  // optional trace: per CTA 8 x u64 {start ns, end ns, pieces, finalizes,
+  // route start ns, route end ns, first stage ready ns, 0}; null when off
+  unsigned long long* trace;
   int* counters;   // finalize tickets per (virtual matrix, row block)
   int* router_done;
   float* partials;

@@ -28,7 +28,6 @@ constexpr int kHdr = 128;
 constexpr int kTailTg = 16;
 constexpr int kExpertTg = 32;
 constexpr int kBigSmem = 227 * 1024;
-constexpr int kSmallSmem = 113 * 1024;
 
 struct KindGeom {
   int RB = 0, C = 0, KL = 0;
@@ -88,8 +87,10 @@ struct moe_plan_s {
   // tuning knobs read once at plan creation (environment): pieces each CTA
   // should get on average, and whether kernels chain with programmatic
   // dependent launch
-  int pieces_per_cta = 8;
+  int pieces_per_cta = 3;
   bool use_pdl = true;
+
+  unsigned long long* trace = nullptr;  // [KIND_COUNT][max grid][8] when MOE_TRACE is set
 
   bool profiling = false;
   cudaEvent_t ev_prof[KIND_COUNT][2] = {};
@@ -171,18 +172,26 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   return f;
 }
 
+int g_max_stages = 6;  // ring depth cap (environment MOE_MAX_STAGES)
+
 struct SmemGeom {
-  int stage_bytes, nstages, act_off, act_stride, table_bytes, stage_off;
+  int stage_bytes, nstages, act_off, act_stride, table_bytes, stage_off, res_bytes;
   size_t total;
 };
 
-SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int slots) {
+// bytes of the tail's resident activation for B tokens (0: too large, use per-stage staging)
+constexpr int kResidentMax = 72 * 1024;
+int resident_stride(int res_k) { return res_k * 4 + 64; }
+
+SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int slots,
+                   int res_bytes = 0) {
   SmemGeom s;
   // routing tables (virtual experts + expert-sorted slots) for the expert kernels
   s.table_bytes = 0;
   if (kind == KIND_EGU || kind == KIND_EDN)
     s.table_bytes = ((ve_max * (int)sizeof(VExpert) + slots * 4) + 127) / 128 * 128;
-  const int stage_off = kStageOff + s.table_bytes;
+  s.res_bytes = res_bytes;
+  const int stage_off = kStageOff + s.table_bytes + res_bytes;
   int act = 0;
   s.act_stride = 0;
   if (kind == KIND_RL || kind == KIND_SGU) {
@@ -192,19 +201,26 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int 
     s.act_stride = 576;
     act = 8 * nt * s.act_stride;
   } else {
-    act = tail_tg_eff * std::max(1, topk) * 256;
+    act = res_bytes ? 0 : tail_tg_eff * std::max(1, topk) * 256;
   }
   const int tile = (kind == KIND_EGU || kind == KIND_EDN) ? kMxTileBytes : kDenseTileBytes;
   s.act_off = kHdr + tile;
   s.stage_bytes = ((kHdr + tile + act) + 127) / 128 * 128;
-  const int budget = s.stage_bytes <= 24 * 1024 ? kSmallSmem : kBigSmem;
-  s.nstages = std::max(2, std::min(8, (budget - stage_off) / s.stage_bytes));
+  // one CTA per SM: the main-stream kernels, the side-stream kernel and a
+  // kernel launched early by programmatic dependent launch then never share an
+  // SM, and the whole shared memory goes to the ring
+  const int budget = kBigSmem;
+  // enough bytes in flight to saturate HBM (about 6 x 16 KB per SM); more only
+  // lengthens the queues every other memory request waits behind
+  s.nstages = std::max(2, std::min(g_max_stages, (budget - stage_off) / s.stage_bytes));
   s.stage_off = stage_off;
   s.total = (size_t)stage_off + (size_t)s.nstages * s.stage_bytes;
+  // more than half of the SM's shared memory: never two CTAs on one SM
+  s.total = std::max(s.total, (size_t)(116 * 1024));
   return s;
 }
 
-int g_pieces_per_cta = 8;  // set from the plan before any geometry call
+int g_pieces_per_cta = 3;  // set from the plan before any geometry call
 int target_pieces(int grid, int nt) { return grid * std::max(1, g_pieces_per_cta / nt); }
 
 Params base_params(const moe_plan_s* p, int B) {
@@ -248,6 +264,7 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   q.C = p->g[kind].C;
   q.KL = p->g[kind].KL;
   q.ctl = p->ctl + kind;
+  q.trace = p->trace ? p->trace + (size_t)kind * p->num_sms * 24 : nullptr;
   q.counters = p->counters[kind];
   q.partials = p->partials[kind];
   q.nstages = s.nstages;
@@ -342,6 +359,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->num_sms = prop.multiProcessorCount;
   if (const char* e = getenv("MOE_PIECES_PER_CTA")) p->pieces_per_cta = std::max(1, atoi(e));
   if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
+  if (const char* e = getenv("MOE_MAX_STAGES")) g_max_stages = std::max(2, std::min(8, atoi(e)));
   g_pieces_per_cta = p->pieces_per_cta;
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
@@ -434,6 +452,11 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
     TRY(alloc(p, &v, sizeof(float) * std::max<size_t>(p->partial_cap[k], 4), false));
     p->partials[k] = (float*)v;
   }
+  if (getenv("MOE_TRACE")) {
+    TRY(alloc(p, &v, sizeof(unsigned long long) * KIND_COUNT * p->num_sms * 24, false));
+    p->trace = (unsigned long long*)v;
+    CUDA_TRY(cudaMemset(v, 0, sizeof(unsigned long long) * KIND_COUNT * p->num_sms * 24));
+  }
   TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
   p->x_stage = (uint16_t*)v;
   TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
@@ -510,6 +533,10 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.main_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
   }
+  // join the side stream here: the down projection cannot prefetch anything
+  // before its dependency resolves anyway, while the tail keeps its
+  // programmatic edge to the down projection and prefetches W_out early
+  if (shared) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));
   {
     Params q = base;
     const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
@@ -519,11 +546,19 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.main_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
   }
-  if (shared) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_TAIL, f.nt_tail, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
+    const int res_k = p->g[KIND_TAIL].C * kDenseChunkK;
+    const int res_bytes =
+        (B * resident_stride(res_k) <= kResidentMax) ? B * resident_stride(res_k) : 0;
+    const SmemGeom sm =
+        smem_geom(KIND_TAIL, f.nt_tail, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, res_bytes);
     set_kind(q, p, KIND_TAIL, sm);
+    if (res_bytes) {
+      q.res_off = kStageOff + sm.table_bytes;
+      q.res_stride = resident_stride(res_k);
+      q.res_k = res_k;
+    }
     const int passes = (B + p->tail_tg - 1) / p->tail_tg;
     q.PPR = ppr_for(target_pieces(f.tail_grid, f.nt_tail), q.RB * passes, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
@@ -803,6 +838,17 @@ moe_status moe_get_plan_info(moe_plan p, moe_plan_info* info) {
   info->expert_weight_bytes =
       (3LL * c.expert_inter * c.latent) / 2 + (3LL * c.expert_inter * c.latent) / 32;
   info->kernels_per_forward = c.shared_inter > 0 ? 5 : 4;
+  return MOE_OK;
+}
+
+moe_status moe_debug_trace(moe_plan p, uint64_t* host, int64_t count) {
+  if (!p || !host) return MOE_ERR_INVALID_ARG;
+  if (!p->trace) return MOE_ERR_UNSUPPORTED;
+  const int64_t n = (int64_t)KIND_COUNT * p->num_sms * 24;
+  if (count != n) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(host, p->trace, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost));
   return MOE_OK;
 }
 

@@ -1,0 +1,1190 @@
+// moe_engine.cuh -- the five kernels of one latent-MoE decode step on sm_100a
+// (device code; each kind is instantiated in its own moe_k_<kind>.cu).
+//
+// One engine serves all five: a CTA of 8 consumer warps and 1 producer warp.
+// The producer grabs "pieces" (a row block of 128 output rows x a run of K
+// chunks) from a global cursor and streams each chunk's weight tile plus the
+// activation rows it multiplies into a ring of shared-memory stages with bulk
+// copies (TMA engine) that complete on mbarriers.  Each consumer warp owns 16
+// of the 128 rows and multiplies them with m16n8k16 warp MMAs, weights as the
+// 16-row A operand and up to 8*NT tokens as the 8-column B operand ("swap
+// AB"), fp32 accumulators in registers.  When a piece ends, its fp32 partial
+// sums go to global memory; the CTA that completes the last piece of a row
+// block sums all of them in piece order (deterministic split-K) and runs the
+// kernel's epilogue.  Dynamic piece grabbing balances the work across SMs and
+// lets a CTA that does extra epilogue work fall behind without stalling the
+// others.
+//
+//   KIND_RL   x . [W_r | W_in] -> router logits (fp32) and latent z (f16 MX);
+//             the CTA that finalises the last router row block runs top-k and
+//             builds the per-expert token lists while the rest of the grid is
+//             still streaming W_in.
+//             (page "Hyper Optimizing Kimi K3 in vLLM: Moving Fast and
+//              Responsibly", section 从算子之间找时间: router scores and the
+//              latent input projection as one matmul.)
+//   KIND_SGU  x . [W_sg | W_su] -> h_s = silu(g) * u (fp32), side stream.
+//             (same section: the shared expert on its own stream.)
+//   KIND_EGU  per routed expert, z . [Wg | Wu] (MXFP4) -> h = silu(g) * u (f16 MX)
+//   KIND_EDN  per routed expert, h . Wd (MXFP4) -> y (fp32, per token slot)
+//   KIND_TAIL c = sum_j w_j y_j formed from y while staging the activation
+//             tile (never written to memory), then [c ; h_s] . [W_out ; W_sd]
+//             -> out (bf16).
+//             (page "Kimi K3 在 vLLM 中的性能优化", section 延迟 MXFP4 最终化:
+//              the MXFP4 top-k finalize fused into the latent-tail kernel.)
+//
+// Only static weights are fetched before griddepcontrol.wait; activations are
+// fetched after it (page 1, section 更快的代码需要更有针对性的验证: an
+// activation load hoisted above a synchronisation wait was a real bug).
+#pragma once
+#include <cuda_runtime.h>
+
+#include "engine.cuh"
+#include "layout.cuh"
+#include "ptx.cuh"
+#include "topk.cuh"
+
+namespace moe {
+
+constexpr int kHdrBytes = 128;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kMaxStages = 8;
+constexpr int kTraceStride = 24;  // u64 per CTA in the optional trace
+
+enum : int { HDR_FIRST = 1, HDR_LAST = 2, HDR_END = 4 };
+
+struct Hdr {
+  int flags;
+  int piece, v, rb;
+  int chunk, nb, ntok, tok0;
+  int expert, ppr, act_bytes, pad;
+};
+
+template <int KIND>
+struct KindTraits {
+  static constexpr bool kMx = (KIND == KIND_EGU || KIND == KIND_EDN);
+  static constexpr int kTileBytes = kMx ? kMxTileBytes : kDenseTileBytes;
+  static constexpr int kChunkK = kMx ? kMxChunkK : kDenseChunkK;
+  // weights may be fetched before the previous kernel finishes
+  static constexpr bool kPrefetchWeights = (KIND == KIND_RL || KIND == KIND_TAIL);
+  static constexpr bool kDynamicSpace = (KIND == KIND_EGU || KIND == KIND_EDN);
+};
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+
+__device__ __forceinline__ float silu(float t) { return __fdividef(t, 1.0f + __expf(-t)); }
+
+// ---------------------------------------------------------------------------
+// iteration space
+
+struct Space {
+  int total;  // pieces
+  int ppr;
+};
+
+template <int KIND>
+__device__ __forceinline__ Space make_space(const Params& p) {
+  Space s;
+  if (KIND == KIND_EGU || KIND == KIND_EDN) {
+    const int V = *reinterpret_cast<volatile int*>(p.nve);
+    const int mats = V * p.RB;
+    int ppr = mats > 0 ? (p.target_pieces + mats - 1) / mats : 1;
+    ppr = ppr < 1 ? 1 : (ppr > p.C ? p.C : ppr);
+    s.ppr = ppr;
+    s.total = mats * ppr;
+  } else if (KIND == KIND_TAIL) {
+    const int passes = (p.B + p.tg - 1) / p.tg;
+    s.ppr = p.PPR;
+    s.total = passes * p.RB * p.PPR;
+  } else {
+    s.ppr = p.PPR;
+    s.total = p.RB * p.PPR;
+  }
+  return s;
+}
+
+// number of 32-wide K blocks in chunk c
+template <int KIND>
+__device__ __forceinline__ int chunk_blocks(const Params& p, int c) {
+  constexpr int kMaxB = KindTraits<KIND>::kChunkK / 32;
+  int k0, kext;
+  if (KIND == KIND_TAIL) {
+    if (c < p.C_lat) {
+      k0 = c * kDenseChunkK;
+      kext = p.L;
+    } else {
+      k0 = (c - p.C_lat) * kDenseChunkK;
+      kext = p.KS;
+    }
+  } else {
+    k0 = c * KindTraits<KIND>::kChunkK;
+    kext = p.KL;
+  }
+  int nb = (kext - k0) / 32;
+  return nb > kMaxB ? kMaxB : nb;
+}
+
+// ---------------------------------------------------------------------------
+// producer warp
+
+// Per piece: everything except the chunk-dependent fields.
+template <int KIND>
+__device__ __forceinline__ void piece_header(const Params& p, const Space& sp, int piece, Hdr& h,
+                                             const VExpert* ve_tab) {
+  const int per_v = p.RB * sp.ppr;
+  const int v = piece / per_v;
+  const int rem = piece - v * per_v;
+  h.piece = piece;
+  h.v = v;
+  h.rb = rem / sp.ppr;
+  h.ppr = sp.ppr;
+  h.expert = 0;
+  if (KIND == KIND_RL || KIND == KIND_SGU) {
+    h.ntok = p.B;
+    h.tok0 = 0;
+  } else if (KIND == KIND_TAIL) {
+    h.tok0 = v * p.tg;
+    h.ntok = min(p.tg, p.B - h.tok0);
+  } else {
+    const VExpert ve = ve_tab[v];
+    h.expert = ve.expert;
+    h.tok0 = ve.start;
+    h.ntok = ve.count;
+  }
+}
+
+// Per chunk: flags, block count and activation bytes.
+template <int KIND>
+__device__ __forceinline__ void chunk_header(const Params& p, int c, int c_first, int c_last, Hdr& h) {
+  h.flags = (c == c_first ? HDR_FIRST : 0) | (c == c_last - 1 ? HDR_LAST : 0);
+  h.chunk = c;
+  h.nb = chunk_blocks<KIND>(p, c);
+  int ab;
+  if (KIND == KIND_RL || KIND == KIND_SGU)
+    ab = h.ntok * h.nb * 64;
+  else if (KIND == KIND_EGU || KIND == KIND_EDN)
+    ab = h.ntok * kActRecBytes;
+  else
+    ab = p.res_off ? 0 : ((c < p.C_lat) ? h.ntok * p.topk * 256 : h.ntok * 256);
+  h.act_bytes = ab;
+}
+
+template <int KIND>
+__device__ __forceinline__ const uint8_t* weight_src(const Params& p, const Hdr& h) {
+  const long long tile = (long long)h.rb * p.C + h.chunk;
+  if (KindTraits<KIND>::kMx)
+    return p.wt + (long long)h.expert * p.matrix_bytes + tile * kMxTileBytes;
+  return p.wt + tile * kDenseTileBytes;
+}
+
+// Issue this stage's activation copies (all 32 producer lanes).
+template <int KIND>
+__device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t* act, uint64_t* bar,
+                                          int lane, const int* slot_tab) {
+  if (KIND == KIND_RL || KIND == KIND_SGU) {
+    const int bytes = h.nb * 64;
+    for (int r = lane; r < h.ntok; r += 32)
+      bulk_g2s(act + r * p.act_stride, p.x + (long long)r * p.H + h.chunk * kDenseChunkK, bytes, bar);
+  } else if (KIND == KIND_EGU) {
+    const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
+    for (int r = lane; r < h.ntok; r += 32) {
+      const int slot = slot_tab[h.tok0 + r];
+      const int tok = slot / p.topk;
+      bulk_g2s(act + r * p.act_stride, p.z_mx + ((long long)tok * cz + h.chunk) * kActRecBytes,
+               kActRecBytes, bar);
+    }
+  } else if (KIND == KIND_EDN) {
+    for (int r = lane; r < h.ntok; r += 32)
+      bulk_g2s(act + r * p.act_stride,
+               p.h_mx + ((long long)h.chunk * p.ld_slots + h.tok0 + r) * kActRecBytes, kActRecBytes,
+               bar);
+  } else {
+    if (lane == 0 && !p.res_off) {
+      if (h.chunk < p.C_lat)
+        bulk_g2s(act, p.y + ((long long)h.chunk * p.ld_slots + (long long)h.tok0 * p.topk) * 64,
+                 h.act_bytes, bar);
+      else
+        bulk_g2s(act, p.h_s + ((long long)(h.chunk - p.C_lat) * p.B + h.tok0) * 64, h.act_bytes,
+                 bar);
+    }
+  }
+}
+
+template <int KIND>
+__device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t* tables,
+                         uint64_t* full, uint64_t* empty, int lane) {
+  int stage = 0;
+  uint32_t ephase = 1;  // empty barriers start "released"
+  Space sp;
+  int prefetched = 0;  // stages filled with weights only, waiting for pdl_wait
+  bool waited = false;
+  if (!KindTraits<KIND>::kPrefetchWeights) {
+    pdl_wait();
+    pdl_trigger();
+    waited = true;
+  }
+  // routing tables in shared memory: the per-stage lookups then cost no
+  // global round trip (they are visible to the consumers through the first
+  // full-barrier completion).  The whole capacity is copied so that these
+  // loads and the count load below are independent and overlap.
+  VExpert* ve_tab = reinterpret_cast<VExpert*>(tables);
+  int* slot_tab = reinterpret_cast<int*>(tables + (size_t)p.ve_max * sizeof(VExpert));
+  if (KindTraits<KIND>::kDynamicSpace) {
+    for (int i = lane; i < p.ve_max; i += 32) ve_tab[i] = p.ve[i];
+    for (int i = lane; i < p.ld_slots; i += 32) slot_tab[i] = p.slots_sorted[i];
+  }
+  sp = make_space<KIND>(p);
+  __syncwarp();
+
+  // every CTA starts on piece blockIdx.x (no round trip before the first
+  // tile); later pieces come from the cursor, offset by the grid size.  Lane 0
+  // keeps one grab in flight and reads its result one piece later.
+  long long pw = 0, pi = 0, nst = 0;
+  int grabbed = 0;
+  int piece = blockIdx.x;
+  if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + (int)gridDim.x;
+  while (true) {
+    if (piece >= sp.total) break;
+    Hdr ph;
+    piece_header<KIND>(p, sp, piece, ph, ve_tab);
+    const int pr = piece - (ph.v * p.RB + ph.rb) * sp.ppr;
+    const int c_first = (pr * p.C) / sp.ppr;
+    const int c_last = ((pr + 1) * p.C) / sp.ppr;
+    for (int c = c_first; c < c_last; ++c) {
+      // before the dependency resolves, fill at most one ring of weight-only stages
+      if (!waited && prefetched == p.nstages) {
+        pdl_wait();
+        pdl_trigger();
+        waited = true;
+        for (int s = 0; s < prefetched; ++s) {
+          uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
+          const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
+          issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
+        }
+      }
+      const long long tw0 = clock64();
+      if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, 200)) return;
+      const long long tw1 = clock64();
+      pw += tw1 - tw0;
+      uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
+      Hdr h = ph;
+      chunk_header<KIND>(p, c, c_first, c_last, h);
+      if (lane == 0) {
+        *reinterpret_cast<Hdr*>(sb) = h;
+        mbar_arrive_expect_tx(&full[stage], KindTraits<KIND>::kTileBytes + h.act_bytes);
+        bulk_g2s(sb + kHdrBytes, weight_src<KIND>(p, h), KindTraits<KIND>::kTileBytes, &full[stage]);
+      }
+      __syncwarp();
+      if (waited)
+        issue_act<KIND>(p, h, sb + p.act_off, &full[stage], lane, slot_tab);
+      else
+        ++prefetched;
+      if (++stage == p.nstages) {
+        stage = 0;
+        ephase ^= 1;
+      }
+      pi += clock64() - tw1;
+      ++nst;
+    }
+    piece = __shfl_sync(0xffffffffu, grabbed, 0);
+    if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + (int)gridDim.x;
+  }
+  if (!waited) {
+    pdl_wait();
+    pdl_trigger();
+    for (int s = 0; s < prefetched; ++s) {
+      uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
+      const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
+      issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
+    }
+  }
+  if (p.trace && lane == 0) {
+    unsigned long long* tr = p.trace + (size_t)blockIdx.x * kTraceStride;
+    tr[11] = (unsigned long long)pw;
+    tr[12] = (unsigned long long)pi;
+    tr[13] = (unsigned long long)nst;
+  }
+  // end marker
+  if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, 200)) return;
+  if (lane == 0) {
+    uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
+    reinterpret_cast<Hdr*>(sb)->flags = HDR_END;
+    mbar_arrive(&full[stage]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// consumer math
+
+template <int NT>
+__device__ __forceinline__ void zero_acc(float (&acc)[NT][4]) {
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[t][q] = 0.f;
+}
+
+// bf16 weights x bf16 token rows (x): RL, SGU
+template <int NT>
+__device__ __forceinline__ void mma_dense_x(const Params& p, const Hdr& h, const uint8_t* tile,
+                                            const uint8_t* act, float (&acc)[NT][4],
+                                            float (&acc2)[NT][4], int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  // loads first and unconditionally (rows past ntok read stale stage bytes and
+  // are zeroed by a select), then the MMAs
+  uint4 a[2][2];
+#pragma unroll
+  for (int b = 0; b < 2; ++b)
+#pragma unroll
+    for (int s = 0; s < 2; ++s) a[b][s] = lds128(tile + ((warp * 2 + b) * 2 + s) * 512 + lane * 16);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int tok = 8 * t + g;
+    const bool tv = tok < h.ntok;
+    const uint8_t* row = act + (tv ? tok : 0) * p.act_stride + 8 * tig * 2;
+    uint4 bv[2] = {lds128(row), lds128(row + 64)};
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (b < h.nb) {
+        const uint32_t A0[4] = {a[b][0].x, a[b][0].y, a[b][0].z, a[b][0].w};
+        const uint32_t A1[4] = {a[b][1].x, a[b][1].y, a[b][1].z, a[b][1].w};
+        const uint4 v = tv ? bv[b] : make_uint4(0, 0, 0, 0);
+        mma_bf16(acc[t], A0, v.x, v.y);
+        mma_bf16(acc2[t], A1, v.z, v.w);
+      }
+    }
+  }
+}
+
+// MXFP4 weights x f16-MX activation records: EGU, EDN.  Every shared-memory
+// load of the stage is issued first and unconditionally (the stage buffer is
+// always full size; rows and blocks outside the valid range are masked by
+// selects), so the loads overlap and the MMAs of the 8 K-blocks interleave.
+template <int NT>
+__device__ __forceinline__ void mma_mx(const Params& p, const Hdr& h, const uint8_t* tile,
+                                       const uint8_t* act, float (&acc)[NT][4], int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  const uint4 sc = lds128(tile + kMxCodeBytes + (warp * 8 + g) * 16);
+  const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+  uint4 cw[4];
+#pragma unroll
+  for (int bp = 0; bp < 4; ++bp) cw[bp] = lds128(tile + (warp * 4 + bp) * 512 + lane * 16);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int tok = 8 * t + g;
+    const bool tv = tok < h.ntok;
+    const int c0 = 8 * t + 2 * tig;
+    const bool v0 = c0 < h.ntok, v1 = c0 + 1 < h.ntok;
+    const uint8_t* arow = act + (tv ? tok : 0) * p.act_stride + tig * 16;
+    const float* s0 = reinterpret_cast<const float*>(act + (v0 ? c0 : 0) * p.act_stride + 512);
+    const float* s1 = reinterpret_cast<const float*>(act + (v1 ? c0 + 1 : 0) * p.act_stride + 512);
+    uint4 bv[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) bv[b] = lds128(arow + b * 64);
+    const float4 s0a = *reinterpret_cast<const float4*>(s0);
+    const float4 s0b = *reinterpret_cast<const float4*>(s0 + 4);
+    const float4 s1a = *reinterpret_cast<const float4*>(s1);
+    const float4 s1b = *reinterpret_cast<const float4*>(s1 + 4);
+    const float sa0[8] = {s0a.x, s0a.y, s0a.z, s0a.w, s0b.x, s0b.y, s0b.z, s0b.w};
+    const float sa1[8] = {s1a.x, s1a.y, s1a.z, s1a.w, s1b.x, s1b.y, s1b.z, s1b.w};
+    const int nb = h.nb == 8 ? 8 : h.nb;  // full chunks: the guard below folds away
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      if (h.nb == 8 || b < nb) {
+        uint32_t A0[4], A1[4];
+        const uint4 w4 = cw[b >> 1];
+        e2m1x8_to_f16x2x4((b & 1) ? w4.z : w4.x, A0);
+        e2m1x8_to_f16x2x4((b & 1) ? w4.w : w4.y, A1);
+        const float sw0 = e8m0_to_float((scw[b >> 2] >> (8 * (b & 3))) & 0xFF);
+        const float sw1 = e8m0_to_float((scw[2 + (b >> 2)] >> (8 * (b & 3))) & 0xFF);
+        const uint32_t b0 = tv ? bv[b].x : 0u, b1 = tv ? bv[b].y : 0u;
+        const uint32_t b2 = tv ? bv[b].z : 0u, b3 = tv ? bv[b].w : 0u;
+        const float a0 = v0 ? sa0[b] : 0.f, a1 = v1 ? sa1[b] : 0.f;
+        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16(tmp, A0, b0, b1);
+        mma_f16(tmp, A1, b2, b3);
+        acc[t][0] = fmaf(sw0 * a0, tmp[0], acc[t][0]);
+        acc[t][1] = fmaf(sw0 * a1, tmp[1], acc[t][1]);
+        acc[t][2] = fmaf(sw1 * a0, tmp[2], acc[t][2]);
+        acc[t][3] = fmaf(sw1 * a1, tmp[3], acc[t][3]);
+      }
+    }
+  }
+}
+
+// TAIL, few tokens: form every token's whole activation once per CTA.  Token
+// b's record holds bf16 hi values for k in [0, res_k), then the lo parts.
+// k < C_lat*64 is the combine c = sum_j w_j y_j (zero past L); the rest is h_s.
+__device__ __forceinline__ void build_resident(const Params& p, uint8_t* res, int tid) {
+  const int K = p.topk, KR = p.res_k, klat = p.C_lat * 64;
+  const int groups = p.B * (KR / 8);
+  for (int gi = tid; gi < groups; gi += kConsumerThreads) {
+    const int b = gi / (KR / 8), k0 = (gi % (KR / 8)) * 8;
+    float v[8];
+    if (k0 < klat) {
+      // K <= 16: compile-time slots keep everything in registers, loads first
+      float4 ya[16], yb[16];
+      float wj[16];
+      const float* ybase = p.y + ((long long)(k0 >> 6) * p.ld_slots + (long long)b * K) * 64 + (k0 & 63);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j < K) {
+          wj[j] = __ldcg(p.wts + b * K + j);
+          ya[j] = __ldcg(reinterpret_cast<const float4*>(ybase + j * 64));
+          yb[j] = __ldcg(reinterpret_cast<const float4*>(ybase + j * 64 + 4));
+        } else {
+          wj[j] = 0.f;
+          ya[j] = yb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v[0] = fmaf(wj[j], ya[j].x, v[0]);
+        v[1] = fmaf(wj[j], ya[j].y, v[1]);
+        v[2] = fmaf(wj[j], ya[j].z, v[2]);
+        v[3] = fmaf(wj[j], ya[j].w, v[3]);
+        v[4] = fmaf(wj[j], yb[j].x, v[4]);
+        v[5] = fmaf(wj[j], yb[j].y, v[5]);
+        v[6] = fmaf(wj[j], yb[j].z, v[6]);
+        v[7] = fmaf(wj[j], yb[j].w, v[7]);
+      }
+      if (k0 >= p.L) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = 0.f;
+      }
+    } else {
+      const int ks = k0 - klat;
+      if (ks < p.KS) {
+        const float* hb = p.h_s + ((long long)(ks >> 6) * p.B + b) * 64 + (ks & 63);
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(hb));
+        const float4 c = __ldcg(reinterpret_cast<const float4*>(hb + 4));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = 0.f;
+      }
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      hi[u] = pack_bf16x2(v[2 * u], v[2 * u + 1]);
+      lo[u] = pack_bf16x2(v[2 * u] - bf16_lo_to_float(hi[u]), v[2 * u + 1] - bf16_hi_to_float(hi[u]));
+    }
+    uint8_t* rec = res + (size_t)b * p.res_stride;
+    *reinterpret_cast<uint4*>(rec + k0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(rec + KR * 2 + k0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+template <int NT>
+__device__ __forceinline__ void mma_tail_resident(const Params& p, const Hdr& h, const uint8_t* tile,
+                                                  const uint8_t* res, float (&acc)[NT][4],
+                                                  float (&acc2)[NT][4], int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  const int kbase = h.chunk * kDenseChunkK;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    if (b < h.nb) {
+      const uint4 a0 = lds128(tile + ((warp * 2 + b) * 2 + 0) * 512 + lane * 16);
+      const uint4 a1 = lds128(tile + ((warp * 2 + b) * 2 + 1) * 512 + lane * 16);
+      const uint32_t A0[4] = {a0.x, a0.y, a0.z, a0.w};
+      const uint32_t A1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int tok = 8 * t + g;
+        const bool tv = tok < h.ntok;
+        const uint8_t* rec = res + (size_t)(h.tok0 + (tv ? tok : 0)) * p.res_stride +
+                             (kbase + 32 * b + 8 * tig) * 2;
+        uint4 bh = lds128(rec), bl = lds128(rec + p.res_k * 2);
+        if (!tv) bh = bl = make_uint4(0, 0, 0, 0);
+        mma_bf16(acc[t], A0, bh.x, bh.y);
+        mma_bf16(acc2[t], A1, bh.z, bh.w);
+        mma_bf16(acc[t], A0, bl.x, bl.y);
+        mma_bf16(acc2[t], A1, bl.z, bl.w);
+      }
+    }
+  }
+}
+
+// TAIL: build the activation tile (combine of y, or h_s) as bf16 hi + lo in a
+// transform buffer, then bf16 MMAs against W_out / W_sd.
+template <int NT>
+__device__ __forceinline__ void mma_tail(const Params& p, const Hdr& h, const uint8_t* tile,
+                                         const uint8_t* act, uint8_t* tbuf, float (&acc)[NT][4],
+                                         float (&acc2)[NT][4], int warp, int lane, int tid) {
+  constexpr int kTStride = 320;  // bytes per token row: 64 bf16 hi, 64 bf16 lo, padding
+  const int K = p.topk;
+  const bool lat = h.chunk < p.C_lat;
+  for (int idx = tid; idx < h.ntok * 16; idx += kConsumerThreads) {
+    const int tk = idx >> 4, q = idx & 15;
+    float4 v;
+    if (lat) {
+      const float* yrow = reinterpret_cast<const float*>(act) + (tk * K) * 64 + q * 4;
+      const float* wrow = p.wts + (long long)(h.tok0 + tk) * K;
+      v = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < K; ++j) {
+        const float wj = wrow[j];
+        const float4 yv = *reinterpret_cast<const float4*>(yrow + j * 64);
+        v.x = fmaf(wj, yv.x, v.x);
+        v.y = fmaf(wj, yv.y, v.y);
+        v.z = fmaf(wj, yv.z, v.z);
+        v.w = fmaf(wj, yv.w, v.w);
+      }
+    } else {
+      v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(act) + tk * 64 + q * 4);
+    }
+    const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
+    const uint32_t l01 = pack_bf16x2(v.x - bf16_lo_to_float(h01), v.y - bf16_hi_to_float(h01));
+    const uint32_t l23 = pack_bf16x2(v.z - bf16_lo_to_float(h23), v.w - bf16_hi_to_float(h23));
+    *reinterpret_cast<uint2*>(tbuf + tk * kTStride + q * 8) = make_uint2(h01, h23);
+    *reinterpret_cast<uint2*>(tbuf + tk * kTStride + 128 + q * 8) = make_uint2(l01, l23);
+  }
+  named_sync(1, kConsumerThreads);
+  const int g = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    if (b < h.nb) {
+      const uint4 a0 = lds128(tile + ((warp * 2 + b) * 2 + 0) * 512 + lane * 16);
+      const uint4 a1 = lds128(tile + ((warp * 2 + b) * 2 + 1) * 512 + lane * 16);
+      const uint32_t A0[4] = {a0.x, a0.y, a0.z, a0.w};
+      const uint32_t A1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int tok = 8 * t + g;
+        uint4 bh = make_uint4(0, 0, 0, 0), bl = make_uint4(0, 0, 0, 0);
+        if (tok < h.ntok) {
+          bh = lds128(tbuf + tok * kTStride + (32 * b + 8 * tig) * 2);
+          bl = lds128(tbuf + tok * kTStride + 128 + (32 * b + 8 * tig) * 2);
+        }
+        mma_bf16(acc[t], A0, bh.x, bh.y);
+        mma_bf16(acc2[t], A1, bh.z, bh.w);
+        mma_bf16(acc[t], A0, bl.x, bl.y);
+        mma_bf16(acc2[t], A1, bl.z, bl.w);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// epilogues
+
+// f16 "MX" store: values of a 32-wide block of the activation index share one
+// power-of-two scale per token, chosen so the block's largest magnitude lands
+// in [2^14, 2^15).  `wpb` warps own one 32-wide block.  Each thread provides
+// up to two rows (r0 = g, r1 = g + 8) per token column.
+__device__ __forceinline__ void mx_scale_of(float amax, float& s, float& inv) {
+  if (!(amax > 0.f)) {
+    s = 1.f;
+    inv = 1.f;
+    if (amax != amax) s = amax;  // NaN propagates through the scale
+    return;
+  }
+  int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+  int se = ex - 14;
+  se = se < -100 ? -100 : (se > 127 ? 127 : se);
+  s = __uint_as_float((uint32_t)(se + 127) << 23);
+  inv = __uint_as_float((uint32_t)(127 - se) << 23);
+}
+
+template <int NT, int ROWS>
+__device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int warp, int lane,
+                                            int wpb, int ntok, float* amax_s,
+                                            uint8_t* const (&rec)[NT][2], const int (&idx)[2],
+                                            bool row_valid0, bool row_valid1) {
+  // val[t][c][r]: token column 8t + 2tig + c, row r (r < ROWS)
+  const int g = lane >> 2, tig = lane & 3;
+  float m[NT][2];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      float a = row_valid0 ? fabsf(val[t][c][0]) : 0.f;
+      if (ROWS > 1 && row_valid1) a = fmaxf(a, fabsf(val[t][c][1]));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
+      m[t][c] = a;
+    }
+  if (g == 0) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) amax_s[warp * (NT * 8) + 8 * t + 2 * tig + c] = m[t][c];
+  }
+  named_sync(1, kConsumerThreads);
+  const int w0 = (warp / wpb) * wpb;
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int col = 8 * t + 2 * tig + c;
+      if (col >= ntok) continue;
+      float a = 0.f;
+      for (int ww = w0; ww < w0 + wpb; ++ww) a = fmaxf(a, amax_s[ww * (NT * 8) + col]);
+      float s, inv;
+      mx_scale_of(a, s, inv);
+      uint8_t* r = rec[t][c];
+#pragma unroll
+      for (int rr = 0; rr < ROWS; ++rr) {
+        const bool ok = rr == 0 ? row_valid0 : row_valid1;
+        if (!ok) continue;
+        const int i = idx[rr] & (kMxChunkK - 1);
+        *reinterpret_cast<uint16_t*>(r + i * 2) =
+            (uint16_t)(pack_f16x2(val[t][c][rr] * inv, 0.f) & 0xFFFF);
+      }
+      if (g == 0 && warp == w0 && row_valid0) {
+        const int i = idx[0] & (kMxChunkK - 1);
+        *reinterpret_cast<float*>(r + 512 + 4 * (i >> 5)) = s;
+      }
+    }
+  named_sync(1, kConsumerThreads);
+}
+
+__device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, int* wtot, int tid,
+                                          int warp, int lane);
+
+template <int KIND, int NT>
+__device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
+                         int* sm_flag, const int* slot_tab, int tid, int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  if (KIND == KIND_RL) {
+    if (h.rb < p.RB_router) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+          const int col = 8 * t + 2 * tig + (q & 1);
+          const int e = h.rb * kRowsPerBlock + row;
+          if (e < p.E && col < p.B) p.logits[(long long)col * p.E + e] = acc[t][q];
+        }
+      // every thread's logits precede thread 0's release (barrier cumulativity)
+      named_sync(1, kConsumerThreads);
+      if (p.trace && tid == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 19] = global_ns();
+      if (tid == 0) *sm_flag = (atom_add_acqrel(p.router_done, 1) == p.RB_router - 1);
+      named_sync(1, kConsumerThreads);
+      if (*sm_flag) {
+        if (p.trace && tid == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 4] = global_ns();
+        route_tokens(p, scratch, sm_flag + 16, tid, warp, lane);  // 16 ints of warp totals
+        if (p.trace && tid == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 5] = global_ns();
+        if (tid == 0) *p.router_done = 0;
+      }
+      named_sync(1, kConsumerThreads);
+    } else {
+      const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
+      const int l0 = (h.rb - p.RB_router) * kRowsPerBlock + 16 * warp + g;
+      const int idx[2] = {l0, l0 + 8};
+      float val[NT][2][2];
+      uint8_t* rec[NT][2];
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          val[t][c][0] = acc[t][c];
+          val[t][c][1] = acc[t][2 + c];
+          const int col = 8 * t + 2 * tig + c;
+          rec[t][c] = p.z_mx + ((long long)(col < p.B ? col : 0) * cz + (l0 >> 8)) * kActRecBytes;
+        }
+      store_f16mx<NT, 2>(val, warp, lane, 2, p.B, reinterpret_cast<float*>(scratch), rec, idx,
+                         l0 < p.L, l0 + 8 < p.L);
+    }
+  } else if (KIND == KIND_SGU) {
+    const int i = 64 * h.rb + 8 * warp + g;
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int col = 8 * t + 2 * tig + c;
+        if (col < p.B && i < p.Is)
+          p.h_s[((long long)(i >> 6) * p.B + col) * 64 + (i & 63)] = silu(acc[t][c]) * acc[t][2 + c];
+      }
+  } else if (KIND == KIND_EGU) {
+    const int i = 64 * h.rb + 8 * warp + g;
+    const int idx[2] = {i, i};
+    float val[NT][2][2];
+    uint8_t* rec[NT][2];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        val[t][c][0] = silu(acc[t][c]) * acc[t][2 + c];
+        val[t][c][1] = 0.f;
+        const int col = 8 * t + 2 * tig + c;
+        const int pos = h.tok0 + (col < h.ntok ? col : 0);
+        rec[t][c] = p.h_mx + ((long long)(i >> 8) * p.ld_slots + pos) * kActRecBytes;
+      }
+    store_f16mx<NT, 1>(val, warp, lane, 4, h.ntok, reinterpret_cast<float*>(scratch), rec, idx,
+                       i < p.I, false);
+  } else if (KIND == KIND_EDN) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int l = h.rb * kRowsPerBlock + 16 * warp + ((q & 2) ? g + 8 : g);
+        const int col = 8 * t + 2 * tig + (q & 1);
+        if (col < h.ntok && l < p.L) {
+          const int slot = slot_tab[h.tok0 + col];
+          p.y[((long long)(l >> 6) * p.ld_slots + slot) * 64 + (l & 63)] = acc[t][q];
+        }
+      }
+  } else {  // TAIL
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int n = h.rb * kRowsPerBlock + 16 * warp + ((q & 2) ? g + 8 : g);
+        const int col = 8 * t + 2 * tig + (q & 1);
+        if (col < h.ntok && n < p.H)
+          p.out[(long long)(h.tok0 + col) * p.H + n] =
+              (uint16_t)(pack_bf16x2(acc[t][q], 0.f) & 0xFFFF);
+      }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// top-k routing and per-expert token lists (one CTA, 256 threads); the
+// per-token selection is warp_topk (topk.cuh).
+
+__device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, int* wtot, int tid,
+                                          int warp, int lane) {
+  const int E = p.E, K = p.topk, B = p.B;
+  const int tg = p.tg > 0 ? p.tg : 1;
+  int* cnt = reinterpret_cast<int*>(scratch);  // [E] slots per expert
+  int* fill = cnt + E;                          // [E] placement cursor
+  int* off = fill + E;                          // [E] first sorted position
+  int* ids_s = off + E;                         // [B*K]
+  unsigned long long* tr = (p.trace && tid == 0) ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
+  for (int i = tid; i < E; i += kConsumerThreads) {
+    cnt[i] = 0;
+    fill[i] = 0;
+  }
+  named_sync(1, kConsumerThreads);
+  if (tr) tr[16] = global_ns();
+  // Few tokens: P warps share a token (each selects within a slice of the
+  // experts, one warp merges); 8 or more tokens: one warp per token.
+  const int P = B >= kConsumerWarps ? 1 : kConsumerWarps / B;  // B * P <= 8 warps
+  if (P == 1) {
+    for (int b = warp; b < B; b += kConsumerWarps) {
+      int sel_id;
+      float sel_w;
+      warp_topk(p.logits + (long long)b * E, E, K, p.score_fn, p.bias, p.renorm, p.routed_scale,
+                lane, sel_id, sel_w);
+      if (lane < K) {
+        p.ids[b * K + lane] = sel_id;
+        p.wts[b * K + lane] = sel_w;
+        ids_s[b * K + lane] = sel_id;
+        atomicAdd(&cnt[sel_id], 1);
+      }
+    }
+  } else {
+    // candidates after the token table: [B][P][K] TopkCand, then [B][P] partials
+    TopkCand* cand = reinterpret_cast<TopkCand*>(
+        reinterpret_cast<uint8_t*>(ids_s) + ((B * K * 4 + 15) & ~15));
+    float2* part = reinterpret_cast<float2*>(cand + B * P * K);
+    if (warp < B * P) {
+      const int b = warp / P, q = warp % P;
+      const int e0 = (int)((long long)q * E / P), e1 = (int)((long long)(q + 1) * E / P);
+      TopkCand c;
+      float smax, ssum;
+      warp_topk_slice_any(p.logits + (long long)b * E, p.bias, e0, e1, K, p.score_fn, lane, c, smax,
+                          ssum);
+      if (lane < K) cand[(b * P + q) * K + lane] = c;
+      if (lane == 0) part[b * P + q] = make_float2(smax, ssum);
+    }
+    named_sync(1, kConsumerThreads);
+    if (warp < B) {
+      const int b = warp;
+      int sel_id;
+      float sel_w;
+      warp_topk_merge(cand + b * P * K, part + b * P, P, K, E, p.score_fn, p.renorm,
+                      p.routed_scale, lane, sel_id, sel_w);
+      if (lane < K) {
+        p.ids[b * K + lane] = sel_id;
+        p.wts[b * K + lane] = sel_w;
+        ids_s[b * K + lane] = sel_id;
+        atomicAdd(&cnt[sel_id], 1);
+      }
+    }
+  }
+  named_sync(1, kConsumerThreads);
+  if (tr) tr[17] = global_ns();
+  // block-wide exclusive scan of (slots, token groups) per expert; thread t
+  // owns experts 4t .. 4t+3 (E <= 1024)
+  int c[4], gsz[4], sc = 0, sg = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 4 * tid + i;
+    c[i] = e < E ? cnt[e] : 0;
+    gsz[i] = (c[i] + tg - 1) / tg;
+    sc += c[i];
+    sg += gsz[i];
+  }
+  int ic = sc, ig = sg;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int uc = __shfl_up_sync(0xffffffffu, ic, o);
+    const int ug = __shfl_up_sync(0xffffffffu, ig, o);
+    if (lane >= o) {
+      ic += uc;
+      ig += ug;
+    }
+  }
+  if (lane == 31) {
+    wtot[warp] = ic;
+    wtot[8 + warp] = ig;
+  }
+  named_sync(1, kConsumerThreads);
+  int bc = ic - sc, bg = ig - sg;  // exclusive within the warp
+  for (int w = 0; w < warp; ++w) {
+    bc += wtot[w];
+    bg += wtot[8 + w];
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 4 * tid + i;
+    if (e < E) {
+      off[e] = bc;
+      for (int gi = 0; gi < gsz[i]; ++gi) {
+        VExpert ve;
+        ve.expert = e;
+        ve.start = bc + gi * tg;
+        ve.count = min(tg, c[i] - gi * tg);
+        ve.pad = 0;
+        if (bg + gi < p.ve_max) p.ve[bg + gi] = ve;
+      }
+    }
+    bc += c[i];
+    bg += gsz[i];
+  }
+  if (tid == kConsumerThreads - 1) *p.nve = bg < p.ve_max ? bg : p.ve_max;
+  named_sync(1, kConsumerThreads);
+  if (tr) tr[18] = global_ns();
+  for (int s = tid; s < B * K; s += kConsumerThreads) {
+    const int e = ids_s[s];
+    const int pos = off[e] + atomicAdd(&fill[e], 1);
+    p.slots_sorted[pos] = s;
+  }
+  named_sync(1, kConsumerThreads);
+}
+
+// ---------------------------------------------------------------------------
+// consumer warps
+
+// Split-K partial sums: [piece][token column][128 rows] floats, only the
+// columns that hold tokens are written.
+template <int NT>
+__device__ __forceinline__ void write_partial(const Params& p, int piece, int ntok,
+                                              const float (&acc)[NT][4], int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  float* base = p.partials + (long long)piece * (NT * 8 * kRowsPerBlock);
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = 8 * t + 2 * tig + (q & 1);
+      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+      if (col < ntok) base[col * kRowsPerBlock + row] = acc[t][q];
+    }
+}
+
+// Sum the row block's pieces in piece order (the same order whatever CTA ran
+// them, so the result is deterministic).
+template <int NT>
+__device__ __forceinline__ void sum_partials(const Params& p, const Hdr& h, float (&acc)[NT][4],
+                                             int warp, int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  const long long first = (long long)(h.v * p.RB + h.rb) * h.ppr;
+  const long long stride = NT * 8 * kRowsPerBlock;
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = 8 * t + 2 * tig + (q & 1);
+      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+      float sum = 0.f;
+      if (col < h.ntok) {
+        const float* src = p.partials + first * stride + col * kRowsPerBlock + row;
+        int pr = 0;
+        for (; pr + 8 <= h.ppr; pr += 8) {
+          float v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (pr + u) * stride);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) sum += v[u];
+        }
+        for (; pr < h.ppr; ++pr) sum += __ldcg(src + pr * stride);
+      }
+      acc[t][q] = sum;
+    }
+}
+
+// Same sums for up to 32 token columns, spread over all consumer threads
+// (one (column, row) value each, 16 loads in flight) and handed back through
+// shared memory.
+template <int NT>
+__device__ __forceinline__ void sum_partials_wide(const Params& p, const Hdr& h, float (&acc)[NT][4],
+                                                  float* rs, int tid, int warp, int lane) {
+  const long long first = (long long)(h.v * p.RB + h.rb) * h.ppr;
+  const long long stride = NT * 8 * kRowsPerBlock;
+  const int n = h.ntok * kRowsPerBlock;
+  for (int i = tid; i < n; i += kConsumerThreads) {
+    const float* src = p.partials + first * stride + i;  // i = col * 128 + row
+    float sum = 0.f;
+    int pr = 0;
+    for (; pr + 16 <= h.ppr; pr += 16) {
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = __ldcg(src + (pr + u) * stride);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) sum += v[u];
+    }
+    for (; pr < h.ppr; ++pr) sum += __ldcg(src + pr * stride);
+    rs[i] = sum;
+  }
+  named_sync(1, kConsumerThreads);
+  const int g = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = 8 * t + 2 * tig + (q & 1);
+      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+      acc[t][q] = col < h.ntok ? rs[col * kRowsPerBlock + row] : 0.f;
+    }
+  named_sync(1, kConsumerThreads);
+}
+
+template <int KIND, int NT>
+__device__ __forceinline__ void finalize(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
+                         int* sm_flag, const int* slot_tab, int tid, int warp, int lane) {
+  if (h.ntok <= 32)
+    sum_partials_wide<NT>(p, h, acc, reinterpret_cast<float*>(scratch), tid, warp, lane);
+  else
+    sum_partials<NT>(p, h, acc, warp, lane);
+  if (tid == 0) p.counters[h.v * p.RB + h.rb] = 0;  // ready for the next launch
+  epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+}
+
+template <int KIND, int NT>
+__device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, uint64_t* empty,
+                         uint8_t* scratch, int* sm_flag, const int* slot_tab, int warp, int lane) {
+  const int tid = warp * 32 + lane;
+  int stage = 0;
+  uint32_t phase = 0;
+  int nbuf = 0;
+  // two accumulator sets (k16 steps 0 and 1) so consecutive MMAs do not wait
+  // on each other; folded together when a piece ends
+  float acc[NT][4], acc2[NT][4];
+  zero_acc(acc);
+  zero_acc(acc2);
+  // A piece whose ticket (finalize counter) is still in flight: thread 0
+  // issues the atomic after the piece's partials are written and reads its
+  // result only at the next piece end, so nobody waits on the round trip.
+  bool pend = false;
+  Hdr pend_h;
+  int ticket = 0;
+  int* tflag = sm_flag + 4;  // two alternating slots
+  int tslot = 0;
+  // activations, routing tables and partial sums of the previous kernel are
+  // read only after the dependency has resolved; the next kernel may then be
+  // scheduled (it cannot overtake this one's own predecessor)
+  pdl_wait();
+  pdl_trigger();
+  uint8_t* res = stage_base - p.stage_off + p.res_off;  // shared-memory base + offset
+  if (KIND == KIND_TAIL && p.res_off) {
+    build_resident(p, res, tid);
+    named_sync(1, kConsumerThreads);
+  }
+  unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
+  int n_pieces = 0, n_fin = 0;
+  long long c_wait = 0, c_comp = 0, c_end = 0, t_a = clock64();
+  while (true) {
+    if (!mbar_wait_bounded(&full[stage], phase, p.err, ERR_WAIT_FULL)) break;
+    long long t_b = clock64();
+    c_wait += t_b - t_a;
+    uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
+    const Hdr h = *reinterpret_cast<const Hdr*>(sb);
+    if (tr && tid == 0 && n_pieces == 0 && (h.flags & HDR_FIRST)) tr[6] = global_ns();
+    if (h.flags & HDR_END) break;
+    if (h.flags & HDR_FIRST) {
+      zero_acc(acc);
+      zero_acc(acc2);
+    }
+    const uint8_t* tile = sb + kHdrBytes;
+    const uint8_t* act = sb + p.act_off;
+    if (KIND == KIND_RL || KIND == KIND_SGU) {
+      mma_dense_x<NT>(p, h, tile, act, acc, acc2, warp, lane);
+    } else if (KIND == KIND_EGU || KIND == KIND_EDN) {
+      mma_mx<NT>(p, h, tile, act, acc, warp, lane);
+    } else if (p.res_off) {
+      mma_tail_resident<NT>(p, h, tile, res, acc, acc2, warp, lane);
+    } else {
+      uint8_t* tbuf = scratch + 4096 + (nbuf & 1) * (16 * 320);
+      ++nbuf;
+      mma_tail<NT>(p, h, tile, act, tbuf, acc, acc2, warp, lane, tid);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (++stage == p.nstages) {
+      stage = 0;
+      phase ^= 1;
+    }
+    t_a = clock64();
+    c_comp += t_a - t_b;
+    if (!(h.flags & HDR_LAST)) continue;
+    ++n_pieces;
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[t][q] += acc2[t][q];
+
+    if (h.ppr == 1) {
+      ++n_fin;
+      epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+      continue;
+    }
+    write_partial<NT>(p, h.piece, h.ntok, acc, warp, lane);
+    if (tid == 0 && pend) tflag[tslot] = (ticket == pend_h.ppr - 1);
+    named_sync(1, kConsumerThreads);  // every warp's partials precede thread 0's release
+    const bool fin = pend && tflag[tslot] != 0;
+    if (tid == 0) ticket = atom_add_acqrel(p.counters + h.v * p.RB + h.rb, 1);
+    const Hdr prev = pend_h;
+    pend_h = h;
+    pend = true;
+    tslot ^= 1;
+    if (fin) {
+      ++n_fin;
+      const unsigned long long t0 = tr ? global_ns() : 0ull;
+      finalize<KIND, NT>(p, prev, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+      if (tr && tid == 0) tr[7] += global_ns() - t0;
+    }
+    const long long t_c = clock64();
+    c_end += t_c - t_a;
+    t_a = t_c;
+  }
+  if (pend) {
+    if (tid == 0) tflag[tslot] = (ticket == pend_h.ppr - 1);
+    named_sync(1, kConsumerThreads);
+    if (tflag[tslot] != 0) {
+      ++n_fin;
+      finalize<KIND, NT>(p, pend_h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+    }
+  }
+  if (tr && tid == 0) {
+    tr[2] = (unsigned long long)n_pieces;
+    tr[3] = (unsigned long long)n_fin;
+    tr[8] = (unsigned long long)c_wait;
+    tr[9] = (unsigned long long)c_comp;
+    tr[10] = (unsigned long long)c_end;
+  }
+}
+
+// ---------------------------------------------------------------------------
+
+template <int KIND, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_kernel(const __grid_constant__ Params p) {
+  // shared memory: [0,128) full barriers, [128,256) empty barriers,
+  // [256,512) flags, [scratch_off, ...) scratch, [table_off, ...) routing
+  // tables (expert kernels), [stage_off, ...) ring
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMaxStages;
+  int* sm_flag = reinterpret_cast<int*>(smem + 256);
+  uint8_t* scratch = smem + p.scratch_off;
+  uint8_t* stages = smem + p.stage_off;
+  uint8_t* tables = smem + p.table_off;
+  const int* slot_tab = reinterpret_cast<const int*>(tables + (size_t)p.ve_max * sizeof(VExpert));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Ctl* ctl = p.ctl;
+  if (p.trace && threadIdx.x == 0) {
+    unsigned long long* tr = p.trace + (size_t)blockIdx.x * kTraceStride;
+    tr[0] = global_ns();
+    for (int i = 2; i < kTraceStride; ++i) tr[i] = 0;
+    tr[14] = smid();
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.nstages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == kConsumerWarps) {
+    producer<KIND>(p, ctl, stages, tables, full, empty, lane);
+  } else {
+    consumer<KIND, NT>(p, stages, full, empty, scratch, sm_flag, slot_tab, warp, lane);
+  }
+  __syncthreads();
+  if (p.trace && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 1] = global_ns();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&ctl->exits, 1) == (int)gridDim.x - 1) {
+      ctl->cursor = 0;
+      ctl->exits = 0;
+      __threadfence();
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host-side launch of one instantiation
+
+template <int KIND, int NT>
+static int launch_one(const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
+  auto kfn = moe_kernel<KIND, NT>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return (int)cudaLaunchKernelEx(&cfg, kfn, p);
+}
+
+template <int KIND, int NT>
+static int set_attr(size_t bytes) {
+  return (int)cudaFuncSetAttribute(moe_kernel<KIND, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)bytes);
+}
+
+// Token tiles (NT) each kind is built for: dense kinds up to 16 (128 tokens),
+// expert kinds up to 4 (groups of 32), the tail up to 2 (groups of 16).
+template <int KIND>
+static int launch_kind_nt(int nt, const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
+  constexpr bool kDense = (KIND == KIND_RL || KIND == KIND_SGU);
+  switch (nt) {
+    case 1: return launch_one<KIND, 1>(p, grid, smem, s, pdl);
+    case 2: return launch_one<KIND, 2>(p, grid, smem, s, pdl);
+    case 4:
+      if constexpr (KIND != KIND_TAIL) return launch_one<KIND, 4>(p, grid, smem, s, pdl);
+      break;
+    case 8:
+      if constexpr (kDense) return launch_one<KIND, 8>(p, grid, smem, s, pdl);
+      break;
+    case 16:
+      if constexpr (kDense) return launch_one<KIND, 16>(p, grid, smem, s, pdl);
+      break;
+    default: break;
+  }
+  return (int)cudaErrorInvalidValue;
+}
+
+template <int KIND>
+static int set_attr_kind(size_t bytes) {
+  int e = set_attr<KIND, 1>(bytes) | set_attr<KIND, 2>(bytes);
+  if constexpr (KIND != KIND_TAIL) e |= set_attr<KIND, 4>(bytes);
+  if constexpr (KIND == KIND_RL || KIND == KIND_SGU) e |= set_attr<KIND, 8>(bytes) | set_attr<KIND, 16>(bytes);
+  return e;
+}
+
+}  // namespace moe
