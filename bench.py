@@ -243,7 +243,7 @@ def run_ours(args):
         w_np, dw = _device_instance(shape, inst, torch)
         if inst == 0:
             host_w0 = w_np
-        p = moe.MoePlan(moe.config_from_shape(shape, shared_sms=args.shared_sms), device=local)
+        p = moe.MoePlan(moe.config_from_shape(shape), device=local)
         p.load(dw, stream)
         del dw
         plans.append(p)
@@ -336,7 +336,7 @@ def run_ours(args):
     H, L, E, I, Is = shape.hidden, shape.latent, shape.num_experts, shape.expert_inter, shape.shared_inter
     per_expert_gu = 2 * I * L // 2 + 2 * I * L // 32
     per_expert_dn = L * I // 2 + L * I // 32
-    kern_bytes = {"router_latent": 2 * H * (E + L), "shared_gate_up": 4 * H * Is,
+    kern_bytes = {"dense_front": 2 * H * (E + L + 2 * Is),
                   "expert_gate_up": mean_distinct * per_expert_gu,
                   "expert_down": mean_distinct * per_expert_dn,
                   "latent_tail": 2 * L * H + 2 * Is * H}
@@ -401,7 +401,7 @@ def run_ours(args):
                     "d2h_bytes_per_step": B * H * 2},
             "gpu_launches": args.steps * info.kernels_per_forward,
             "clocks": clk,
-            "plan": {"main_ctas": info.main_ctas, "shared_ctas": info.shared_ctas},
+            "plan": {"front_ctas": info.front_ctas, "expert_ctas": info.expert_ctas},
             "parity_spot_check": spot,
         }
         print(json.dumps(line), flush=True)
@@ -420,7 +420,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="b1", choices=["tiny", "b1", "b8", "b64", "b128"])
-    ap.add_argument("--shared-sms", type=int, default=0)
     ap.add_argument("--instances", type=int, default=4,
                     help="resident weight instances rotated per step (4 keeps every step out of L2)")
     ap.add_argument("--no-cpu", action="store_true")

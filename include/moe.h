@@ -75,7 +75,6 @@ typedef struct moe_config {
   int32_t score_fn;     /* MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID */
   int32_t renormalize;  /* 1: combine weights divided by their sum over the k chosen */
   float routed_scale;   /* factor applied to every combine weight (1.0 = none) */
-  int32_t shared_sms;   /* CTAs given to the side-stream shared expert, 0 = automatic */
 } moe_config;
 
 /*
@@ -116,8 +115,8 @@ typedef struct moe_plan_s *moe_plan;
 typedef struct moe_plan_info {
   int32_t device;
   int32_t num_sms;
-  int32_t main_ctas;        /* CTAs of the main-stream kernels while the side stream runs */
-  int32_t shared_ctas;      /* CTAs of the side-stream shared-expert kernel */
+  int32_t front_ctas;       /* CTAs streaming the router / latent / shared gate-up rows */
+  int32_t expert_ctas;      /* CTAs of each routed-expert kernel */
   int64_t packed_bytes;     /* library-owned packed weights */
   int64_t workspace_bytes;  /* library-owned activations, routing metadata, partial sums */
   int64_t dense_weight_bytes;      /* bf16 bytes one forward streams regardless of routing */
@@ -126,8 +125,8 @@ typedef struct moe_plan_info {
 } moe_plan_info;
 
 /*
- * Create a plan on `device`: checks the shape, allocates packed-weight storage,
- * workspace, a side stream and events.  *out receives the plan.
+ * Create a plan on `device`: checks the shape, allocates packed-weight storage
+ * and workspace.  *out receives the plan.
  * Errors: INVALID_ARG (null, bad shape), UNSUPPORTED (no sm_100 device, shape
  * beyond the limits above), OOM, CUDA.
  */
@@ -144,9 +143,9 @@ MOE_API moe_status moe_load_weights(moe_plan p, const moe_weights *w, void *stre
  * out[B][H] (bf16, device) = block(x[B][H] bf16, device).  B = num_tokens,
  * 1..max_tokens.  x and out must be 16-byte aligned and must not overlap.
  * Asynchronous on `stream`: allocates nothing, does no host synchronisation,
- * may be captured into a CUDA graph.  Internally forks the shared expert onto
- * the plan's side stream and joins it back before returning control of
- * `stream`.  Errors: INVALID_ARG, NOT_LOADED, CUDA (launch failure).
+ * may be captured into a CUDA graph.  Every kernel runs on `stream`, each a
+ * programmatic dependent launch of the one before.  Errors: INVALID_ARG,
+ * NOT_LOADED, CUDA (launch failure).
  */
 MOE_API moe_status moe_forward(moe_plan p, const void *x, int32_t num_tokens, void *out, void *stream);
 
@@ -187,16 +186,16 @@ MOE_API moe_status moe_get_plan_info(moe_plan p, moe_plan_info *info);
  * each of its kernels with CUDA events on the stream that kernel runs on and
  * waits for them before returning (so profiled forwards are synchronous and
  * must not be captured into a graph).  moe_get_profile writes the accumulated
- * milliseconds per kernel in launch-kind order {router+latent, shared gate/up,
- * expert gate/up, expert down, latent tail} to ms[0..4] and the number of
- * profiled forwards to *count, then clears both.
+ * milliseconds per kernel in launch order {dense front (router, latent, shared
+ * gate/up, top-k), expert gate/up, expert down, latent tail} to ms[0..3] and
+ * the number of profiled forwards to *count, then clears both.
  */
 MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
 
 /*
  * Per-CTA timeline of the most recent forward, for measurement only; exists
  * when the plan was created with the environment variable MOE_TRACE set
- * (else MOE_ERR_UNSUPPORTED).  host receives count = 5 * num_sms * 24 uint64:
+ * (else MOE_ERR_UNSUPPORTED).  host receives count = 4 * num_sms * 24 uint64:
  * for kernel kind k (launch order as in moe_get_profile) and CTA c, the 24
  * values at (k * num_sms + c) * 24 are {start ns, end ns, pieces, finalizes,
  * top-k start ns, top-k end ns, first stage ready ns, finalize ns, consumer

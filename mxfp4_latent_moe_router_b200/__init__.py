@@ -27,7 +27,9 @@ ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forwar
                "moe_last_routing", "moe_debug_fetch", "moe_sync_status", "moe_get_plan_info",
                "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile",
                "moe_route_noalloc", "moe_debug_trace"]
-KERNEL_NAMES = ["router_latent", "shared_gate_up", "expert_gate_up", "expert_down", "latent_tail"]
+# kernel kinds in launch order: the dense front kernel streams the router,
+# latent-projection and shared-expert gate/up rows (and runs top-k)
+KERNEL_NAMES = ["dense_front", "expert_gate_up", "expert_down", "latent_tail"]
 
 
 class MoeError(RuntimeError):
@@ -41,8 +43,7 @@ class moe_config(ctypes.Structure):
                 ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("expert_inter", ctypes.c_int32), ("shared_inter", ctypes.c_int32),
                 ("max_tokens", ctypes.c_int32), ("score_fn", ctypes.c_int32),
-                ("renormalize", ctypes.c_int32), ("routed_scale", ctypes.c_float),
-                ("shared_sms", ctypes.c_int32)]
+                ("renormalize", ctypes.c_int32), ("routed_scale", ctypes.c_float)]
 
 
 class moe_weights(ctypes.Structure):
@@ -53,7 +54,7 @@ class moe_weights(ctypes.Structure):
 
 class moe_plan_info(ctypes.Structure):
     _fields_ = [("device", ctypes.c_int32), ("num_sms", ctypes.c_int32),
-                ("main_ctas", ctypes.c_int32), ("shared_ctas", ctypes.c_int32),
+                ("front_ctas", ctypes.c_int32), ("expert_ctas", ctypes.c_int32),
                 ("packed_bytes", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64),
                 ("dense_weight_bytes", ctypes.c_int64), ("expert_weight_bytes", ctypes.c_int64),
                 ("kernels_per_forward", ctypes.c_int32)]
@@ -169,7 +170,7 @@ def moe_set_profiling(plan: int, enable: bool) -> None:
 
 def moe_get_profile(plan: int):
     """-> (milliseconds per kernel kind as a dict, number of profiled forwards)."""
-    ms = (ctypes.c_float * 5)()
+    ms = (ctypes.c_float * len(KERNEL_NAMES))()
     n = ctypes.c_int32()
     _check(load_library().moe_get_profile(plan, ms, ctypes.byref(n)), "moe_get_profile")
     return dict(zip(KERNEL_NAMES, list(ms))), n.value
@@ -186,9 +187,9 @@ def moe_route_noalloc(x, router_w, router_bias, num_tokens: int, hidden: int, nu
 
 
 def moe_debug_trace(plan: int, num_sms: int):
-    """Per-CTA timeline of the last forward: uint64 array [5 kinds][num_sms][24]."""
+    """Per-CTA timeline of the last forward: uint64 array [4 kinds][num_sms][24]."""
     import numpy as np
-    a = np.zeros((5, num_sms, 24), np.uint64)
+    a = np.zeros((len(KERNEL_NAMES), num_sms, 24), np.uint64)
     _check(load_library().moe_debug_trace(plan, a.ctypes.data, a.size), "moe_debug_trace")
     return a
 
@@ -200,11 +201,11 @@ def moe_plan_destroy(plan: int) -> None:
 
 # ---- convenience wrapper ---------------------------------------------------
 
-def config_from_shape(shape, max_tokens: int | None = None, shared_sms: int = 0) -> moe_config:
+def config_from_shape(shape, max_tokens: int | None = None) -> moe_config:
     return moe_config(shape.hidden, shape.latent, shape.num_experts, shape.top_k,
                       shape.expert_inter, shape.shared_inter,
                       shape.tokens if max_tokens is None else max_tokens, shape.score_fn,
-                      shape.renormalize, float(shape.routed_scale), shared_sms)
+                      shape.renormalize, float(shape.routed_scale))
 
 
 def weights_to_device(w: dict, device: str = "cuda"):

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["moe_kernels.cu", "moe_k_rl.cu", "moe_k_sgu.cu", "moe_k_egu.cu", "moe_k_edn.cu",
+SOURCES = ["moe_kernels.cu", "moe_k_front.cu", "moe_k_egu.cu", "moe_k_edn.cu",
            "moe_k_tail.cu", "moe_pack.cu", "moe_api.cu", "moe_static.cu"]
 HEADERS = ["ptx.cuh", "layout.cuh", "engine.cuh", "topk.cuh", "moe_engine.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

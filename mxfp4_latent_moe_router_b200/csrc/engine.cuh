@@ -7,12 +7,11 @@
 namespace moe {
 
 enum Kind : int {
-  KIND_RL = 0,    // router logits + latent projection (+ top-k by the last router row block)
-  KIND_SGU = 1,   // shared expert gate/up + SwiGLU (side stream)
-  KIND_EGU = 2,   // routed experts gate/up + SwiGLU, MXFP4
-  KIND_EDN = 3,   // routed experts down projection, MXFP4
-  KIND_TAIL = 4,  // weighted combine + W_out, plus shared down projection -> out
-  KIND_COUNT = 5
+  KIND_FRONT = 0,  // x . [W_r | W_in | W_sg,W_su]: router logits, latent z, shared h_s
+  KIND_EGU = 1,    // routed experts gate/up + SwiGLU, MXFP4
+  KIND_EDN = 2,    // routed experts down projection, MXFP4
+  KIND_TAIL = 3,   // weighted combine + W_out, plus shared down projection -> out
+  KIND_COUNT = 4
 };
 
 // Per-kernel scheduling state in device memory, zero between launches: the
@@ -28,6 +27,7 @@ enum : int {
   ERR_WAIT_FULL = 0,
   ERR_WAIT_EMPTY = 1,
   ERR_NAN_SCALE = 2,
+  ERR_WAIT_ROUTE = 3,  // the routing tables never became ready
 };
 
 struct VExpert {  // one token group of one routed expert
@@ -46,7 +46,10 @@ struct Params {
   int PPR;            // pieces per row block (0: computed on the device, EGU/EDN)
   int target_pieces;  // EGU/EDN: aim for at least this many pieces
   int C_lat;          // TAIL: chunks covering L; chunks >= C_lat cover I_s
-  int RB_router;      // RL: row blocks holding router rows
+  int RB_router;      // FRONT: leading row blocks holding router rows
+  int RB_lat;         // FRONT: row blocks of the latent projection (after the router's);
+                      // the shared expert's gate/up row blocks follow
+  int route_cta;      // FRONT: 1 when the grid's last CTA is the routing CTA (no pieces)
   int tg;             // tokens per group (EGU/EDN/TAIL)
   int KL;             // K extent of the chunked dimension (for ragged last chunk)
   int KS;             // TAIL: K extent of the shared part (I_s)
@@ -84,6 +87,11 @@ struct Params {
   unsigned long long* trace;
   int* counters;   // finalize tickets per (virtual matrix, row block)
   int* router_done;
+  // 1 once this forward's routing tables are published (release by the
+  // routing CTA); the expert kernels stream their experts' tiles as soon as
+  // it is set, before their own dependency resolves.  Cleared by the tail,
+  // which no reader of it can still be running beside.
+  int* route_ready;
   float* partials;
   int* err;
 };

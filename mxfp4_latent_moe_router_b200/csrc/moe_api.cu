@@ -1,8 +1,8 @@
 // moe_api.cu -- the C ABI declared in include/moe.h.
 //
 // A plan owns: packed weights, the per-forward workspace (activations, routing
-// tables, split-K partial sums, scheduling counters), a side stream and two
-// events.  moe_forward only enqueues work; all memory exists from
+// tables, split-K partial sums, scheduling counters and flags).  moe_forward
+// only enqueues work on the caller's stream; all memory exists from
 // moe_plan_create on.
 #include <cuda_runtime.h>
 
@@ -50,13 +50,12 @@ struct moe_plan_s {
   int last_B = 0;
 
   KindGeom g[KIND_COUNT];
-  int RB_router = 0, C_lat = 0, tail_tg = kTailTg, ve_max = 0;
+  int RB_router = 0, RB_lat = 0, C_lat = 0, tail_tg = kTailTg, ve_max = 0;
 
   std::vector<void*> allocs;
   size_t packed_bytes = 0, workspace_bytes = 0;
 
-  uint8_t* w_rl = nullptr;
-  uint8_t* w_sgu = nullptr;
+  uint8_t* w_front = nullptr;
   uint8_t* w_egu = nullptr;
   uint8_t* w_edn = nullptr;
   uint8_t* w_tail = nullptr;
@@ -75,14 +74,13 @@ struct moe_plan_s {
   Ctl* ctl = nullptr;  // [KIND_COUNT]
   int* counters[KIND_COUNT] = {};
   int* router_done = nullptr;
+  int* route_ready = nullptr;
   float* partials[KIND_COUNT] = {};
   size_t partial_cap[KIND_COUNT] = {};  // floats
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* out_stage = nullptr;
 
-  cudaStream_t side = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 
   // tuning knobs read once at plan creation (environment): pieces each CTA
   // should get on average, and whether kernels chain with programmatic
@@ -140,35 +138,22 @@ bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 
 
 // token geometry of one forward
 struct FwdGeom {
-  int nt_rl, nt_e, nt_tail, tail_tg;
-  int main_grid, side_grid, tail_grid;
+  int nt_front, nt_e, nt_tail, tail_tg;
+  int front_grid, front_workers, tail_grid, expert_grid;
 };
 
 FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   FwdGeom f;
-  f.nt_rl = pow2_at_least((B + 7) / 8);
+  f.nt_front = pow2_at_least((B + 7) / 8);
   f.nt_e = pow2_at_least((std::min(B, kExpertTg) + 7) / 8);
   f.tail_tg = p->tail_tg;
   f.nt_tail = pow2_at_least((std::min(B, p->tail_tg) + 7) / 8);
-  const moe_config& c = p->cfg;
-  int side = 0;
-  if (c.shared_inter > 0) {
-    if (c.shared_sms > 0) {
-      side = c.shared_sms;
-    } else {
-      // share the SMs in proportion to the bytes each stream has to move
-      const double E = c.num_experts, k = c.top_k;
-      const double distinct = E * (1.0 - std::pow(1.0 - k / E, (double)B));
-      const double sgu = 2.0 * c.hidden * 2.0 * c.shared_inter;
-      const double rl = 2.0 * c.hidden * (double)(c.num_experts + c.latent);
-      const double ex = distinct * (double)(p->g[KIND_EGU].weight_bytes + p->g[KIND_EDN].weight_bytes);
-      side = (int)std::lround(p->num_sms * sgu / (sgu + rl + ex));
-    }
-    side = std::max(4, std::min(side, p->num_sms / 2));
-  }
-  f.side_grid = side;
-  f.main_grid = p->num_sms - side;
+  // every kernel takes every SM (one CTA each); the front kernel's last CTA
+  // is the routing CTA and streams nothing
+  f.front_grid = p->num_sms;
+  f.front_workers = p->num_sms - 1;
   f.tail_grid = p->num_sms;
+  f.expert_grid = p->num_sms;
   return f;
 }
 
@@ -194,7 +179,7 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int 
   const int stage_off = kStageOff + s.table_bytes + res_bytes;
   int act = 0;
   s.act_stride = 0;
-  if (kind == KIND_RL || kind == KIND_SGU) {
+  if (kind == KIND_FRONT) {
     s.act_stride = 192;
     act = 8 * nt * s.act_stride;
   } else if (kind == KIND_EGU || kind == KIND_EDN) {
@@ -206,9 +191,9 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int 
   const int tile = (kind == KIND_EGU || kind == KIND_EDN) ? kMxTileBytes : kDenseTileBytes;
   s.act_off = kHdr + tile;
   s.stage_bytes = ((kHdr + tile + act) + 127) / 128 * 128;
-  // one CTA per SM: the main-stream kernels, the side-stream kernel and a
-  // kernel launched early by programmatic dependent launch then never share an
-  // SM, and the whole shared memory goes to the ring
+  // one CTA per SM: a running kernel and the next one, launched early by
+  // programmatic dependent launch, never share an SM, and the whole shared
+  // memory goes to the ring
   const int budget = kBigSmem;
   // enough bytes in flight to saturate HBM (about 6 x 16 KB per SM); more only
   // lengthens the queues every other memory request waits behind
@@ -251,8 +236,8 @@ Params base_params(const moe_plan_s* p, int B) {
   q.nve = p->nve;
   q.ve_max = p->ve_max;
   q.router_done = p->router_done;
+  q.route_ready = p->route_ready;
   q.err = p->err;
-  q.RB_router = p->RB_router;
   q.C_lat = p->C_lat;
   q.KS = c.shared_inter;
   q.scratch_off = kScratchOff;
@@ -275,8 +260,13 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   q.stage_off = s.stage_off;
   q.matrix_bytes = (long long)p->g[kind].weight_bytes;
   switch (kind) {
-    case KIND_RL: q.wt = p->w_rl; q.tg = kExpertTg; break;  // top-k groups expert tokens
-    case KIND_SGU: q.wt = p->w_sgu; break;
+    case KIND_FRONT:  // its routing CTA groups expert tokens by tg
+      q.wt = p->w_front;
+      q.tg = kExpertTg;
+      q.RB_router = p->RB_router;
+      q.RB_lat = p->RB_lat;
+      q.route_cta = 1;
+      break;
     case KIND_EGU: q.wt = p->w_egu; q.tg = kExpertTg; break;
     case KIND_EDN: q.wt = p->w_edn; q.tg = kExpertTg; break;
     default: q.wt = p->w_tail; q.tg = p->tail_tg; break;
@@ -296,13 +286,9 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     size_t pieces = 0;
     int nt = 1;
     const KindGeom& g = p->g[kind];
-    if (kind == KIND_RL) {
-      nt = f.nt_rl;
-      pieces = (size_t)g.RB * ppr_for(target_pieces(f.main_grid, nt), g.RB, g.C);
-    } else if (kind == KIND_SGU) {
-      nt = f.nt_rl;
-      if (!p->cfg.shared_inter) continue;
-      pieces = (size_t)g.RB * ppr_for(target_pieces(f.side_grid, nt), g.RB, g.C);
+    if (kind == KIND_FRONT) {
+      nt = f.nt_front;
+      pieces = (size_t)g.RB * ppr_for(target_pieces(f.front_workers, nt), g.RB, g.C);
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
@@ -311,7 +297,7 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
       nt = f.nt_e;
       // PPR > 1 only while (virtual experts x row blocks) < target, so the
       // pieces that need partial storage stay below 2 x target
-      pieces = 2 * (size_t)target_pieces(f.main_grid, nt) + g.RB;
+      pieces = 2 * (size_t)target_pieces(f.expert_grid, nt) + g.RB;
     }
     best = std::max(best, pieces * (size_t)nt * 1024);
   }
@@ -334,7 +320,7 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
 moe_status check_cfg(const moe_config* c) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (c->hidden <= 0 || c->latent <= 0 || c->num_experts <= 0 || c->expert_inter <= 0 ||
-      c->shared_inter < 0 || c->top_k <= 0 || c->max_tokens <= 0 || c->shared_sms < 0)
+      c->shared_inter < 0 || c->top_k <= 0 || c->max_tokens <= 0)
     return MOE_ERR_INVALID_ARG;
   if (c->hidden % 32 || c->latent % 32 || c->expert_inter % 32 || c->shared_inter % 32)
     return MOE_ERR_INVALID_ARG;
@@ -368,17 +354,15 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
 
   const moe_config& c = *cfg;
   const int H = c.hidden, L = c.latent, E = c.num_experts, I = c.expert_inter, Is = c.shared_inter;
+  // the front kernel's row blocks: router (first, so the routing starts
+  // early), latent projection, shared expert gate/up (64 + 64 rows a block)
   p->RB_router = ceil_div(E, kRowsPerBlock);
-  KindGeom& rl = p->g[KIND_RL];
-  rl.RB = p->RB_router + ceil_div(L, kRowsPerBlock);
-  rl.C = ceil_div(H, kDenseChunkK);
-  rl.KL = H;
-  rl.weight_bytes = (size_t)rl.RB * rl.C * kDenseTileBytes;
-  KindGeom& sg = p->g[KIND_SGU];
-  sg.RB = ceil_div(Is, 64);
-  sg.C = ceil_div(H, kDenseChunkK);
-  sg.KL = H;
-  sg.weight_bytes = (size_t)sg.RB * sg.C * kDenseTileBytes;
+  p->RB_lat = ceil_div(L, kRowsPerBlock);
+  KindGeom& fr = p->g[KIND_FRONT];
+  fr.RB = p->RB_router + p->RB_lat + ceil_div(Is, 64);
+  fr.C = ceil_div(H, kDenseChunkK);
+  fr.KL = H;
+  fr.weight_bytes = (size_t)fr.RB * fr.C * kDenseTileBytes;
   KindGeom& eg = p->g[KIND_EGU];
   eg.RB = ceil_div(I, 64);
   eg.C = ceil_div(L, kMxChunkK);
@@ -402,12 +386,8 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->ve_max = std::min(E, slots) + ceil_div(slots, kExpertTg) + 1;
 
   void* v;
-  TRY(alloc(p, &v, rl.weight_bytes, true));
-  p->w_rl = (uint8_t*)v;
-  if (Is > 0) {
-    TRY(alloc(p, &v, sg.weight_bytes, true));
-    p->w_sgu = (uint8_t*)v;
-  }
+  TRY(alloc(p, &v, fr.weight_bytes, true));
+  p->w_front = (uint8_t*)v;
   TRY(alloc(p, &v, (size_t)E * eg.weight_bytes, true));
   p->w_egu = (uint8_t*)v;
   TRY(alloc(p, &v, (size_t)E * ed.weight_bytes, true));
@@ -440,10 +420,10 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->nve = (int*)v;
   p->router_done = p->nve + 1;
   p->err = p->nve + 2;
+  p->route_ready = p->nve + 3;
   p->ctl = reinterpret_cast<Ctl*>((uint8_t*)v + 1024);
   CUDA_TRY(cudaMemset(v, 0, 1024 + sizeof(Ctl) * KIND_COUNT));
-  const int cnt_n[KIND_COUNT] = {rl.RB, std::max(sg.RB, 1), p->ve_max * eg.RB, p->ve_max * ed.RB,
-                                 ceil_div(maxB, 1) * tl.RB};
+  const int cnt_n[KIND_COUNT] = {fr.RB, p->ve_max * eg.RB, p->ve_max * ed.RB, maxB * tl.RB};
   for (int k = 0; k < KIND_COUNT; ++k) {
     TRY(alloc(p, &v, sizeof(int) * cnt_n[k], false));
     p->counters[k] = (int*)v;
@@ -462,9 +442,6 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
   p->out_stage = (uint16_t*)v;
 
-  CUDA_TRY(cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking));
-  CUDA_TRY(cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming));
-  CUDA_TRY(cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming));
   for (int k = 0; k < KIND_COUNT; ++k)
     for (int j = 0; j < 2; ++j) CUDA_TRY(cudaEventCreate(&p->ev_prof[k][j]));
   CUDA_TRY(cudaDeviceSynchronize());
@@ -483,9 +460,6 @@ void destroy_impl(moe_plan p) {
   DeviceGuard g(p->device);
   cudaDeviceSynchronize();
   for (void* a : p->allocs) cudaFree(a);
-  if (p->side) cudaStreamDestroy(p->side);
-  if (p->ev_fork) cudaEventDestroy(p->ev_fork);
-  if (p->ev_join) cudaEventDestroy(p->ev_join);
   for (int k = 0; k < KIND_COUNT; ++k)
     for (int j = 0; j < 2; ++j)
       if (p->ev_prof[k][j]) cudaEventDestroy(p->ev_prof[k][j]);
@@ -498,52 +472,37 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   g_pieces_per_cta = p->pieces_per_cta;
   const FwdGeom f = fwd_geom(p, B);
   const int tail_tg_eff = std::min(B, p->tail_tg);
-  const bool shared = c.shared_inter > 0;
   Params base = base_params(p, B);
   base.x = (const uint16_t*)x;
   base.out = (uint16_t*)out;
 
-  if (shared) {
-    CUDA_TRY(cudaEventRecord(p->ev_fork, s));
-    CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_fork, 0));
-    Params q = base;
-    const SmemGeom sm = smem_geom(KIND_SGU, f.nt_rl, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
-    set_kind(q, p, KIND_SGU, sm);
-    q.PPR = ppr_for(target_pieces(f.side_grid, f.nt_rl), q.RB, q.C);
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_SGU][0], p->side));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_SGU, f.nt_rl, q, f.side_grid, sm.total, p->side, false));
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_SGU][1], p->side));
-    CUDA_TRY(cudaEventRecord(p->ev_join, p->side));
-  }
+  // One stream, each kernel a programmatic dependent of the one before:
+  //   front (router, latent, shared gate/up) -> expert gate/up -> expert down -> tail.
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_RL, f.nt_rl, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
-    set_kind(q, p, KIND_RL, sm);
-    q.PPR = ppr_for(target_pieces(f.main_grid, f.nt_rl), q.RB, q.C);
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_RL][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_RL, f.nt_rl, q, f.main_grid, sm.total, s, p->use_pdl));
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_RL][1], s));
+    const SmemGeom sm = smem_geom(KIND_FRONT, f.nt_front, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
+    set_kind(q, p, KIND_FRONT, sm);
+    q.PPR = ppr_for(target_pieces(f.front_workers, f.nt_front), q.RB, q.C);
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][0], s));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_FRONT, f.nt_front, q, f.front_grid, sm.total, s, p->use_pdl));
+    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][1], s));
   }
   {
     Params q = base;
     const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EGU, sm);
-    q.target_pieces = target_pieces(f.main_grid, f.nt_e);
+    q.target_pieces = target_pieces(f.expert_grid, f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.main_grid, sm.total, s, p->use_pdl));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
   }
-  // join the side stream here: the down projection cannot prefetch anything
-  // before its dependency resolves anyway, while the tail keeps its
-  // programmatic edge to the down projection and prefetches W_out early
-  if (shared) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));
   {
     Params q = base;
     const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EDN, sm);
-    q.target_pieces = target_pieces(f.main_grid, f.nt_e);
+    q.target_pieces = target_pieces(f.expert_grid, f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.main_grid, sm.total, s, p->use_pdl));
+    CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
   }
   {
@@ -568,7 +527,6 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   p->last_B = B;
   if (p->profiling) {
     for (int k = 0; k < KIND_COUNT; ++k) {
-      if (k == KIND_SGU && !shared) continue;
       CUDA_TRY(cudaEventSynchronize(p->ev_prof[k][1]));
       float ms = 0.f;
       CUDA_TRY(cudaEventElapsedTime(&ms, p->ev_prof[k][0], p->ev_prof[k][1]));
@@ -657,18 +615,19 @@ moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
   p->loaded = false;
   const int H = c.hidden, L = c.latent, E = c.num_experts, I = c.expert_inter, Is = c.shared_inter;
   CUDA_TRY(cudaMemsetAsync(p->err, 0, sizeof(int), s));
-  // RL: router rows then latent rows, both from [H][N] tensors
-  const KindGeom& rl = p->g[KIND_RL];
-  CUDA_TRY((cudaError_t)launch_pack_dense(w->router_w, H, E, 0, p->RB_router, rl.C, E, p->w_rl, s,
-                                          nullptr, 0, 0));
-  CUDA_TRY((cudaError_t)launch_pack_dense(
-      w->w_in, H, L, 0, rl.RB - p->RB_router, rl.C, L,
-      p->w_rl + (size_t)p->RB_router * rl.C * kDenseTileBytes, s, nullptr, 0, 0));
-  if (Is > 0) {
-    const KindGeom& sg = p->g[KIND_SGU];
-    CUDA_TRY((cudaError_t)launch_pack_dense(w->sh_gate, H, Is, 1, sg.RB, sg.C, Is, p->w_sgu, s,
+  // front tiles: router row blocks, then latent, then shared gate/up, all
+  // from [H][N] tensors
+  const KindGeom& fr = p->g[KIND_FRONT];
+  const size_t rb_bytes = (size_t)fr.C * kDenseTileBytes;
+  CUDA_TRY((cudaError_t)launch_pack_dense(w->router_w, H, E, 0, p->RB_router, fr.C, E, p->w_front,
+                                          s, nullptr, 0, 0));
+  CUDA_TRY((cudaError_t)launch_pack_dense(w->w_in, H, L, 0, p->RB_lat, fr.C, L,
+                                          p->w_front + p->RB_router * rb_bytes, s, nullptr, 0, 0));
+  if (Is > 0)
+    CUDA_TRY((cudaError_t)launch_pack_dense(w->sh_gate, H, Is, 1, fr.RB - p->RB_router - p->RB_lat,
+                                            fr.C, Is,
+                                            p->w_front + (p->RB_router + p->RB_lat) * rb_bytes, s,
                                             w->sh_up, 0, 0));
-  }
   const KindGeom& tl = p->g[KIND_TAIL];
   CUDA_TRY((cudaError_t)launch_pack_dense(w->w_out, L, H, 2, tl.RB, tl.C, H, p->w_tail, s,
                                           Is > 0 ? w->sh_down : w->w_out, Is, p->C_lat));
@@ -827,8 +786,8 @@ moe_status moe_get_plan_info(moe_plan p, moe_plan_info* info) {
   const FwdGeom f = fwd_geom(p, p->cfg.max_tokens);
   info->device = p->device;
   info->num_sms = p->num_sms;
-  info->main_ctas = f.main_grid;
-  info->shared_ctas = f.side_grid;
+  info->front_ctas = f.front_workers;
+  info->expert_ctas = f.expert_grid;
   info->packed_bytes = (int64_t)p->packed_bytes;
   info->workspace_bytes = (int64_t)p->workspace_bytes;
   const moe_config& c = p->cfg;
@@ -837,7 +796,7 @@ moe_status moe_get_plan_info(moe_plan p, moe_plan_info* info) {
       6LL * c.hidden * c.shared_inter;
   info->expert_weight_bytes =
       (3LL * c.expert_inter * c.latent) / 2 + (3LL * c.expert_inter * c.latent) / 32;
-  info->kernels_per_forward = c.shared_inter > 0 ? 5 : 4;
+  info->kernels_per_forward = KIND_COUNT;
   return MOE_OK;
 }
 

@@ -1,7 +1,7 @@
-// moe_engine.cuh -- the five kernels of one latent-MoE decode step on sm_100a
+// moe_engine.cuh -- the four kernels of one latent-MoE decode step on sm_100a
 // (device code; each kind is instantiated in its own moe_k_<kind>.cu).
 //
-// One engine serves all five: a CTA of 8 consumer warps and 1 producer warp.
+// One engine serves all four: a CTA of 8 consumer warps and 1 producer warp.
 // The producer grabs "pieces" (a row block of 128 output rows x a run of K
 // chunks) from a global cursor and streams each chunk's weight tile plus the
 // activation rows it multiplies into a ring of shared-memory stages with bulk
@@ -15,15 +15,18 @@
 // lets a CTA that does extra epilogue work fall behind without stalling the
 // others.
 //
-//   KIND_RL   x . [W_r | W_in] -> router logits (fp32) and latent z (f16 MX);
-//             the CTA that finalises the last router row block runs top-k and
-//             builds the per-expert token lists while the rest of the grid is
-//             still streaming W_in.
+//   KIND_FRONT x . [W_r | W_in | W_sg,W_su] in one weight-streaming pass over
+//             every SM: router logits (fp32), latent z (f16 MX) and the shared
+//             expert's h_s = silu(g) * u (fp32).  The router row blocks come
+//             first; the grid's last CTA takes no pieces and runs top-k and
+//             the per-expert token lists as soon as they are summed, while
+//             the other CTAs still stream the rest.
 //             (page "Hyper Optimizing Kimi K3 in vLLM: Moving Fast and
-//              Responsibly", section 从算子之间找时间: router scores and the
-//              latent input projection as one matmul.)
-//   KIND_SGU  x . [W_sg | W_su] -> h_s = silu(g) * u (fp32), side stream.
-//             (same section: the shared expert on its own stream.)
+//              Responsibly", section 从算子之间找时间: the router scores and the
+//              latent input projection as one matmul, and the shared expert
+//              overlapping the routing.  One GPU has no ranks to split the
+//              matmul over, and a second stream would only contend for the
+//              same HBM, so the shared expert's rows join the same pass.)
 //   KIND_EGU  per routed expert, z . [Wg | Wu] (MXFP4) -> h = silu(g) * u (f16 MX)
 //   KIND_EDN  per routed expert, h . Wd (MXFP4) -> y (fp32, per token slot)
 //   KIND_TAIL c = sum_j w_j y_j formed from y while staging the activation
@@ -33,8 +36,11 @@
 //              the MXFP4 top-k finalize fused into the latent-tail kernel.)
 //
 // Only static weights are fetched before griddepcontrol.wait; activations are
-// fetched after it (page 1, section 更快的代码需要更有针对性的验证: an
-// activation load hoisted above a synchronisation wait was a real bug).
+// fetched after it (page "Hyper Optimizing Kimi K3 in vLLM: Moving Fast and
+// Responsibly", section 更快的代码需要更有针对性的验证: an activation load
+// hoisted above a synchronisation wait was a real bug).  The expert kernels
+// may also read the routing tables before it, but only after acquiring the
+// flag that publishes them.
 #pragma once
 #include <cuda_runtime.h>
 
@@ -64,8 +70,8 @@ struct KindTraits {
   static constexpr bool kMx = (KIND == KIND_EGU || KIND == KIND_EDN);
   static constexpr int kTileBytes = kMx ? kMxTileBytes : kDenseTileBytes;
   static constexpr int kChunkK = kMx ? kMxChunkK : kDenseChunkK;
-  // weights may be fetched before the previous kernel finishes
-  static constexpr bool kPrefetchWeights = (KIND == KIND_RL || KIND == KIND_TAIL);
+  // every kind streams one ring of weight tiles before its dependency resolves
+  static constexpr bool kPrefetchWeights = true;
   static constexpr bool kDynamicSpace = (KIND == KIND_EGU || KIND == KIND_EDN);
 };
 
@@ -140,7 +146,7 @@ __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, i
   h.rb = rem / sp.ppr;
   h.ppr = sp.ppr;
   h.expert = 0;
-  if (KIND == KIND_RL || KIND == KIND_SGU) {
+  if (KIND == KIND_FRONT) {
     h.ntok = p.B;
     h.tok0 = 0;
   } else if (KIND == KIND_TAIL) {
@@ -161,7 +167,7 @@ __device__ __forceinline__ void chunk_header(const Params& p, int c, int c_first
   h.chunk = c;
   h.nb = chunk_blocks<KIND>(p, c);
   int ab;
-  if (KIND == KIND_RL || KIND == KIND_SGU)
+  if (KIND == KIND_FRONT)
     ab = h.ntok * h.nb * 64;
   else if (KIND == KIND_EGU || KIND == KIND_EDN)
     ab = h.ntok * kActRecBytes;
@@ -182,7 +188,7 @@ __device__ __forceinline__ const uint8_t* weight_src(const Params& p, const Hdr&
 template <int KIND>
 __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t* act, uint64_t* bar,
                                           int lane, const int* slot_tab) {
-  if (KIND == KIND_RL || KIND == KIND_SGU) {
+  if (KIND == KIND_FRONT) {
     const int bytes = h.nb * 64;
     for (int r = lane; r < h.ntok; r += 32)
       bulk_g2s(act + r * p.act_stride, p.x + (long long)r * p.H + h.chunk * kDenseChunkK, bytes, bar);
@@ -211,6 +217,17 @@ __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t
   }
 }
 
+// Bounded wait (about a second) until *flag != 0, with acquire semantics for
+// the calling thread; false (and an error bit) if it never is.
+__device__ __forceinline__ bool wait_flag(const int* flag, int* err, int err_bit, int lane) {
+  for (uint32_t i = 0; i < (1u << 22); ++i) {
+    if (ld_acquire(flag) != 0) return true;
+    __nanosleep(256);
+  }
+  if (lane == 0) atomicOr(err, 1 << err_bit);
+  return false;
+}
+
 template <int KIND>
 __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t* tables,
                          uint64_t* full, uint64_t* empty, int lane) {
@@ -230,11 +247,22 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   // loads and the count load below are independent and overlap.
   VExpert* ve_tab = reinterpret_cast<VExpert*>(tables);
   int* slot_tab = reinterpret_cast<int*>(tables + (size_t)p.ve_max * sizeof(VExpert));
-  if (KindTraits<KIND>::kDynamicSpace) {
-    for (int i = lane; i < p.ve_max; i += 32) ve_tab[i] = p.ve[i];
-    for (int i = lane; i < p.ld_slots; i += 32) slot_tab[i] = p.slots_sorted[i];
+  // The routing is published by the front kernel's routing CTA while the
+  // front kernel may still run (every CTA of it is resident before this
+  // kernel can launch, so the wait ends): wait for its flag, then read the
+  // tables and start streaming the chosen experts' tiles before this kernel's
+  // own dependency resolves.
+  const bool route_ok = KindTraits<KIND>::kDynamicSpace ? wait_flag(p.route_ready, p.err, ERR_WAIT_ROUTE, lane) : true;
+  if (KindTraits<KIND>::kDynamicSpace && route_ok) {
+    // L2 reads: the tables were written by another kernel that may still run
+    for (int i = lane; i < p.ve_max; i += 32) {
+      const int4 v = __ldcg(reinterpret_cast<const int4*>(p.ve + i));
+      ve_tab[i] = VExpert{v.x, v.y, v.z, v.w};
+    }
+    for (int i = lane; i < p.ld_slots; i += 32) slot_tab[i] = __ldcg(p.slots_sorted + i);
   }
   sp = make_space<KIND>(p);
+  if (!route_ok) sp.total = 0;  // no pieces: straight to the end marker
   __syncwarp();
 
   // every CTA starts on piece blockIdx.x (no round trip before the first
@@ -242,8 +270,9 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   // keeps one grab in flight and reads its result one piece later.
   long long pw = 0, pi = 0, nst = 0;
   int grabbed = 0;
+  const int workers = (int)gridDim.x - (KIND == KIND_FRONT ? p.route_cta : 0);
   int piece = blockIdx.x;
-  if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + (int)gridDim.x;
+  if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
   while (true) {
     if (piece >= sp.total) break;
     Hdr ph;
@@ -288,7 +317,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       ++nst;
     }
     piece = __shfl_sync(0xffffffffu, grabbed, 0);
-    if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + (int)gridDim.x;
+    if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
   }
   if (!waited) {
     pdl_wait();
@@ -331,8 +360,9 @@ __device__ __forceinline__ void mma_dense_x(const Params& p, const Hdr& h, const
                                             const uint8_t* act, float (&acc)[NT][4],
                                             float (&acc2)[NT][4], int warp, int lane) {
   const int g = lane >> 2, tig = lane & 3;
-  // loads first and unconditionally (rows past ntok read stale stage bytes and
-  // are zeroed by a select), then the MMAs
+  // loads first and unconditionally, then the MMAs.  Token columns past ntok
+  // read token 0's row again: their sums are finite duplicates that no
+  // epilogue, partial or store ever reads.
   uint4 a[2][2];
 #pragma unroll
   for (int b = 0; b < 2; ++b)
@@ -349,18 +379,30 @@ __device__ __forceinline__ void mma_dense_x(const Params& p, const Hdr& h, const
       if (b < h.nb) {
         const uint32_t A0[4] = {a[b][0].x, a[b][0].y, a[b][0].z, a[b][0].w};
         const uint32_t A1[4] = {a[b][1].x, a[b][1].y, a[b][1].z, a[b][1].w};
-        const uint4 v = tv ? bv[b] : make_uint4(0, 0, 0, 0);
-        mma_bf16(acc[t], A0, v.x, v.y);
-        mma_bf16(acc2[t], A1, v.z, v.w);
+        mma_bf16(acc[t], A0, bv[b].x, bv[b].y);
+        mma_bf16(acc2[t], A1, bv[b].z, bv[b].w);
       }
     }
   }
 }
 
 // MXFP4 weights x f16-MX activation records: EGU, EDN.  Every shared-memory
-// load of the stage is issued first and unconditionally (the stage buffer is
-// always full size; rows and blocks outside the valid range are masked by
-// selects), so the loads overlap and the MMAs of the 8 K-blocks interleave.
+// load of the stage is issued first and unconditionally; token columns past
+// ntok read token 0's record (finite duplicates that nothing downstream
+// reads), so the inner loop carries no per-element selects.  The loop is bound
+// by the integer pipe (two warp instructions per clock per SM): per 32-wide
+// block a lane spends 8 e2m1 conversions and 2 scale extractions there, the
+// scale shifts go to the multiply-add pipe as integer multiplies.
+//
+// e8m0 scale byte s -> fp32 2^(s-127) by placing s in the exponent field.
+// s = 0 (2^-127, below fp32's normal range) becomes 0.0: every weight of such
+// a block has magnitude at most 6 * 2^-127.  0xFF (NaN) is rejected at load.
+// (j is a constant after unrolling, so the branch folds away)
+__device__ __forceinline__ float e8m0_byte_to_float(uint32_t word, int j) {
+  const uint32_t t = (j == 3) ? __umulhi(word, 0x80000000u) : word * (1u << (23 - 8 * j));
+  return __uint_as_float(t & 0x7F800000u);
+}
+
 template <int NT>
 __device__ __forceinline__ void mma_mx(const Params& p, const Hdr& h, const uint8_t* tile,
                                        const uint8_t* act, float (&acc)[NT][4], int warp, int lane) {
@@ -370,15 +412,14 @@ __device__ __forceinline__ void mma_mx(const Params& p, const Hdr& h, const uint
   uint4 cw[4];
 #pragma unroll
   for (int bp = 0; bp < 4; ++bp) cw[bp] = lds128(tile + (warp * 4 + bp) * 512 + lane * 16);
+  const bool full = h.nb == 8;
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
     const int tok = 8 * t + g;
-    const bool tv = tok < h.ntok;
     const int c0 = 8 * t + 2 * tig;
-    const bool v0 = c0 < h.ntok, v1 = c0 + 1 < h.ntok;
-    const uint8_t* arow = act + (tv ? tok : 0) * p.act_stride + tig * 16;
-    const float* s0 = reinterpret_cast<const float*>(act + (v0 ? c0 : 0) * p.act_stride + 512);
-    const float* s1 = reinterpret_cast<const float*>(act + (v1 ? c0 + 1 : 0) * p.act_stride + 512);
+    const uint8_t* arow = act + (tok < h.ntok ? tok : 0) * p.act_stride + tig * 16;
+    const float* s0 = reinterpret_cast<const float*>(act + (c0 < h.ntok ? c0 : 0) * p.act_stride + 512);
+    const float* s1 = reinterpret_cast<const float*>(act + (c0 + 1 < h.ntok ? c0 + 1 : 0) * p.act_stride + 512);
     uint4 bv[8];
 #pragma unroll
     for (int b = 0; b < 8; ++b) bv[b] = lds128(arow + b * 64);
@@ -388,26 +429,22 @@ __device__ __forceinline__ void mma_mx(const Params& p, const Hdr& h, const uint
     const float4 s1b = *reinterpret_cast<const float4*>(s1 + 4);
     const float sa0[8] = {s0a.x, s0a.y, s0a.z, s0a.w, s0b.x, s0b.y, s0b.z, s0b.w};
     const float sa1[8] = {s1a.x, s1a.y, s1a.z, s1a.w, s1b.x, s1b.y, s1b.z, s1b.w};
-    const int nb = h.nb == 8 ? 8 : h.nb;  // full chunks: the guard below folds away
 #pragma unroll
     for (int b = 0; b < 8; ++b) {
-      if (h.nb == 8 || b < nb) {
+      if (full || b < h.nb) {
         uint32_t A0[4], A1[4];
         const uint4 w4 = cw[b >> 1];
         e2m1x8_to_f16x2x4((b & 1) ? w4.z : w4.x, A0);
         e2m1x8_to_f16x2x4((b & 1) ? w4.w : w4.y, A1);
-        const float sw0 = e8m0_to_float((scw[b >> 2] >> (8 * (b & 3))) & 0xFF);
-        const float sw1 = e8m0_to_float((scw[2 + (b >> 2)] >> (8 * (b & 3))) & 0xFF);
-        const uint32_t b0 = tv ? bv[b].x : 0u, b1 = tv ? bv[b].y : 0u;
-        const uint32_t b2 = tv ? bv[b].z : 0u, b3 = tv ? bv[b].w : 0u;
-        const float a0 = v0 ? sa0[b] : 0.f, a1 = v1 ? sa1[b] : 0.f;
-        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_f16(tmp, A0, b0, b1);
-        mma_f16(tmp, A1, b2, b3);
-        acc[t][0] = fmaf(sw0 * a0, tmp[0], acc[t][0]);
-        acc[t][1] = fmaf(sw0 * a1, tmp[1], acc[t][1]);
-        acc[t][2] = fmaf(sw1 * a0, tmp[2], acc[t][2]);
-        acc[t][3] = fmaf(sw1 * a1, tmp[3], acc[t][3]);
+        const float sw0 = e8m0_byte_to_float(scw[b >> 2], b & 3);
+        const float sw1 = e8m0_byte_to_float(scw[2 + (b >> 2)], b & 3);
+        float tmp[4];
+        mma_f16_zc(tmp, A0, bv[b].x, bv[b].y);
+        mma_f16(tmp, A1, bv[b].z, bv[b].w);
+        acc[t][0] = fmaf(sw0 * sa0[b], tmp[0], acc[t][0]);
+        acc[t][1] = fmaf(sw0 * sa1[b], tmp[1], acc[t][1]);
+        acc[t][2] = fmaf(sw1 * sa0[b], tmp[2], acc[t][2]);
+        acc[t][3] = fmaf(sw1 * sa1[b], tmp[3], acc[t][3]);
       }
     }
   }
@@ -499,8 +536,7 @@ __device__ __forceinline__ void mma_tail_resident(const Params& p, const Hdr& h,
         const bool tv = tok < h.ntok;
         const uint8_t* rec = res + (size_t)(h.tok0 + (tv ? tok : 0)) * p.res_stride +
                              (kbase + 32 * b + 8 * tig) * 2;
-        uint4 bh = lds128(rec), bl = lds128(rec + p.res_k * 2);
-        if (!tv) bh = bl = make_uint4(0, 0, 0, 0);
+        const uint4 bh = lds128(rec), bl = lds128(rec + p.res_k * 2);
         mma_bf16(acc[t], A0, bh.x, bh.y);
         mma_bf16(acc2[t], A1, bh.z, bh.w);
         mma_bf16(acc[t], A0, bl.x, bl.y);
@@ -554,12 +590,9 @@ __device__ __forceinline__ void mma_tail(const Params& p, const Hdr& h, const ui
       const uint32_t A1[4] = {a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        const int tok = 8 * t + g;
-        uint4 bh = make_uint4(0, 0, 0, 0), bl = make_uint4(0, 0, 0, 0);
-        if (tok < h.ntok) {
-          bh = lds128(tbuf + tok * kTStride + (32 * b + 8 * tig) * 2);
-          bl = lds128(tbuf + tok * kTStride + 128 + (32 * b + 8 * tig) * 2);
-        }
+        const int tok = 8 * t + g < h.ntok ? 8 * t + g : 0;
+        const uint4 bh = lds128(tbuf + tok * kTStride + (32 * b + 8 * tig) * 2);
+        const uint4 bl = lds128(tbuf + tok * kTStride + 128 + (32 * b + 8 * tig) * 2);
         mma_bf16(acc[t], A0, bh.x, bh.y);
         mma_bf16(acc2[t], A1, bh.z, bh.w);
         mma_bf16(acc[t], A0, bl.x, bl.y);
@@ -651,49 +684,42 @@ template <int KIND, int NT>
 __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
                          int* sm_flag, const int* slot_tab, int tid, int warp, int lane) {
   const int g = lane >> 2, tig = lane & 3;
-  if (KIND == KIND_RL) {
-    if (h.rb < p.RB_router) {
+  if (KIND == KIND_FRONT && h.rb < p.RB_router) {
+    // router rows: publish the logits; the routing CTA waits for all of them
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
+    for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int row = 16 * warp + ((q & 2) ? g + 8 : g);
-          const int col = 8 * t + 2 * tig + (q & 1);
-          const int e = h.rb * kRowsPerBlock + row;
-          if (e < p.E && col < p.B) p.logits[(long long)col * p.E + e] = acc[t][q];
-        }
-      // every thread's logits precede thread 0's release (barrier cumulativity)
-      named_sync(1, kConsumerThreads);
-      if (p.trace && tid == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 19] = global_ns();
-      if (tid == 0) *sm_flag = (atom_add_acqrel(p.router_done, 1) == p.RB_router - 1);
-      named_sync(1, kConsumerThreads);
-      if (*sm_flag) {
-        if (p.trace && tid == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 4] = global_ns();
-        route_tokens(p, scratch, sm_flag + 16, tid, warp, lane);  // 16 ints of warp totals
-        if (p.trace && tid == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 5] = global_ns();
-        if (tid == 0) *p.router_done = 0;
+      for (int q = 0; q < 4; ++q) {
+        const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+        const int col = 8 * t + 2 * tig + (q & 1);
+        const int e = h.rb * kRowsPerBlock + row;
+        if (e < p.E && col < p.B) p.logits[(long long)col * p.E + e] = acc[t][q];
       }
-      named_sync(1, kConsumerThreads);
-    } else {
-      const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
-      const int l0 = (h.rb - p.RB_router) * kRowsPerBlock + 16 * warp + g;
-      const int idx[2] = {l0, l0 + 8};
-      float val[NT][2][2];
-      uint8_t* rec[NT][2];
+    // every thread's logits precede thread 0's release (barrier cumulativity)
+    named_sync(1, kConsumerThreads);
+    if (p.trace && tid == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 19] = global_ns();
+    if (tid == 0) atom_add_acqrel(p.router_done, 1);
+  } else if (KIND == KIND_FRONT && h.rb < p.RB_router + p.RB_lat) {
+    // latent rows -> z records
+    const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
+    const int l0 = (h.rb - p.RB_router) * kRowsPerBlock + 16 * warp + g;
+    const int idx[2] = {l0, l0 + 8};
+    float val[NT][2][2];
+    uint8_t* rec[NT][2];
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
+    for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          val[t][c][0] = acc[t][c];
-          val[t][c][1] = acc[t][2 + c];
-          const int col = 8 * t + 2 * tig + c;
-          rec[t][c] = p.z_mx + ((long long)(col < p.B ? col : 0) * cz + (l0 >> 8)) * kActRecBytes;
-        }
-      store_f16mx<NT, 2>(val, warp, lane, 2, p.B, reinterpret_cast<float*>(scratch), rec, idx,
-                         l0 < p.L, l0 + 8 < p.L);
-    }
-  } else if (KIND == KIND_SGU) {
-    const int i = 64 * h.rb + 8 * warp + g;
+      for (int c = 0; c < 2; ++c) {
+        val[t][c][0] = acc[t][c];
+        val[t][c][1] = acc[t][2 + c];
+        const int col = 8 * t + 2 * tig + c;
+        rec[t][c] = p.z_mx + ((long long)(col < p.B ? col : 0) * cz + (l0 >> 8)) * kActRecBytes;
+      }
+    store_f16mx<NT, 2>(val, warp, lane, 2, p.B, reinterpret_cast<float*>(scratch), rec, idx,
+                       l0 < p.L, l0 + 8 < p.L);
+  } else if (KIND == KIND_FRONT) {
+    // shared expert gate/up rows (64 gate + 64 up per block) -> h_s
+    const int i = 64 * (h.rb - p.RB_router - p.RB_lat) + 8 * warp + g;
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
@@ -872,6 +898,40 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
 }
 
 // ---------------------------------------------------------------------------
+// the front kernel's routing CTA
+
+// The front grid's last CTA takes no pieces.  Its consumer warps wait until
+// every router row block has been summed, select the experts, build the
+// per-expert token lists and publish them; the other CTAs keep streaming the
+// latent and shared-expert rows meanwhile.
+__device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, int* sm_flag, int tid,
+                                          int warp, int lane) {
+  unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
+  if (tid == 0) {
+    bool ok = false;
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+      if (ld_acquire(p.router_done) >= p.RB_router) {
+        ok = true;
+        break;
+      }
+      __nanosleep(64);
+    }
+    if (!ok) atomicOr(p.err, 1 << ERR_WAIT_ROUTE);
+    sm_flag[0] = ok ? 1 : 0;
+  }
+  named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
+  if (!sm_flag[0]) return;
+  if (tr && tid == 0) tr[4] = global_ns();
+  route_tokens(p, scratch, sm_flag + 16, tid, warp, lane);  // ends with a barrier
+  if (tid == 0) {
+    if (tr) tr[5] = global_ns();
+    *p.router_done = 0;
+    // every thread's table writes precede this release (barrier cumulativity)
+    st_release(p.route_ready, 1);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // consumer warps
 
 // Split-K partial sums: [piece][token column][128 rows] floats, only the
@@ -994,6 +1054,9 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   // scheduled (it cannot overtake this one's own predecessor)
   pdl_wait();
   pdl_trigger();
+  // Past this wait every earlier kernel of the forward has finished, so no
+  // reader of the routing flag is left: clear it for the next forward.
+  if (KIND == KIND_TAIL && blockIdx.x == 0 && tid == 0) *p.route_ready = 0;
   uint8_t* res = stage_base - p.stage_off + p.res_off;  // shared-memory base + offset
   if (KIND == KIND_TAIL && p.res_off) {
     build_resident(p, res, tid);
@@ -1016,7 +1079,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
     }
     const uint8_t* tile = sb + kHdrBytes;
     const uint8_t* act = sb + p.act_off;
-    if (KIND == KIND_RL || KIND == KIND_SGU) {
+    if (KIND == KIND_FRONT) {
       mma_dense_x<NT>(p, h, tile, act, acc, acc2, warp, lane);
     } else if (KIND == KIND_EGU || KIND == KIND_EDN) {
       mma_mx<NT>(p, h, tile, act, acc, warp, lane);
@@ -1048,6 +1111,34 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       continue;
     }
     write_partial<NT>(p, h.piece, h.ntok, acc, warp, lane);
+    if ((KIND == KIND_FRONT) && h.rb < p.RB_router) {
+      // Router row blocks take their ticket at once: the routing waits on
+      // all of them, and the latent rows behind it hide the round trip.
+      if (tid == 0) {
+        if (pend) tflag[tslot] = (ticket == pend_h.ppr - 1);
+        sm_flag[6] = (atom_add_acqrel(p.counters + h.v * p.RB + h.rb, 1) == h.ppr - 1);
+      }
+      named_sync(1, kConsumerThreads);
+      const bool fin_prev = pend && tflag[tslot] != 0;
+      const bool fin_now = sm_flag[6] != 0;
+      const Hdr prev = pend_h;
+      pend = false;
+      named_sync(1, kConsumerThreads);  // flags read before they are reused
+      if (fin_prev) {
+        ++n_fin;
+        finalize<KIND, NT>(p, prev, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+      }
+      if (fin_now) {
+        ++n_fin;
+        const unsigned long long t0 = tr ? global_ns() : 0ull;
+        finalize<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
+        if (tr && tid == 0) tr[7] += global_ns() - t0;
+      }
+      const long long t_c = clock64();
+      c_end += t_c - t_a;
+      t_a = t_c;
+      continue;
+    }
     if (tid == 0 && pend) tflag[tslot] = (ticket == pend_h.ppr - 1);
     named_sync(1, kConsumerThreads);  // every warp's partials precede thread 0's release
     const bool fin = pend && tflag[tslot] != 0;
@@ -1115,7 +1206,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  if (warp == kConsumerWarps) {
+  if (KIND == KIND_FRONT && p.route_cta && blockIdx.x == gridDim.x - 1) {
+    // it writes the routing tables the previous forward's tail reads
+    pdl_wait();
+    pdl_trigger();
+    if (warp < kConsumerWarps) route_cta(p, scratch, sm_flag, threadIdx.x, warp, lane);
+  } else if (warp == kConsumerWarps) {
     producer<KIND>(p, ctl, stages, tables, full, empty, lane);
   } else {
     consumer<KIND, NT>(p, stages, full, empty, scratch, sm_flag, slot_tab, warp, lane);
@@ -1161,7 +1257,7 @@ static int set_attr(size_t bytes) {
 // expert kinds up to 4 (groups of 32), the tail up to 2 (groups of 16).
 template <int KIND>
 static int launch_kind_nt(int nt, const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
-  constexpr bool kDense = (KIND == KIND_RL || KIND == KIND_SGU);
+  constexpr bool kDense = (KIND == KIND_FRONT);
   switch (nt) {
     case 1: return launch_one<KIND, 1>(p, grid, smem, s, pdl);
     case 2: return launch_one<KIND, 2>(p, grid, smem, s, pdl);
@@ -1183,7 +1279,7 @@ template <int KIND>
 static int set_attr_kind(size_t bytes) {
   int e = set_attr<KIND, 1>(bytes) | set_attr<KIND, 2>(bytes);
   if constexpr (KIND != KIND_TAIL) e |= set_attr<KIND, 4>(bytes);
-  if constexpr (KIND == KIND_RL || KIND == KIND_SGU) e |= set_attr<KIND, 8>(bytes) | set_attr<KIND, 16>(bytes);
+  if constexpr (KIND == KIND_FRONT) e |= set_attr<KIND, 8>(bytes) | set_attr<KIND, 16>(bytes);
   return e;
 }
 

@@ -1,4 +1,4 @@
-// moe_kernels.cu -- dispatch of the five kernel kinds (device code in
+// moe_kernels.cu -- dispatch of the four kernel kinds (device code in
 // moe_engine.cuh, one translation unit per kind).
 #include <cuda_runtime.h>
 
@@ -6,20 +6,17 @@
 
 namespace moe {
 
-int launch_rl(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
-int launch_sgu(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
+int launch_front(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
 int launch_egu(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
 int launch_edn(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
 int launch_tail(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
-int set_attr_rl(size_t bytes);
-int set_attr_sgu(size_t bytes);
+int set_attr_front(size_t bytes);
 int set_attr_egu(size_t bytes);
 int set_attr_edn(size_t bytes);
 int set_attr_tail(size_t bytes);
 
 int set_smem_limits(size_t bytes) {
-  return set_attr_rl(bytes) | set_attr_sgu(bytes) | set_attr_egu(bytes) | set_attr_edn(bytes) |
-         set_attr_tail(bytes);
+  return set_attr_front(bytes) | set_attr_egu(bytes) | set_attr_edn(bytes) | set_attr_tail(bytes);
 }
 
 int max_smem_optin() {
@@ -31,8 +28,7 @@ int max_smem_optin() {
 
 int launch_kind(int kind, int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl) {
   switch (kind) {
-    case KIND_RL: return launch_rl(nt, p, grid, smem, stream, pdl);
-    case KIND_SGU: return launch_sgu(nt, p, grid, smem, stream, pdl);
+    case KIND_FRONT: return launch_front(nt, p, grid, smem, stream, pdl);
     case KIND_EGU: return launch_egu(nt, p, grid, smem, stream, pdl);
     case KIND_EDN: return launch_edn(nt, p, grid, smem, stream, pdl);
     case KIND_TAIL: return launch_tail(nt, p, grid, smem, stream, pdl);

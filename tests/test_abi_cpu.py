@@ -44,13 +44,13 @@ def test_status_strings(lib):
 def test_bad_config_rejected_on_host(lib):
     h = ctypes.c_void_p()
     assert lib.moe_plan_create(None, 0, ctypes.byref(h)) == 1
-    cfg = moe.moe_config(100, 256, 16, 2, 128, 256, 1, 0, 1, 1.0, 0)  # H not a multiple of 32
+    cfg = moe.moe_config(100, 256, 16, 2, 128, 256, 1, 0, 1, 1.0)  # H not a multiple of 32
     assert lib.moe_plan_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == 1
-    cfg = moe.moe_config(512, 256, 16, 17, 128, 256, 1, 0, 1, 1.0, 0)  # k > E
+    cfg = moe.moe_config(512, 256, 16, 17, 128, 256, 1, 0, 1, 1.0)  # k > E
     assert lib.moe_plan_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == 1
-    cfg = moe.moe_config(512, 256, 2048, 2, 128, 256, 1, 0, 1, 1.0, 0)  # E beyond the limit
+    cfg = moe.moe_config(512, 256, 2048, 2, 128, 256, 1, 0, 1, 1.0)  # E beyond the limit
     assert lib.moe_plan_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == 2
-    cfg = moe.moe_config(512, 256, 16, 2, 128, 256, 256, 0, 1, 1.0, 0)  # B beyond the limit
+    cfg = moe.moe_config(512, 256, 16, 2, 128, 256, 256, 0, 1, 1.0)  # B beyond the limit
     assert lib.moe_plan_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == 2
 
 
@@ -65,5 +65,5 @@ def test_no_device_means_no_fallback(lib):
     if torch.cuda.is_available():
         pytest.skip("a device is present")
     h = ctypes.c_void_p()
-    cfg = moe.moe_config(512, 256, 16, 2, 128, 256, 1, 0, 1, 1.0, 0)
+    cfg = moe.moe_config(512, 256, 16, 2, 128, 256, 1, 0, 1, 1.0)
     assert lib.moe_plan_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == 2

@@ -19,11 +19,10 @@ pytestmark = pytest.mark.gpu
 
 
 class GpuBlock:
-    def __init__(self, shape, w, max_tokens, shared_sms=0):
+    def __init__(self, shape, w, max_tokens):
         self.shape = shape
         self.w = w
-        self.plan = moe.MoePlan(moe.config_from_shape(shape, max_tokens=max_tokens,
-                                                      shared_sms=shared_sms))
+        self.plan = moe.MoePlan(moe.config_from_shape(shape, max_tokens=max_tokens))
         self.dev_w = moe.weights_to_device(w)
         self.plan.load(self.dev_w)
         torch.cuda.synchronize()
