@@ -44,6 +44,7 @@ struct Params {
   int RB;             // row blocks per virtual matrix
   int C;              // K chunks per row block
   int PPR;            // pieces per row block (0: computed on the device, EGU/EDN)
+  int PPR_r;          // FRONT: pieces per router row block
   int target_pieces;  // EGU/EDN: aim for at least this many pieces
   int C_lat;          // TAIL: chunks covering L; chunks >= C_lat cover I_s
   int RB_router;      // FRONT: leading row blocks holding router rows

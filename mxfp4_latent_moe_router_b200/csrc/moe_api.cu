@@ -85,7 +85,7 @@ struct moe_plan_s {
   // tuning knobs read once at plan creation (environment): pieces each CTA
   // should get on average, and whether kernels chain with programmatic
   // dependent launch
-  int pieces_per_cta = 3;
+  int pieces_per_cta = 2;
   bool use_pdl = true;
 
   unsigned long long* trace = nullptr;  // [KIND_COUNT][max grid][8] when MOE_TRACE is set
@@ -157,7 +157,7 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   return f;
 }
 
-int g_max_stages = 6;  // ring depth cap (environment MOE_MAX_STAGES)
+int g_max_stages = 5;  // ring depth cap (environment MOE_MAX_STAGES)
 
 struct SmemGeom {
   int stage_bytes, nstages, act_off, act_stride, table_bytes, stage_off, res_bytes;
@@ -205,7 +205,7 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int 
   return s;
 }
 
-int g_pieces_per_cta = 3;  // set from the plan before any geometry call
+int g_pieces_per_cta = 2;  // set from the plan before any geometry call
 int target_pieces(int grid, int nt) { return grid * std::max(1, g_pieces_per_cta / nt); }
 
 Params base_params(const moe_plan_s* p, int B) {
@@ -278,6 +278,10 @@ int ppr_for(int target, int rb, int C) {
   return std::max(1, std::min(C, v));
 }
 
+// Router row blocks get pieces a third of the others' size: they are the
+// first pieces handed out, and the routing waits for all of them.
+int router_ppr(int ppr, int C) { return std::max(1, std::min(C, 3 * ppr)); }
+
 // largest number of partial-sum floats a kind can need for B <= maxB
 size_t partial_floats(const moe_plan_s* p, int kind) {
   size_t best = 0;
@@ -288,7 +292,8 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     const KindGeom& g = p->g[kind];
     if (kind == KIND_FRONT) {
       nt = f.nt_front;
-      pieces = (size_t)g.RB * ppr_for(target_pieces(f.front_workers, nt), g.RB, g.C);
+      const int ppr = ppr_for(target_pieces(f.front_workers, nt), g.RB, g.C);
+      pieces = (size_t)p->RB_router * router_ppr(ppr, g.C) + (size_t)(g.RB - p->RB_router) * ppr;
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
@@ -399,6 +404,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
 
   TRY(alloc(p, &v, sizeof(float) * maxB * E, false));
   p->logits = (float*)v;
+  CUDA_TRY(cudaMemset(v, 0, sizeof(float) * maxB * E));  // read by the top-k rehearsal
   TRY(alloc(p, &v, (size_t)maxB * ceil_div(L, kMxChunkK) * kActRecBytes, false));
   p->z_mx = (uint8_t*)v;
   TRY(alloc(p, &v, sizeof(float) * (size_t)ceil_div(std::max(Is, 1), 64) * maxB * 64, false));
@@ -483,6 +489,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     const SmemGeom sm = smem_geom(KIND_FRONT, f.nt_front, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_FRONT, sm);
     q.PPR = ppr_for(target_pieces(f.front_workers, f.nt_front), q.RB, q.C);
+    q.PPR_r = router_ppr(q.PPR, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_FRONT, f.nt_front, q, f.front_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][1], s));

@@ -62,7 +62,8 @@ struct Hdr {
   int flags;
   int piece, v, rb;
   int chunk, nb, ntok, tok0;
-  int expert, ppr, act_bytes, pad;
+  int expert, ppr, act_bytes;
+  int p0;  // first piece of this row block (its partial sums are p0 .. p0 + ppr - 1)
 };
 
 template <int KIND>
@@ -104,8 +105,9 @@ __device__ __forceinline__ Space make_space(const Params& p) {
     s.ppr = p.PPR;
     s.total = passes * p.RB * p.PPR;
   } else {
+    // FRONT: the router row blocks come first, in pieces of their own size
     s.ppr = p.PPR;
-    s.total = p.RB * p.PPR;
+    s.total = p.RB_router * p.PPR_r + (p.RB - p.RB_router) * p.PPR;
   }
   return s;
 }
@@ -138,22 +140,33 @@ __device__ __forceinline__ int chunk_blocks(const Params& p, int c) {
 template <int KIND>
 __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, int piece, Hdr& h,
                                              const VExpert* ve_tab) {
-  const int per_v = p.RB * sp.ppr;
-  const int v = piece / per_v;
-  const int rem = piece - v * per_v;
   h.piece = piece;
-  h.v = v;
-  h.rb = rem / sp.ppr;
-  h.ppr = sp.ppr;
   h.expert = 0;
+  const int nr = KIND == KIND_FRONT ? p.RB_router * p.PPR_r : 0;
+  if (piece < nr) {  // router row blocks (smaller pieces, so the logits are summed early)
+    h.v = 0;
+    h.rb = piece / p.PPR_r;
+    h.ppr = p.PPR_r;
+    h.p0 = h.rb * p.PPR_r;
+  } else {
+    const int q = piece - nr;
+    const int rb0 = KIND == KIND_FRONT ? p.RB_router : 0;
+    const int per_v = (p.RB - rb0) * sp.ppr;
+    const int v = q / per_v;
+    const int rem = q - v * per_v;
+    h.v = v;
+    h.rb = rb0 + rem / sp.ppr;
+    h.ppr = sp.ppr;
+    h.p0 = piece - rem % sp.ppr;
+  }
   if (KIND == KIND_FRONT) {
     h.ntok = p.B;
     h.tok0 = 0;
   } else if (KIND == KIND_TAIL) {
-    h.tok0 = v * p.tg;
+    h.tok0 = h.v * p.tg;
     h.ntok = min(p.tg, p.B - h.tok0);
   } else {
-    const VExpert ve = ve_tab[v];
+    const VExpert ve = ve_tab[h.v];
     h.expert = ve.expert;
     h.tok0 = ve.start;
     h.ntok = ve.count;
@@ -266,20 +279,28 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   __syncwarp();
 
   // every CTA starts on piece blockIdx.x (no round trip before the first
-  // tile); later pieces come from the cursor, offset by the grid size.  Lane 0
-  // keeps one grab in flight and reads its result one piece later.
+  // tile); later pieces come from the cursor, offset by the number of
+  // piece-taking CTAs.  Lane 0 keeps one grab in flight and reads its result
+  // one piece later -- but only once the dependency has resolved: CTAs that
+  // land early (while the previous kernel's last CTAs still run) would
+  // otherwise take several pieces each before the late ones can start, and
+  // finish last.
   long long pw = 0, pi = 0, nst = 0;
   int grabbed = 0;
+  bool in_flight = false;
   const int workers = (int)gridDim.x - (KIND == KIND_FRONT ? p.route_cta : 0);
   int piece = blockIdx.x;
-  if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
+  if (waited && piece < sp.total) {
+    if (lane == 0) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
+    in_flight = true;
+  }
   while (true) {
     if (piece >= sp.total) break;
     Hdr ph;
     piece_header<KIND>(p, sp, piece, ph, ve_tab);
-    const int pr = piece - (ph.v * p.RB + ph.rb) * sp.ppr;
-    const int c_first = (pr * p.C) / sp.ppr;
-    const int c_last = ((pr + 1) * p.C) / sp.ppr;
+    const int pr = piece - ph.p0;
+    const int c_first = (pr * p.C) / ph.ppr;
+    const int c_last = ((pr + 1) * p.C) / ph.ppr;
     for (int c = c_first; c < c_last; ++c) {
       // before the dependency resolves, fill at most one ring of weight-only stages
       if (!waited && prefetched == p.nstages) {
@@ -316,8 +337,21 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       pi += clock64() - tw1;
       ++nst;
     }
+    if (!waited) {
+      // first piece issued and still no dependency: stop prefetching here
+      pdl_wait();
+      pdl_trigger();
+      waited = true;
+      for (int s = 0; s < prefetched; ++s) {
+        uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
+        const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
+        issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
+      }
+    }
+    if (!in_flight && lane == 0) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
     piece = __shfl_sync(0xffffffffu, grabbed, 0);
-    if (lane == 0 && piece < sp.total) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
+    in_flight = piece < sp.total;
+    if (lane == 0 && in_flight) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
   }
   if (!waited) {
     pdl_wait();
@@ -678,7 +712,7 @@ __device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int wa
 }
 
 __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, int* wtot, int tid,
-                                          int warp, int lane);
+                                          int warp, int lane, bool dry);
 
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
@@ -775,8 +809,11 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
 // top-k routing and per-expert token lists (one CTA, 256 threads); the
 // per-token selection is warp_topk (topk.cuh).
 
+// dry: the same instructions with every global store skipped (a rehearsal
+// that brings the code into the instruction cache while the logits are not
+// ready yet; its shared-memory results are discarded)
 __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, int* wtot, int tid,
-                                          int warp, int lane) {
+                                          int warp, int lane, bool dry) {
   const int E = p.E, K = p.topk, B = p.B;
   const int tg = p.tg > 0 ? p.tg : 1;
   int* cnt = reinterpret_cast<int*>(scratch);  // [E] slots per expert
@@ -800,8 +837,10 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
       warp_topk(p.logits + (long long)b * E, E, K, p.score_fn, p.bias, p.renorm, p.routed_scale,
                 lane, sel_id, sel_w);
       if (lane < K) {
-        p.ids[b * K + lane] = sel_id;
-        p.wts[b * K + lane] = sel_w;
+        if (!dry) {
+          p.ids[b * K + lane] = sel_id;
+          p.wts[b * K + lane] = sel_w;
+        }
         ids_s[b * K + lane] = sel_id;
         atomicAdd(&cnt[sel_id], 1);
       }
@@ -829,8 +868,10 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
       warp_topk_merge(cand + b * P * K, part + b * P, P, K, E, p.score_fn, p.renorm,
                       p.routed_scale, lane, sel_id, sel_w);
       if (lane < K) {
-        p.ids[b * K + lane] = sel_id;
-        p.wts[b * K + lane] = sel_w;
+        if (!dry) {
+          p.ids[b * K + lane] = sel_id;
+          p.wts[b * K + lane] = sel_w;
+        }
         ids_s[b * K + lane] = sel_id;
         atomicAdd(&cnt[sel_id], 1);
       }
@@ -880,19 +921,19 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
         ve.start = bc + gi * tg;
         ve.count = min(tg, c[i] - gi * tg);
         ve.pad = 0;
-        if (bg + gi < p.ve_max) p.ve[bg + gi] = ve;
+        if (!dry && bg + gi < p.ve_max) p.ve[bg + gi] = ve;
       }
     }
     bc += c[i];
     bg += gsz[i];
   }
-  if (tid == kConsumerThreads - 1) *p.nve = bg < p.ve_max ? bg : p.ve_max;
+  if (!dry && tid == kConsumerThreads - 1) *p.nve = bg < p.ve_max ? bg : p.ve_max;
   named_sync(1, kConsumerThreads);
   if (tr) tr[18] = global_ns();
   for (int s = tid; s < B * K; s += kConsumerThreads) {
     const int e = ids_s[s];
     const int pos = off[e] + atomicAdd(&fill[e], 1);
-    p.slots_sorted[pos] = s;
+    if (!dry) p.slots_sorted[pos] = s;
   }
   named_sync(1, kConsumerThreads);
 }
@@ -907,6 +948,11 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
 __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, int* sm_flag, int tid,
                                           int warp, int lane) {
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
+  // Selection is a short serial program run once per forward: cold, every
+  // instruction fetch would miss and queue behind the HBM stream.  Rehearse
+  // it on whatever the logits buffer holds while the router rows stream.
+  route_tokens(p, scratch, sm_flag + 16, tid, warp, lane, true);
+  if (tr && tid == 0) tr[20] = global_ns();
   if (tid == 0) {
     bool ok = false;
     for (uint32_t i = 0; i < (1u << 22); ++i) {
@@ -922,7 +968,7 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, int
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
   if (!sm_flag[0]) return;
   if (tr && tid == 0) tr[4] = global_ns();
-  route_tokens(p, scratch, sm_flag + 16, tid, warp, lane);  // ends with a barrier
+  route_tokens(p, scratch, sm_flag + 16, tid, warp, lane, false);  // ends with a barrier
   if (tid == 0) {
     if (tr) tr[5] = global_ns();
     *p.router_done = 0;
@@ -957,7 +1003,7 @@ template <int NT>
 __device__ __forceinline__ void sum_partials(const Params& p, const Hdr& h, float (&acc)[NT][4],
                                              int warp, int lane) {
   const int g = lane >> 2, tig = lane & 3;
-  const long long first = (long long)(h.v * p.RB + h.rb) * h.ppr;
+  const long long first = h.p0;
   const long long stride = NT * 8 * kRowsPerBlock;
 #pragma unroll
   for (int t = 0; t < NT; ++t)
@@ -988,7 +1034,7 @@ __device__ __forceinline__ void sum_partials(const Params& p, const Hdr& h, floa
 template <int NT>
 __device__ __forceinline__ void sum_partials_wide(const Params& p, const Hdr& h, float (&acc)[NT][4],
                                                   float* rs, int tid, int warp, int lane) {
-  const long long first = (long long)(h.v * p.RB + h.rb) * h.ppr;
+  const long long first = h.p0;
   const long long stride = NT * 8 * kRowsPerBlock;
   const int n = h.ntok * kRowsPerBlock;
   for (int i = tid; i < n; i += kConsumerThreads) {
