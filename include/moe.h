@@ -121,7 +121,7 @@ typedef struct moe_plan_info {
   int64_t workspace_bytes;  /* library-owned activations, routing metadata, partial sums */
   int64_t dense_weight_bytes;      /* bf16 bytes one forward streams regardless of routing */
   int64_t expert_weight_bytes;     /* MXFP4 bytes of one expert (gate/up + down, codes + scales) */
-  int32_t kernels_per_forward;     /* launches one moe_forward makes */
+  int32_t kernels_per_forward;     /* launches one moe_forward of max_tokens tokens makes */
 } moe_plan_info;
 
 /*
@@ -186,16 +186,18 @@ MOE_API moe_status moe_get_plan_info(moe_plan p, moe_plan_info *info);
  * each of its kernels with CUDA events on the stream that kernel runs on and
  * waits for them before returning (so profiled forwards are synchronous and
  * must not be captured into a graph).  moe_get_profile writes the accumulated
- * milliseconds per kernel in launch order {dense front (router, latent, shared
- * gate/up, top-k), expert gate/up, expert down, latent tail} to ms[0..3] and
- * the number of profiled forwards to *count, then clears both.
+ * milliseconds per kernel to ms[0..4] -- {dense front (router, latent, shared
+ * gate/up, top-k), expert gate/up, expert down, latent tail, fused single
+ * launch}; a forward of at most 8 tokens runs only the last, larger ones the
+ * first four -- and the number of profiled forwards to *count, then clears
+ * both.
  */
 MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
 
 /*
  * Per-CTA timeline of the most recent forward, for measurement only; exists
  * when the plan was created with the environment variable MOE_TRACE set
- * (else MOE_ERR_UNSUPPORTED).  host receives count = 4 * num_sms * 24 uint64:
+ * (else MOE_ERR_UNSUPPORTED).  host receives count = 5 * num_sms * 24 uint64:
  * for kernel kind k (launch order as in moe_get_profile) and CTA c, the 24
  * values at (k * num_sms + c) * 24 are {start ns, end ns, pieces, finalizes,
  * top-k start ns, top-k end ns, first stage ready ns, finalize ns, consumer

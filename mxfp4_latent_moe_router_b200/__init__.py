@@ -27,9 +27,10 @@ ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forwar
                "moe_last_routing", "moe_debug_fetch", "moe_sync_status", "moe_get_plan_info",
                "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile",
                "moe_route_noalloc", "moe_debug_trace"]
-# kernel kinds in launch order: the dense front kernel streams the router,
-# latent-projection and shared-expert gate/up rows (and runs top-k)
-KERNEL_NAMES = ["dense_front", "expert_gate_up", "expert_down", "latent_tail"]
+# launch slots: the four kernels a forward of more than 8 tokens runs (the
+# dense front kernel streams the router, latent-projection and shared-expert
+# gate/up rows and runs top-k), then the single fused launch of smaller ones
+KERNEL_NAMES = ["dense_front", "expert_gate_up", "expert_down", "latent_tail", "fused_block"]
 
 
 class MoeError(RuntimeError):
@@ -187,7 +188,7 @@ def moe_route_noalloc(x, router_w, router_bias, num_tokens: int, hidden: int, nu
 
 
 def moe_debug_trace(plan: int, num_sms: int):
-    """Per-CTA timeline of the last forward: uint64 array [4 kinds][num_sms][24]."""
+    """Per-CTA timeline of the last forward: uint64 array [5 launch slots][num_sms][24]."""
     import numpy as np
     a = np.zeros((len(KERNEL_NAMES), num_sms, 24), np.uint64)
     _check(load_library().moe_debug_trace(plan, a.ctypes.data, a.size), "moe_debug_trace")

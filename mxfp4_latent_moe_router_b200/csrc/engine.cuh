@@ -45,7 +45,8 @@ struct Params {
   int C;              // K chunks per row block
   int PPR;            // pieces per row block (0: computed on the device, EGU/EDN)
   int PPR_r;          // FRONT: pieces per router row block
-  int target_pieces;  // EGU/EDN: aim for at least this many pieces
+  int piece_ctas;     // EGU/EDN: CTAs taking pieces (for the split-K choice)
+  int split_cost;     // EGU/EDN: price of a split-K piece end, in stages
   int C_lat;          // TAIL: chunks covering L; chunks >= C_lat cover I_s
   int RB_router;      // FRONT: leading row blocks holding router rows
   int RB_lat;         // FRONT: row blocks of the latent projection (after the router's);
@@ -93,12 +94,30 @@ struct Params {
   // it is set, before their own dependency resolves.  Cleared by the tail,
   // which no reader of it can still be running beside.
   int* route_ready;
+  // fused single-launch path only (null otherwise): completion counts that
+  // later phases wait on, each raised with release semantics once a row
+  // block's outputs are stored: [0] latent row blocks (z), [1] shared-expert
+  // row blocks (h_s), [2] expert gate/up matrices (h), [3] expert down
+  // matrices (y)
+  int* done;
+  // fused launch, tail phase: the counts it waits for (expert-down row
+  // blocks per virtual expert; shared-expert row blocks)
+  int need_rb_edn, need_rb_sh;
   float* partials;
   int* err;
 };
 
-// Host-side launcher (defined in moe_kernels.cu).
+// The single-launch path (few tokens): one Params per phase, all with the
+// same shared-memory layout and ring, and the size of the front phase (the
+// first part of the ordered piece list).
+struct MegaParams {
+  Params k[KIND_COUNT];
+  int n_front;
+};
+
+// Host-side launchers (defined in moe_kernels.cu and moe_k_mega.cu).
 int launch_kind(int kind, int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
+int launch_mega(const MegaParams& mp, int grid, size_t smem, void* stream, bool pdl);
 int max_smem_optin();
 int set_smem_limits(size_t bytes);
 

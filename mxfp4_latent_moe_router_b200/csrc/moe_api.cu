@@ -25,6 +25,12 @@ constexpr int kScratchOff = 1024;
 constexpr int kScratchBytes = 20480;
 constexpr int kStageOff = kScratchOff + kScratchBytes;
 constexpr int kHdr = 128;
+// per-kind slots (scheduling state, profile, trace) plus one for the fused
+// single launch, which uses slot KIND_COUNT
+constexpr int kSlots = KIND_COUNT + 1;
+constexpr int kFused = KIND_COUNT;
+// largest batch the fused single launch takes (one 8-column token tile)
+constexpr int kFusedMaxTokens = 8;
 constexpr int kTailTg = 16;
 constexpr int kExpertTg = 32;
 constexpr int kBigSmem = 227 * 1024;
@@ -71,7 +77,8 @@ struct moe_plan_s {
   int* slots_sorted = nullptr;
   VExpert* ve = nullptr;
   int* nve = nullptr;
-  Ctl* ctl = nullptr;  // [KIND_COUNT]
+  Ctl* ctl = nullptr;  // [kSlots]
+  int* done = nullptr;  // [4] phase completion counts of the fused launch
   int* counters[KIND_COUNT] = {};
   int* router_done = nullptr;
   int* route_ready = nullptr;
@@ -82,17 +89,20 @@ struct moe_plan_s {
   uint16_t* out_stage = nullptr;
 
 
-  // tuning knobs read once at plan creation (environment): pieces each CTA
-  // should get on average, and whether kernels chain with programmatic
-  // dependent launch
-  int pieces_per_cta = 2;
+  // tuning knobs read once at plan creation (environment): the price of a
+  // split-K piece end in the split choice, whether kernels chain with
+  // programmatic dependent launch, and whether small batches run fused
+  int split_cost = 2;
   bool use_pdl = true;
+  // one launch per forward for B <= kFusedMaxTokens (environment MOE_FUSED=1);
+  // off by default: measured slower than the four-launch chain at B = 1
+  bool use_fused = false;
 
   unsigned long long* trace = nullptr;  // [KIND_COUNT][max grid][8] when MOE_TRACE is set
 
   bool profiling = false;
-  cudaEvent_t ev_prof[KIND_COUNT][2] = {};
-  double prof_ms[KIND_COUNT] = {};
+  cudaEvent_t ev_prof[kSlots][2] = {};
+  double prof_ms[kSlots] = {};
   int prof_count = 0;
 };
 
@@ -205,8 +215,7 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int 
   return s;
 }
 
-int g_pieces_per_cta = 2;  // set from the plan before any geometry call
-int target_pieces(int grid, int nt) { return grid * std::max(1, g_pieces_per_cta / nt); }
+int g_split_cost = 2;  // split-K piece-end price in stages (environment MOE_SPLIT_COST)
 
 Params base_params(const moe_plan_s* p, int B) {
   Params q;
@@ -273,10 +282,8 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   }
 }
 
-int ppr_for(int target, int rb, int C) {
-  int v = (target + rb - 1) / rb;
-  return std::max(1, std::min(C, v));
-}
+// split-K factor of a kind whose row-block count the host knows
+int ppr_for(int mats, int C, int ctas) { return best_ppr(mats, C, ctas, g_split_cost); }
 
 // Router row blocks get pieces a third of the others' size: they are the
 // first pieces handed out, and the routing waits for all of them.
@@ -292,17 +299,18 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     const KindGeom& g = p->g[kind];
     if (kind == KIND_FRONT) {
       nt = f.nt_front;
-      const int ppr = ppr_for(target_pieces(f.front_workers, nt), g.RB, g.C);
+      const int ppr = ppr_for(g.RB, g.C, f.front_workers);
       pieces = (size_t)p->RB_router * router_ppr(ppr, g.C) + (size_t)(g.RB - p->RB_router) * ppr;
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      pieces = (size_t)passes * g.RB * ppr_for(target_pieces(f.tail_grid, nt), g.RB * passes, g.C);
+      pieces = (size_t)passes * g.RB * ppr_for(g.RB * passes, g.C, f.tail_grid);
     } else {
       nt = f.nt_e;
-      // PPR > 1 only while (virtual experts x row blocks) < target, so the
-      // pieces that need partial storage stay below 2 x target
-      pieces = 2 * (size_t)target_pieces(f.expert_grid, nt) + g.RB;
+      // the split depends on the routing: take the largest over every
+      // possible count of virtual experts
+      for (int V = 1; V <= p->ve_max; ++V)
+        pieces = std::max(pieces, (size_t)V * g.RB * ppr_for(V * g.RB, g.C, f.expert_grid));
     }
     best = std::max(best, pieces * (size_t)nt * 1024);
   }
@@ -348,10 +356,11 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   CUDA_TRY(cudaGetDeviceProperties(&prop, device));
   if (prop.major != 10) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
   p->num_sms = prop.multiProcessorCount;
-  if (const char* e = getenv("MOE_PIECES_PER_CTA")) p->pieces_per_cta = std::max(1, atoi(e));
+  if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
+  if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
   if (const char* e = getenv("MOE_MAX_STAGES")) g_max_stages = std::max(2, std::min(8, atoi(e)));
-  g_pieces_per_cta = p->pieces_per_cta;
+  g_split_cost = p->split_cost;
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -422,13 +431,14 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   TRY(alloc(p, &v, sizeof(VExpert) * p->ve_max, false));
   p->ve = (VExpert*)v;
   // small control block: nve, router_done, err, Ctl[KIND_COUNT]
-  TRY(alloc(p, &v, 1024 + sizeof(Ctl) * KIND_COUNT, false));
+  TRY(alloc(p, &v, 1024 + sizeof(Ctl) * kSlots, false));
   p->nve = (int*)v;
   p->router_done = p->nve + 1;
   p->err = p->nve + 2;
+  p->done = p->nve + 8;
   p->route_ready = p->nve + 3;
   p->ctl = reinterpret_cast<Ctl*>((uint8_t*)v + 1024);
-  CUDA_TRY(cudaMemset(v, 0, 1024 + sizeof(Ctl) * KIND_COUNT));
+  CUDA_TRY(cudaMemset(v, 0, 1024 + sizeof(Ctl) * kSlots));
   const int cnt_n[KIND_COUNT] = {fr.RB, p->ve_max * eg.RB, p->ve_max * ed.RB, maxB * tl.RB};
   for (int k = 0; k < KIND_COUNT; ++k) {
     TRY(alloc(p, &v, sizeof(int) * cnt_n[k], false));
@@ -439,16 +449,16 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
     p->partials[k] = (float*)v;
   }
   if (getenv("MOE_TRACE")) {
-    TRY(alloc(p, &v, sizeof(unsigned long long) * KIND_COUNT * p->num_sms * 24, false));
+    TRY(alloc(p, &v, sizeof(unsigned long long) * kSlots * p->num_sms * 24, false));
     p->trace = (unsigned long long*)v;
-    CUDA_TRY(cudaMemset(v, 0, sizeof(unsigned long long) * KIND_COUNT * p->num_sms * 24));
+    CUDA_TRY(cudaMemset(v, 0, sizeof(unsigned long long) * kSlots * p->num_sms * 24));
   }
   TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
   p->x_stage = (uint16_t*)v;
   TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
   p->out_stage = (uint16_t*)v;
 
-  for (int k = 0; k < KIND_COUNT; ++k)
+  for (int k = 0; k < kSlots; ++k)
     for (int j = 0; j < 2; ++j) CUDA_TRY(cudaEventCreate(&p->ev_prof[k][j]));
   CUDA_TRY(cudaDeviceSynchronize());
   if (getenv("MOE_LOG")) {
@@ -466,21 +476,86 @@ void destroy_impl(moe_plan p) {
   DeviceGuard g(p->device);
   cudaDeviceSynchronize();
   for (void* a : p->allocs) cudaFree(a);
-  for (int k = 0; k < KIND_COUNT; ++k)
+  for (int k = 0; k < kSlots; ++k)
     for (int j = 0; j < 2; ++j)
       if (p->ev_prof[k][j]) cudaEventDestroy(p->ev_prof[k][j]);
   cudaGetLastError();
   delete p;
 }
 
+// The whole block as one launch (B <= kFusedMaxTokens): every phase's
+// Params share one shared-memory layout -- routing tables, the tail's resident
+// activation, and a ring of the largest stage any phase needs.
+moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B, cudaStream_t s) {
+  const moe_config& c = p->cfg;
+  const int tail_tg_eff = std::min(B, p->tail_tg);
+  const int res_k = p->g[KIND_TAIL].C * kDenseChunkK;
+  const int res_bytes = (B * resident_stride(res_k) <= kResidentMax) ? B * resident_stride(res_k) : 0;
+  SmemGeom g[KIND_COUNT];
+  int stage_bytes = 0;
+  for (int k = 0; k < KIND_COUNT; ++k) {
+    g[k] = smem_geom(k, 1, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, k == KIND_TAIL ? res_bytes : 0);
+    stage_bytes = std::max(stage_bytes, g[k].stage_bytes);
+  }
+  const int table_bytes = g[KIND_EGU].table_bytes;
+  const int stage_off = kStageOff + table_bytes + res_bytes;
+  const int nstages = std::max(2, std::min(g_max_stages, (kBigSmem - stage_off) / stage_bytes));
+  const size_t total = std::max((size_t)stage_off + (size_t)nstages * stage_bytes, (size_t)(116 * 1024));
+  MegaParams mp;
+  std::memset(&mp, 0, sizeof(mp));
+  for (int k = 0; k < KIND_COUNT; ++k) {
+    Params q = base;
+    set_kind(q, p, k, g[k]);
+    q.nstages = nstages;
+    q.stage_bytes = stage_bytes;
+    q.stage_off = stage_off;
+    q.table_off = kStageOff;
+    q.ctl = p->ctl + kFused;
+    q.trace = p->trace ? p->trace + (size_t)kFused * p->num_sms * 24 : nullptr;
+    q.done = p->done;
+    q.need_rb_edn = p->g[KIND_EDN].RB;
+    q.need_rb_sh = p->g[KIND_FRONT].RB - p->RB_router - p->RB_lat;
+    if (k == KIND_FRONT) {
+      q.PPR = ppr_for(q.RB, q.C, f.front_workers);
+      q.PPR_r = router_ppr(q.PPR, q.C);
+      mp.n_front = p->RB_router * q.PPR_r + (q.RB - p->RB_router) * q.PPR;
+    } else if (k == KIND_EGU || k == KIND_EDN) {
+      q.piece_ctas = f.expert_grid;
+      q.split_cost = g_split_cost;
+    } else {
+      if (res_bytes) {
+        q.res_off = kStageOff + table_bytes;
+        q.res_stride = resident_stride(res_k);
+        q.res_k = res_k;
+      }
+      const int passes = (B + p->tail_tg - 1) / p->tail_tg;
+      q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid);
+    }
+    mp.k[k] = q;
+  }
+  if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[kFused][0], s));
+  CUDA_TRY((cudaError_t)launch_mega(mp, p->num_sms, total, s, p->use_pdl));
+  if (p->profiling) {
+    CUDA_TRY(cudaEventRecord(p->ev_prof[kFused][1], s));
+    CUDA_TRY(cudaEventSynchronize(p->ev_prof[kFused][1]));
+    float ms = 0.f;
+    CUDA_TRY(cudaEventElapsedTime(&ms, p->ev_prof[kFused][0], p->ev_prof[kFused][1]));
+    p->prof_ms[kFused] += ms;
+    ++p->prof_count;
+  }
+  p->last_B = B;
+  return MOE_OK;
+}
+
 moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStream_t s) {
   const moe_config& c = p->cfg;
-  g_pieces_per_cta = p->pieces_per_cta;
+  g_split_cost = p->split_cost;
   const FwdGeom f = fwd_geom(p, B);
   const int tail_tg_eff = std::min(B, p->tail_tg);
   Params base = base_params(p, B);
   base.x = (const uint16_t*)x;
   base.out = (uint16_t*)out;
+  if (p->use_fused && B <= kFusedMaxTokens) return enqueue_fused(p, base, f, B, s);
 
   // One stream, each kernel a programmatic dependent of the one before:
   //   front (router, latent, shared gate/up) -> expert gate/up -> expert down -> tail.
@@ -488,7 +563,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     Params q = base;
     const SmemGeom sm = smem_geom(KIND_FRONT, f.nt_front, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_FRONT, sm);
-    q.PPR = ppr_for(target_pieces(f.front_workers, f.nt_front), q.RB, q.C);
+    q.PPR = ppr_for(q.RB, q.C, f.front_workers);
     q.PPR_r = router_ppr(q.PPR, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_FRONT, f.nt_front, q, f.front_grid, sm.total, s, p->use_pdl));
@@ -498,7 +573,8 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     Params q = base;
     const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EGU, sm);
-    q.target_pieces = target_pieces(f.expert_grid, f.nt_e);
+    q.piece_ctas = f.expert_grid;
+    q.split_cost = g_split_cost;
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
@@ -507,7 +583,8 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     Params q = base;
     const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EDN, sm);
-    q.target_pieces = target_pieces(f.expert_grid, f.nt_e);
+    q.piece_ctas = f.expert_grid;
+    q.split_cost = g_split_cost;
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
@@ -526,7 +603,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       q.res_k = res_k;
     }
     const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-    q.PPR = ppr_for(target_pieces(f.tail_grid, f.nt_tail), q.RB * passes, q.C);
+    q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][1], s));
@@ -803,14 +880,14 @@ moe_status moe_get_plan_info(moe_plan p, moe_plan_info* info) {
       6LL * c.hidden * c.shared_inter;
   info->expert_weight_bytes =
       (3LL * c.expert_inter * c.latent) / 2 + (3LL * c.expert_inter * c.latent) / 32;
-  info->kernels_per_forward = KIND_COUNT;
+  info->kernels_per_forward = (p->use_fused && p->cfg.max_tokens <= kFusedMaxTokens) ? 1 : KIND_COUNT;
   return MOE_OK;
 }
 
 moe_status moe_debug_trace(moe_plan p, uint64_t* host, int64_t count) {
   if (!p || !host) return MOE_ERR_INVALID_ARG;
   if (!p->trace) return MOE_ERR_UNSUPPORTED;
-  const int64_t n = (int64_t)KIND_COUNT * p->num_sms * 24;
+  const int64_t n = (int64_t)kSlots * p->num_sms * 24;
   if (count != n) return MOE_ERR_INVALID_ARG;
   DeviceGuard g(p->device);
   CUDA_TRY(cudaDeviceSynchronize());
@@ -826,7 +903,7 @@ moe_status moe_set_profiling(moe_plan p, int32_t enable) {
 
 moe_status moe_get_profile(moe_plan p, float* ms, int32_t* count) {
   if (!p || !ms || !count) return MOE_ERR_INVALID_ARG;
-  for (int k = 0; k < KIND_COUNT; ++k) {
+  for (int k = 0; k < kSlots; ++k) {
     ms[k] = (float)p->prof_ms[k];
     p->prof_ms[k] = 0.0;
   }

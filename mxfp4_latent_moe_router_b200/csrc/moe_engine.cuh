@@ -64,6 +64,9 @@ struct Hdr {
   int chunk, nb, ntok, tok0;
   int expert, ppr, act_bytes;
   int p0;  // first piece of this row block (its partial sums are p0 .. p0 + ppr - 1)
+  // fused single-launch path: this piece's kind, and on its last stage the
+  // kind of the piece the producer streams next (-1: none)
+  int kind, next_kind;
 };
 
 template <int KIND>
@@ -96,8 +99,7 @@ __device__ __forceinline__ Space make_space(const Params& p) {
   if (KIND == KIND_EGU || KIND == KIND_EDN) {
     const int V = *reinterpret_cast<volatile int*>(p.nve);
     const int mats = V * p.RB;
-    int ppr = mats > 0 ? (p.target_pieces + mats - 1) / mats : 1;
-    ppr = ppr < 1 ? 1 : (ppr > p.C ? p.C : ppr);
+    const int ppr = best_ppr(mats, p.C, p.piece_ctas, p.split_cost);
     s.ppr = ppr;
     s.total = mats * ppr;
   } else if (KIND == KIND_TAIL) {
@@ -750,7 +752,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
         rec[t][c] = p.z_mx + ((long long)(col < p.B ? col : 0) * cz + (l0 >> 8)) * kActRecBytes;
       }
     store_f16mx<NT, 2>(val, warp, lane, 2, p.B, reinterpret_cast<float*>(scratch), rec, idx,
-                       l0 < p.L, l0 + 8 < p.L);
+                       l0 < p.L, l0 + 8 < p.L);  // ends with a barrier
+    if (p.done && tid == 0) red_release_add(p.done + 0, 1);
   } else if (KIND == KIND_FRONT) {
     // shared expert gate/up rows (64 gate + 64 up per block) -> h_s
     const int i = 64 * (h.rb - p.RB_router - p.RB_lat) + 8 * warp + g;
@@ -762,6 +765,10 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
         if (col < p.B && i < p.Is)
           p.h_s[((long long)(i >> 6) * p.B + col) * 64 + (i & 63)] = silu(acc[t][c]) * acc[t][2 + c];
       }
+    if (p.done) {
+      named_sync(1, kConsumerThreads);  // every thread's h_s precede the release
+      if (tid == 0) red_release_add(p.done + 1, 1);
+    }
   } else if (KIND == KIND_EGU) {
     const int i = 64 * h.rb + 8 * warp + g;
     const int idx[2] = {i, i};
@@ -778,7 +785,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
         rec[t][c] = p.h_mx + ((long long)(i >> 8) * p.ld_slots + pos) * kActRecBytes;
       }
     store_f16mx<NT, 1>(val, warp, lane, 4, h.ntok, reinterpret_cast<float*>(scratch), rec, idx,
-                       i < p.I, false);
+                       i < p.I, false);  // ends with a barrier
+    if (p.done && tid == 0) red_release_add(p.done + 2, 1);
   } else if (KIND == KIND_EDN) {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
@@ -791,6 +799,10 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
           p.y[((long long)(l >> 6) * p.ld_slots + slot) * 64 + (l & 63)] = acc[t][q];
         }
       }
+    if (p.done) {
+      named_sync(1, kConsumerThreads);  // every thread's y precede the release
+      if (tid == 0) red_release_add(p.done + 3, 1);
+    }
   } else {  // TAIL
 #pragma unroll
     for (int t = 0; t < NT; ++t)

@@ -6,6 +6,8 @@
 
 namespace moe {
 
+int set_attr_mega(size_t bytes);
+
 int launch_front(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
 int launch_egu(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
 int launch_edn(int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
@@ -16,7 +18,8 @@ int set_attr_edn(size_t bytes);
 int set_attr_tail(size_t bytes);
 
 int set_smem_limits(size_t bytes) {
-  return set_attr_front(bytes) | set_attr_egu(bytes) | set_attr_edn(bytes) | set_attr_tail(bytes);
+  return set_attr_front(bytes) | set_attr_egu(bytes) | set_attr_edn(bytes) | set_attr_tail(bytes) |
+         set_attr_mega(bytes);
 }
 
 int max_smem_optin() {

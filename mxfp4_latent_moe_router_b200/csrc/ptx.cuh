@@ -109,6 +109,9 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
 __device__ __forceinline__ void st_release(int* p, int v) {
   asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // ---- warp MMA: D = A(16x16, row) * B(16x8, col) + C, fp32 accumulate ----------
 // (not volatile: independent MMAs may be interleaved by the compiler)

@@ -9,39 +9,37 @@
 // takes the top-k of a slice of the experts (warp_topk_slice), and one warp
 // merges the candidates of all slices (warp_topk_merge).  With one slice the
 // merge is skipped (warp_topk).
+//
+// A selection round is two warp reductions (redux.sync): the largest key, as
+// an order-preserving unsigned integer, and the lowest expert index among the
+// lanes that hold it -- instead of a five-level shuffle tree carrying key,
+// index and logit.  The winner's logit then comes from its lane with one
+// shuffle.
 #pragma once
 #include <cstdint>
 
 namespace moe {
 
 // Scores use the hardware exp2 and fast divide (a few ulp, far below the
-// 1e-5 relative accuracy the combine weights need): the selection runs once
-// per forward as cold, straight-line code whose instruction footprint matters.
+// 1e-5 relative accuracy the combine weights need).
 __device__ __forceinline__ float fast_sigmoid(float l) { return __fdividef(1.0f, 1.0f + __expf(-l)); }
 
-__device__ __forceinline__ bool topk_better(float ka, int ia, float kb, int ib) {
-  return ka > kb || (ka == kb && ia < ib);
+// float -> unsigned with the same order (NaN lowest, never preferred)
+__device__ __forceinline__ uint32_t key_order(float f) {
+  const uint32_t b = __float_as_uint(f);
+  const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return f == f ? o : 0u;
 }
-
-// One selection round: the warp-wide best (key, index, logit) under topk_better.
-__device__ __forceinline__ void warp_best(float& bk, int& bi, float& bl) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
-    if (topk_better(ok, oi, bk, bi)) {
-      bk = ok;
-      bi = oi;
-      bl = ol;
-    }
-  }
+__device__ __forceinline__ float key_value(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
 struct TopkCand {
   float key, logit;
   int id, pad;
 };
+
+constexpr uint32_t kNoExpert = 0xffffffffu;
 
 // Top-K of experts [e0, e1) of one token (K <= 16, e1 - e0 <= 32 * EPL).
 // On return lane r < K holds the r-th best candidate (key-descending), and
@@ -51,25 +49,26 @@ template <int EPL>
 __device__ __forceinline__ void warp_topk_slice(const float* logits, const float* bias, int e0, int e1,
                                              int K, int score_fn, int lane, TopkCand& out,
                                              float& smax, float& ssum) {
-  float key[EPL], lg[EPL], bs[EPL];
+  float lg[EPL], bs[EPL];
+  uint32_t ok[EPL];
   // all loads first (one round trip), arithmetic after
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     const int e = e0 + lane + 32 * j;
-    const bool ok = e < e1;
-    lg[j] = ok ? __ldcg(logits + e) : 0.f;
-    bs[j] = (ok && bias) ? __ldg(bias + e) : 0.f;
+    const bool in = e < e1;
+    lg[j] = in ? __ldcg(logits + e) : 0.f;
+    bs[j] = (in && bias) ? __ldg(bias + e) : 0.f;
   }
   float mx = -INFINITY;
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     const int e = e0 + lane + 32 * j;
-    key[j] = -INFINITY;
+    ok[j] = 0u;  // below every real key
     if (e < e1) {
       if (score_fn == 1) {
-        key[j] = fast_sigmoid(lg[j]) + bs[j];
+        ok[j] = key_order(fast_sigmoid(lg[j]) + bs[j]);
       } else {
-        key[j] = lg[j];
+        ok[j] = key_order(lg[j]);
         mx = fmaxf(mx, lg[j]);
       }
     }
@@ -93,25 +92,33 @@ __device__ __forceinline__ void warp_topk_slice(const float* logits, const float
   out.logit = 0.f;
   out.pad = 0;
   for (int r = 0; r < K; ++r) {
-    float bk = -INFINITY, bl = 0.f;
-    int bi = 0x7fffffff;
+    // local best: largest key, then lowest index (lower j = lower index)
+    uint32_t bo = 0u, bj = 0u;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = e0 + lane + 32 * j;
-      if (e < e1 && topk_better(key[j], e, bk, bi)) {
-        bk = key[j];
-        bi = e;
-        bl = lg[j];
+    for (int j = EPL - 1; j >= 0; --j)
+      if (ok[j] >= bo) {
+        bo = ok[j];
+        bj = (uint32_t)j;
       }
-    }
-    warp_best(bk, bi, bl);
+    const uint32_t bi = bo ? (uint32_t)(e0 + lane) + 32u * bj : kNoExpert;
+    const uint32_t wo = __reduce_max_sync(0xffffffffu, bo);
+    const uint32_t wi = __reduce_min_sync(0xffffffffu, bo == wo ? bi : kNoExpert);
+    if (wi == kNoExpert) break;  // fewer than K experts in the slice
+    const int wl = (int)((wi - (uint32_t)e0) & 31u), wj = (int)((wi - (uint32_t)e0) >> 5);
+    float my = 0.f;
 #pragma unroll
     for (int j = 0; j < EPL; ++j)
-      if (e0 + lane + 32 * j == bi) key[j] = -INFINITY;
+      if (j == wj) my = lg[j];
+    const float wlog = __shfl_sync(0xffffffffu, my, wl);
+    if (lane == wl) {
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (j == wj) ok[j] = 0u;
+    }
     if (lane == r) {
-      out.key = bk;
-      out.id = bi;
-      out.logit = bl;
+      out.key = key_value(wo);
+      out.id = (int)wi;
+      out.logit = wlog;
     }
   }
 }
@@ -135,24 +142,60 @@ __device__ __forceinline__ void warp_topk_slice_any(const float* logits, const f
     warp_topk_slice<16>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);  // n <= 512
 }
 
+// K rounds over two candidates per lane (candidate slots lane and lane + 32):
+// lane r < K receives the r-th expert and its combine weight.
+__device__ __forceinline__ void topk_pick(uint32_t o0, uint32_t i0, float l0, uint32_t o1, uint32_t i1,
+                                          float l1, int K, int E, int score_fn, int renorm,
+                                          float routed_scale, float mx, float den, int lane,
+                                          int& sel_id, float& sel_w) {
+  sel_id = 0;
+  float sel_src = 0.f, tot = 0.f;
+  for (int r = 0; r < K; ++r) {
+    // local best of the two slots: larger key, then lower index
+    const bool second = o1 > o0 || (o1 == o0 && i1 < i0);
+    const uint32_t bo = second ? o1 : o0, bi = second ? i1 : i0;
+    const uint32_t wo = __reduce_max_sync(0xffffffffu, bo);
+    const uint32_t wi = __reduce_min_sync(0xffffffffu, bo == wo ? bi : kNoExpert);
+    // the lane that holds it: exactly one slot matches (indices are distinct)
+    const bool mine0 = i0 == wi, mine1 = i1 == wi;
+    const unsigned who = __ballot_sync(0xffffffffu, mine0 || mine1);
+    const int wl = who ? __ffs(who) - 1 : 0;
+    const float wlog = __shfl_sync(0xffffffffu, mine1 ? l1 : l0, wl);
+    if (mine0) {
+      o0 = 0u;
+      i0 = kNoExpert;
+    }
+    if (mine1) {
+      o1 = 0u;
+      i1 = kNoExpert;
+    }
+    const float sv = (score_fn == 0) ? __fdividef(__expf(wlog - mx), den) : fast_sigmoid(wlog);
+    tot += sv;
+    if (lane == r) {
+      sel_id = (wi < (uint32_t)E) ? (int)wi : 0;  // out of range only after NaN logits
+      sel_src = sv;
+    }
+  }
+  sel_w = (renorm ? __fdividef(sel_src, tot) : sel_src) * routed_scale;
+}
+
 // Final choice from P slices' candidates (cand[q * K + r], P * K <= 64) and
-// their softmax partials part[q] = {max, sum}; lane r < K receives the r-th
-// expert and its combine weight.
+// their softmax partials part[q] = {max, sum}.
 __device__ __forceinline__ void warp_topk_merge(const TopkCand* cand, const float2* part, int P,
                                                 int K, int E, int score_fn, int renorm,
                                                 float routed_scale, int lane, int& sel_id,
                                                 float& sel_w) {
   const int n = P * K;
-  float k0 = -INFINITY, k1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  int i0 = 0x7fffffff, i1 = 0x7fffffff;
-  if (lane < n) {
-    k0 = cand[lane].key;
-    i0 = cand[lane].id;
+  uint32_t o0 = 0u, o1 = 0u, i0 = kNoExpert, i1 = kNoExpert;
+  float l0 = 0.f, l1 = 0.f;
+  if (lane < n && cand[lane].id != 0x7fffffff) {
+    o0 = key_order(cand[lane].key);
+    i0 = (uint32_t)cand[lane].id;
     l0 = cand[lane].logit;
   }
-  if (lane + 32 < n) {
-    k1 = cand[lane + 32].key;
-    i1 = cand[lane + 32].id;
+  if (lane + 32 < n && cand[lane + 32].id != 0x7fffffff) {
+    o1 = key_order(cand[lane + 32].key);
+    i1 = (uint32_t)cand[lane + 32].id;
     l1 = cand[lane + 32].logit;
   }
   float mx = -INFINITY, den = 1.f;
@@ -162,33 +205,8 @@ __device__ __forceinline__ void warp_topk_merge(const TopkCand* cand, const floa
     for (int q = 0; q < P; ++q) s += part[q].y * __expf(part[q].x - mx);
     den = s;
   }
-  sel_id = 0;
-  float sel_src = 0.f, tot = 0.f;
-  for (int r = 0; r < K; ++r) {
-    float bk = k0, bl = l0;
-    int bi = i0;
-    if (topk_better(k1, i1, bk, bi)) {
-      bk = k1;
-      bi = i1;
-      bl = l1;
-    }
-    warp_best(bk, bi, bl);
-    if (i0 == bi) {
-      k0 = -INFINITY;
-      i0 = 0x7fffffff;
-    }
-    if (i1 == bi) {
-      k1 = -INFINITY;
-      i1 = 0x7fffffff;
-    }
-    const float sv = (score_fn == 0) ? __fdividef(__expf(bl - mx), den) : fast_sigmoid(bl);
-    tot += sv;
-    if (lane == r) {
-      sel_id = (bi >= 0 && bi < E) ? bi : 0;  // out of range only after NaN logits
-      sel_src = sv;
-    }
-  }
-  sel_w = (renorm ? __fdividef(sel_src, tot) : sel_src) * routed_scale;
+  topk_pick(o0, i0, l0, o1, i1, l1, K, E, score_fn, renorm, routed_scale, mx, den, lane, sel_id,
+            sel_w);
 }
 
 // Whole selection for one token on one warp: one slice of up to 512 experts,
@@ -204,38 +222,13 @@ __device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int
   c1.id = 0x7fffffff;
   c1.logit = 0.f;
   if (split < E) warp_topk_slice_any(logits, bias, split, E, K, score_fn, lane, c1, m1, s1);
-  float mx = fmaxf(m0, m1), den = 1.f;
+  const float mx = fmaxf(m0, m1);
+  float den = 1.f;
   if (score_fn == 0) den = s0 * __expf(m0 - mx) + (split < E ? s1 * __expf(m1 - mx) : 0.f);
-  float k0 = lane < K ? c0.key : -INFINITY, k1 = lane < K ? c1.key : -INFINITY;
-  int i0 = lane < K ? c0.id : 0x7fffffff, i1 = lane < K ? c1.id : 0x7fffffff;
-  const float l0 = c0.logit, l1 = c1.logit;
-  sel_id = 0;
-  float sel_src = 0.f, tot = 0.f;
-  for (int r = 0; r < K; ++r) {
-    float bk = k0, bl = l0;
-    int bi = i0;
-    if (topk_better(k1, i1, bk, bi)) {
-      bk = k1;
-      bi = i1;
-      bl = l1;
-    }
-    warp_best(bk, bi, bl);
-    if (i0 == bi) {
-      k0 = -INFINITY;
-      i0 = 0x7fffffff;
-    }
-    if (i1 == bi) {
-      k1 = -INFINITY;
-      i1 = 0x7fffffff;
-    }
-    const float sv = (score_fn == 0) ? __fdividef(__expf(bl - mx), den) : fast_sigmoid(bl);
-    tot += sv;
-    if (lane == r) {
-      sel_id = (bi >= 0 && bi < E) ? bi : 0;  // out of range only after NaN logits
-      sel_src = sv;
-    }
-  }
-  sel_w = (renorm ? __fdividef(sel_src, tot) : sel_src) * routed_scale;
+  const bool v0 = lane < K && c0.id != 0x7fffffff, v1 = lane < K && c1.id != 0x7fffffff;
+  topk_pick(v0 ? key_order(c0.key) : 0u, v0 ? (uint32_t)c0.id : kNoExpert, c0.logit,
+            v1 ? key_order(c1.key) : 0u, v1 ? (uint32_t)c1.id : kNoExpert, c1.logit, K, E,
+            score_fn, renorm, routed_scale, mx, den, lane, sel_id, sel_w);
 }
 
 }  // namespace moe

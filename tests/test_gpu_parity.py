@@ -128,10 +128,12 @@ def test_zero_input_gives_exact_zero(tiny):
     np.testing.assert_allclose(wts, 0.5, rtol=0, atol=1e-7)
 
 
-def test_back_to_back_forwards_read_their_own_inputs(tiny):
+@pytest.mark.parametrize("fused", [0, 1])
+def test_back_to_back_forwards_read_their_own_inputs(tiny, fused, monkeypatch):
     """Two forwards on one stream with different x: a read hoisted above a
     dependency wait would pick up the other step's activations."""
     shape, w = tiny
+    monkeypatch.setenv("MOE_FUSED", str(fused))
     blk = GpuBlock(shape, w, max_tokens=8)
     xa = synth.make_x(shape, tokens=8, step=100)
     xb = synth.make_x(shape, tokens=8, step=101)
@@ -147,8 +149,10 @@ def test_back_to_back_forwards_read_their_own_inputs(tiny):
         assert_close(bf16_to_f32(o.cpu().numpy().view(np.uint16)), ref["out"], "out")
 
 
-def test_deterministic_and_graph_replay(tiny):
+@pytest.mark.parametrize("fused", [0, 1])
+def test_deterministic_and_graph_replay(tiny, fused, monkeypatch):
     shape, w = tiny
+    monkeypatch.setenv("MOE_FUSED", str(fused))
     blk = GpuBlock(shape, w, max_tokens=8)
     x = torch.from_numpy(synth.make_x(shape, tokens=8, step=7).view(np.int16)).cuda()
     o1, o2, o3 = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
@@ -202,6 +206,30 @@ def test_argument_errors(tiny):
         fresh.load(moe.weights_to_device(bad))
     assert ei.value.status == 7
     assert moe.moe_forward(fresh.handle, x, 4, out) == 3
+
+
+@pytest.mark.parametrize("B", [1, 4, 8])
+def test_fused_launch_matches_multi_kernel_path(tiny, B, monkeypatch):
+    """With MOE_FUSED=1 at plan creation, up to 8 tokens run as one fused
+    launch; it must agree with the four-kernel path and with the oracle.
+    The split-K piece boundaries differ, so agreement is to rounding."""
+    shape, w = tiny
+    x = synth.make_x(shape, tokens=B, step=40 + B)
+    monkeypatch.setenv("MOE_FUSED", "1")
+    fused = GpuBlock(shape, w, max_tokens=8)
+    monkeypatch.delenv("MOE_FUSED")
+    assert fused.plan.info().kernels_per_forward == 1
+    multi = GpuBlock(shape, w, max_tokens=8)
+    assert multi.plan.info().kernels_per_forward == 4
+    of = bf16_to_f32(fused.run(x))
+    om = bf16_to_f32(multi.run(x))
+    ref = oracle.forward(shape, w, x, intermediates=False)
+    assert_close(of, ref["out"], "fused out")
+    assert_close(om, ref["out"], "multi-kernel out")
+    assert_close(of, om, "fused vs multi-kernel", max_rel=1e-2, mean_rel=1e-3)
+    ids_f, w_f = fused.plan.routing(B)
+    ids_m, w_m = multi.plan.routing(B)
+    assert np.array_equal(np.sort(ids_f, axis=1), np.sort(ids_m, axis=1))
 
 
 # ---------------------------------------------------------------------------
