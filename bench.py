@@ -220,6 +220,39 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 
 
+def _sources_digest() -> str:
+    """sha256 over the CUDA sources and the C header: DRAM counters taken from
+    an ncu capture apply only to the kernels these sources build."""
+    import hashlib
+    h = hashlib.sha256()
+    root = os.path.dirname(os.path.abspath(__file__))
+    csrc = os.path.join(root, "mxfp4_latent_moe_router_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    files.append(os.path.join(root, "include", "moe.h"))
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def _measured_traffic(workload: str) -> dict:
+    """Per-launch DRAM bytes (read + write) per kernel from the committed ncu
+    summary profiles/dram_traffic_<workload>.txt ("key = value" lines), or {}
+    when there is none or it was taken from different sources."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                        "dram_traffic_%s.txt" % workload)
+    if not os.path.exists(path):
+        return {}
+    kv = {}
+    for line in open(path):
+        if "=" in line and not line.lstrip().startswith("#"):
+            k, v = line.split("=", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("sources_sha256") != _sources_digest():
+        return {}
+    return {k[len("bytes."):]: float(v) for k, v in kv.items() if k.startswith("bytes.")}
+
+
 def run_ours(args):
     import torch
     import mxfp4_latent_moe_router_b200 as moe
@@ -342,9 +375,10 @@ def run_ours(args):
                   "latent_tail": 2 * L * H + 2 * Is * H}
     kern_bytes["fused_block"] = sum(kern_bytes.values())  # one launch streams them all
     dom = max(kern_us, key=lambda n: kern_us[n])
+    traffic = _measured_traffic(args.workload)
     ach = kern_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9 if kern_us[dom] > 0 else 0.0
     roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-            "frac": ach / hbm_peak, "traffic": None, "peak_source": peak_src,
+            "frac": ach / hbm_peak, "traffic": traffic.get(dom), "peak_source": peak_src,
             "algorithmic_bytes_per_launch": kern_bytes[dom], "launch_us": kern_us[dom],
             "per_kernel_us": kern_us,
             "per_kernel_gbs": {n: (kern_bytes[n] / (kern_us[n] * 1e-6) / 1e9 if kern_us[n] > 0 else None)

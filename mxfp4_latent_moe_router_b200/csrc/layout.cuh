@@ -53,19 +53,20 @@ __host__ __device__ constexpr int frag_k(int t, int s, int q, int e) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Pieces per row block (split-K factor) that minimise the makespan of `mats`
-// row blocks of C chunks each, dealt dynamically to `ctas` CTAs:
-//   rounds x (chunks per piece + split_cost when split),
-// rounds = ceil(mats * ppr / ctas).  split_cost is the price of a split-K
-// piece end (partial sums out, a ticket, sometimes the finalising sums) in
-// chunk-stage units.  Splitting only pays when it shortens the last round.
+// Pieces per row block (split-K factor) for `mats` row blocks of C chunks
+// each, dealt dynamically to `ctas` CTAs.  A dynamic schedule ends within one
+// piece of the average load, and CTAs arrive skewed, so the estimate is
+//   total work / ctas + one piece,
+// a piece costing its chunks plus, when split, split_cost: the price of a
+// split-K piece end (partial sums out, a ticket, sometimes the finalising
+// sums) in chunk-stage units.
 __host__ __device__ inline int best_ppr(int mats, int C, int ctas, int split_cost) {
   if (mats <= 0 || ctas <= 0 || C <= 1) return 1;
   int best = 1;
   long long best_t = -1;
   for (int ppr = 1; ppr <= C; ++ppr) {
-    const long long rounds = ((long long)mats * ppr + ctas - 1) / ctas;
-    const long long t = rounds * (ceil_div(C, ppr) + (ppr > 1 ? split_cost : 0));
+    const long long piece = ceil_div(C, ppr) + (ppr > 1 ? split_cost : 0);
+    const long long t = ((long long)mats * ppr * piece + ctas - 1) / ctas + piece;
     if (best_t < 0 || t < best_t) {
       best_t = t;
       best = ppr;

@@ -285,9 +285,9 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
 // split-K factor of a kind whose row-block count the host knows
 int ppr_for(int mats, int C, int ctas) { return best_ppr(mats, C, ctas, g_split_cost); }
 
-// Router row blocks get pieces a third of the others' size: they are the
-// first pieces handed out, and the routing waits for all of them.
-int router_ppr(int ppr, int C) { return std::max(1, std::min(C, 3 * ppr)); }
+// Router row blocks are the first pieces handed out and the routing waits
+// for all of them: they get pieces of at most ~C/12 chunks.
+int router_ppr(int ppr, int C) { return std::max(1, std::min(C, std::max(ppr, 12))); }
 
 // largest number of partial-sum floats a kind can need for B <= maxB
 size_t partial_floats(const moe_plan_s* p, int kind) {
