@@ -243,6 +243,17 @@ __device__ __forceinline__ bool wait_flag(const int* flag, int* err, int err_bit
   return false;
 }
 
+// Bounded wait until *counter >= target (acquire); false and an error bit on
+// expiry.
+__device__ __forceinline__ bool wait_count(const int* counter, int target, int* err, int lane) {
+  for (uint32_t i = 0; i < (1u << 22); ++i) {
+    if (ld_acquire(counter) >= target) return true;
+    __nanosleep(128);
+  }
+  if (lane == 0) atomicOr(err, 1 << ERR_WAIT_ROUTE);
+  return false;
+}
+
 template <int KIND>
 __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t* tables,
                          uint64_t* full, uint64_t* empty, int lane) {
@@ -713,8 +724,8 @@ __device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int wa
   named_sync(1, kConsumerThreads);
 }
 
-__device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, int* wtot, int tid,
-                                          int warp, int lane, bool dry);
+__device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
+                                          int* wtot, int tid, int warp, int lane, bool dry);
 
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
@@ -824,8 +835,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
 // dry: the same instructions with every global store skipped (a rehearsal
 // that brings the code into the instruction cache while the logits are not
 // ready yet; its shared-memory results are discarded)
-__device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, int* wtot, int tid,
-                                          int warp, int lane, bool dry) {
+__device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
+                                          int* wtot, int tid, int warp, int lane, bool dry) {
   const int E = p.E, K = p.topk, B = p.B;
   const int tg = p.tg > 0 ? p.tg : 1;
   int* cnt = reinterpret_cast<int*>(scratch);  // [E] slots per expert
@@ -846,7 +857,7 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
     for (int b = warp; b < B; b += kConsumerWarps) {
       int sel_id;
       float sel_w;
-      warp_topk(p.logits + (long long)b * E, E, K, p.score_fn, p.bias, p.renorm, p.routed_scale,
+      warp_topk(p.logits + (long long)b * E, E, K, p.score_fn, bias, p.renorm, p.routed_scale,
                 lane, sel_id, sel_w);
       if (lane < K) {
         if (!dry) {
@@ -867,11 +878,12 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
       const int e0 = (int)((long long)q * E / P), e1 = (int)((long long)(q + 1) * E / P);
       TopkCand c;
       float smax, ssum;
-      warp_topk_slice_any(p.logits + (long long)b * E, p.bias, e0, e1, K, p.score_fn, lane, c, smax,
+      warp_topk_slice_any(p.logits + (long long)b * E, bias, e0, e1, K, p.score_fn, lane, c, smax,
                           ssum);
       if (lane < K) cand[(b * P + q) * K + lane] = c;
       if (lane == 0) part[b * P + q] = make_float2(smax, ssum);
     }
+    if (tr) tr[21] = global_ns();
     named_sync(1, kConsumerThreads);
     if (warp < B) {
       const int b = warp;
@@ -879,6 +891,7 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
       float sel_w;
       warp_topk_merge(cand + b * P * K, part + b * P, P, K, E, p.score_fn, p.renorm,
                       p.routed_scale, lane, sel_id, sel_w);
+      if (tr) tr[22] = global_ns();
       if (lane < K) {
         if (!dry) {
           p.ids[b * K + lane] = sel_id;
@@ -957,13 +970,21 @@ __device__ __forceinline__ void route_tokens(const Params& p, uint8_t* scratch, 
 // every router row block has been summed, select the experts, build the
 // per-expert token lists and publish them; the other CTAs keep streaming the
 // latent and shared-expert rows meanwhile.
-__device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, int* sm_flag, int tid,
-                                          int warp, int lane) {
+__device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, float* bias_s,
+                                          int* sm_flag, int tid, int warp, int lane) {
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
+  // the selection bias is static: stage it in shared memory before the
+  // logits exist, so the selection waits on one round trip, not two
+  const float* bias = nullptr;
+  if (p.bias) {
+    for (int i = tid; i < p.E; i += kConsumerThreads) bias_s[i] = __ldg(p.bias + i);
+    bias = bias_s;
+  }
+  named_sync(1, kConsumerThreads);
   // Selection is a short serial program run once per forward: cold, every
   // instruction fetch would miss and queue behind the HBM stream.  Rehearse
   // it on whatever the logits buffer holds while the router rows stream.
-  route_tokens(p, scratch, sm_flag + 16, tid, warp, lane, true);
+  route_tokens(p, bias, scratch, sm_flag + 16, tid, warp, lane, true);
   if (tr && tid == 0) tr[20] = global_ns();
   if (tid == 0) {
     bool ok = false;
@@ -980,7 +1001,7 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, int
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
   if (!sm_flag[0]) return;
   if (tr && tid == 0) tr[4] = global_ns();
-  route_tokens(p, scratch, sm_flag + 16, tid, warp, lane, false);  // ends with a barrier
+  route_tokens(p, bias, scratch, sm_flag + 16, tid, warp, lane, false);  // ends with a barrier
   if (tid == 0) {
     if (tr) tr[5] = global_ns();
     *p.router_done = 0;
@@ -1268,7 +1289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // it writes the routing tables the previous forward's tail reads
     pdl_wait();
     pdl_trigger();
-    if (warp < kConsumerWarps) route_cta(p, scratch, sm_flag, threadIdx.x, warp, lane);
+    if (warp < kConsumerWarps)
+      route_cta(p, scratch, reinterpret_cast<float*>(stages), sm_flag, threadIdx.x, warp, lane);
   } else if (warp == kConsumerWarps) {
     producer<KIND>(p, ctl, stages, tables, full, empty, lane);
   } else {

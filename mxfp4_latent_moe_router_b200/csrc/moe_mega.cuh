@@ -41,17 +41,6 @@ struct MegaProd {
   bool in_flight;
 };
 
-// Bounded wait until *counter >= target (acquire); false and an error bit on
-// expiry.
-__device__ __forceinline__ bool wait_count(const int* counter, int target, int* err, int lane) {
-  for (uint32_t i = 0; i < (1u << 22); ++i) {
-    if (ld_acquire(counter) >= target) return true;
-    __nanosleep(128);
-  }
-  if (lane == 0) atomicOr(err, 1 << ERR_WAIT_ROUTE);
-  return false;
-}
-
 // Blocking: phase KIND's activations may be read.
 template <int KIND>
 __device__ __forceinline__ void mega_wait_deps(const MegaParams& mp, const MegaProd& st, int lane) {
@@ -523,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_mega_kernel(const __grid_cons
     // the routing CTA: it writes the routing tables the previous forward read
     pdl_wait();
     pdl_trigger();
-    if (warp < kConsumerWarps) route_cta(pf, scratch, sm_flag, threadIdx.x, warp, lane);
+    if (warp < kConsumerWarps)
+      route_cta(pf, scratch, reinterpret_cast<float*>(stages), sm_flag, threadIdx.x, warp, lane);
   } else if (warp == kConsumerWarps) {
     mega_producer(mp, stages, tables, full, empty, lane);
   } else {

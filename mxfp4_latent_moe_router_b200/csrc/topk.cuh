@@ -57,7 +57,7 @@ __device__ __forceinline__ void warp_topk_slice(const float* logits, const float
     const int e = e0 + lane + 32 * j;
     const bool in = e < e1;
     lg[j] = in ? __ldcg(logits + e) : 0.f;
-    bs[j] = (in && bias) ? __ldg(bias + e) : 0.f;
+    bs[j] = (in && bias) ? bias[e] : 0.f;  // (global or shared memory)
   }
   float mx = -INFINITY;
 #pragma unroll
