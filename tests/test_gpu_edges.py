@@ -1,0 +1,79 @@
+"""Edge cases of the CUDA path against the CPU oracle: the largest expert count
+and top-k the library takes, the largest batch, sigmoid scoring without a
+selection bias, and the fused single launch with a tail activation too large
+to keep in shared memory."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import mxfp4_latent_moe_router_b200 as moe  # noqa: E402
+from mxfp4_latent_moe_router_b200 import synth  # noqa: E402
+from helpers import assert_close, bf16_to_f32, check_routing  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(shape, w, x, max_tokens):
+    plan = moe.MoePlan(moe.config_from_shape(shape, max_tokens=max_tokens))
+    try:
+        plan.load(moe.weights_to_device(w))
+        xd = torch.from_numpy(x.view(np.int16)).cuda()
+        out = torch.empty_like(xd)
+        plan.forward(xd, out)
+        torch.cuda.synchronize()
+        assert plan.sync_status() == 0
+        B = x.shape[0]
+        ids, wts = plan.routing(B)
+        logits = plan.fetch(moe.MOE_DBG_LOGITS, B)
+        return out.cpu().numpy().view(np.uint16), ids, wts, logits
+    finally:
+        plan.close()
+
+
+def _check(shape, w, x, max_tokens):
+    out, ids, wts, logits = _run(shape, w, x, max_tokens)
+    orc = oracle.forward(shape, w, x, intermediates=False)
+    near = check_routing(shape, w, x, ids, wts, logits, orc)
+    ok = [b for b in range(x.shape[0]) if b not in near]
+    assert_close(bf16_to_f32(out[ok]), orc["out"][ok], shape.name + " out")
+    return ids, near
+
+
+@pytest.mark.parametrize("B", [3, 9])
+def test_largest_expert_count_and_top_k(B):
+    # E = 1024 and k = 16 are the library's limits; B = 3 splits each token's
+    # experts over two warps, B = 9 selects from two 512-expert slices on one
+    shape = synth.custom_shape("e1024", B, 256, 128, 1024, 16, 64, 64, synth.SCORE_SIGMOID,
+                               seed=61 + B, scale_exp_lo=-5, scale_exp_hi=-2)
+    w = synth.make_weights(shape)
+    ids, near = _check(shape, w, synth.make_x(shape), max_tokens=16)
+    assert all(len(set(r.tolist())) == 16 for r in ids)
+
+
+def test_largest_batch():
+    # B = 128 (the library's limit) in one forward: sixteen 8-token tiles in
+    # the front kernel, token groups in the expert kernels, several tail passes
+    shape = synth.custom_shape("b128-small", 128, 512, 256, 32, 4, 128, 128,
+                               synth.SCORE_SOFTMAX, seed=71)
+    w = synth.make_weights(shape)
+    _check(shape, w, synth.make_x(shape), max_tokens=128)
+
+
+def test_sigmoid_without_selection_bias():
+    shape = synth.custom_shape("nobias", 6, 256, 128, 24, 3, 64, 64, synth.SCORE_SIGMOID, seed=81)
+    w = dict(synth.make_weights(shape))
+    w["router_bias"] = None
+    _check(shape, w, synth.make_x(shape), max_tokens=8)
+
+
+def test_fused_launch_with_staged_tail(monkeypatch):
+    # L + I_s = 3072: eight tokens' tail activation (about 98 KB as bf16 hi/lo)
+    # does not fit the shared-memory budget, so the fused launch stages y and
+    # h_s per chunk instead
+    shape = synth.custom_shape("staged", 8, 256, 1024, 16, 2, 128, 2048, synth.SCORE_SOFTMAX,
+                               seed=91, scale_exp_lo=-5, scale_exp_hi=-2)
+    w = synth.make_weights(shape)
+    monkeypatch.setenv("MOE_FUSED", "1")
+    _check(shape, w, synth.make_x(shape), max_tokens=8)
