@@ -87,7 +87,9 @@ typedef struct moe_config {
  *   w_out      bf16 [L][H]
  *   gu_codes   u8   [E][2I][L/2]   rows 0..I-1 gate, rows I..2I-1 up;
  *                                  element 2t in the low nibble of byte t
- *   gu_scales  u8   [E][2I][L/32]  e8m0, value 2^(s-127); 0xFF (NaN) rejected
+ *   gu_scales  u8   [E][2I][L/32]  e8m0, value 2^(s-127); 0xFF (NaN) rejected;
+ *                                  0 (2^-127) is applied as 0 (every weight of
+ *                                  such a block is below fp32's normal range)
  *   dn_codes   u8   [E][L][I/2]
  *   dn_scales  u8   [E][L][I/32]
  *   sh_gate    bf16 [H][I_s]   (ignored when I_s == 0)
@@ -198,12 +200,17 @@ MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
  * Per-CTA timeline of the most recent forward, for measurement only; exists
  * when the plan was created with the environment variable MOE_TRACE set
  * (else MOE_ERR_UNSUPPORTED).  host receives count = 5 * num_sms * 24 uint64:
- * for kernel kind k (launch order as in moe_get_profile) and CTA c, the 24
- * values at (k * num_sms + c) * 24 are {start ns, end ns, pieces, finalizes,
- * top-k start ns, top-k end ns, first stage ready ns, finalize ns, consumer
- * cycles waiting for data, computing, closing pieces, producer cycles waiting
- * for a free stage, issuing, stages issued, 0, 0} (ns from globaltimer,
- * cycles from clock64); value 14 is the SM the CTA ran on.
+ * for launch slot k (as in moe_get_profile) and CTA c, the 24 values at
+ * (k * num_sms + c) * 24 are (ns from globaltimer, cycles from clock64):
+ *   0 start ns, 1 end ns, 2 pieces, 3 finalizes, 4/5 top-k start/end ns (the
+ *   routing CTA), 6 first stage ready ns, 7 ns spent finalising, 8..10
+ *   consumer cycles waiting for data / computing / closing pieces (8..11 in
+ *   the fused slot: ns the producer took its first piece of each phase),
+ *   11..13 producer cycles waiting for a free stage / issuing / stages issued,
+ *   14 the SM the CTA ran on, 15..18 fused slot: ns of the consumers' first
+ *   stage of each phase (the routing CTA: top-k phase stamps in 16..18),
+ *   19 ns the router logits of a row block were published, 20..22 routing CTA:
+ *   rehearsal end, slice selection end, merge end.
  * Synchronises the device.
  */
 MOE_API moe_status moe_debug_trace(moe_plan p, uint64_t *host, int64_t count);

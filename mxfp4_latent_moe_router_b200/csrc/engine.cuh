@@ -27,7 +27,7 @@ enum : int {
   ERR_WAIT_FULL = 0,
   ERR_WAIT_EMPTY = 1,
   ERR_NAN_SCALE = 2,
-  ERR_WAIT_ROUTE = 3,  // the routing tables never became ready
+  ERR_WAIT_DEP = 3,  // a routing flag or a phase-completion count never arrived
 };
 
 struct VExpert {  // one token group of one routed expert

@@ -773,7 +773,7 @@ moe_status moe_sync_status(moe_plan p) {
   CUDA_TRY(cudaMemcpy(&err, p->err, sizeof(int), cudaMemcpyDeviceToHost));
   if (err) {
     CUDA_TRY(cudaMemset(p->err, 0, sizeof(int)));
-    if (err & ((1 << ERR_WAIT_FULL) | (1 << ERR_WAIT_EMPTY))) return MOE_ERR_TIMEOUT;
+    if (err & ((1 << ERR_WAIT_FULL) | (1 << ERR_WAIT_EMPTY) | (1 << ERR_WAIT_DEP))) return MOE_ERR_TIMEOUT;
     return MOE_ERR_RANGE;
   }
   return MOE_OK;

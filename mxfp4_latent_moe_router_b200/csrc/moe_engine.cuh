@@ -93,11 +93,12 @@ struct Space {
   int ppr;
 };
 
+// V: virtual experts (the routing's nve), read by the caller together with
+// the routing tables so that sizing the space costs no extra round trip
 template <int KIND>
-__device__ __forceinline__ Space make_space(const Params& p) {
+__device__ __forceinline__ Space make_space(const Params& p, int V = 0) {
   Space s;
   if (KIND == KIND_EGU || KIND == KIND_EDN) {
-    const int V = *reinterpret_cast<volatile int*>(p.nve);
     const int mats = V * p.RB;
     const int ppr = best_ppr(mats, p.C, p.piece_ctas, p.split_cost);
     s.ppr = ppr;
@@ -250,7 +251,7 @@ __device__ __forceinline__ bool wait_count(const int* counter, int target, int* 
     if (ld_acquire(counter) >= target) return true;
     __nanosleep(128);
   }
-  if (lane == 0) atomicOr(err, 1 << ERR_WAIT_ROUTE);
+  if (lane == 0) atomicOr(err, 1 << ERR_WAIT_DEP);
   return false;
 }
 
@@ -278,16 +279,19 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   // kernel can launch, so the wait ends): wait for its flag, then read the
   // tables and start streaming the chosen experts' tiles before this kernel's
   // own dependency resolves.
-  const bool route_ok = KindTraits<KIND>::kDynamicSpace ? wait_flag(p.route_ready, p.err, ERR_WAIT_ROUTE, lane) : true;
+  const bool route_ok = KindTraits<KIND>::kDynamicSpace ? wait_flag(p.route_ready, p.err, ERR_WAIT_DEP, lane) : true;
+  int V = 0;
   if (KindTraits<KIND>::kDynamicSpace && route_ok) {
-    // L2 reads: the tables were written by another kernel that may still run
+    // L2 reads, all in one round trip: the tables and the count were written
+    // by another kernel that may still run
+    V = __ldcg(p.nve);
     for (int i = lane; i < p.ve_max; i += 32) {
       const int4 v = __ldcg(reinterpret_cast<const int4*>(p.ve + i));
       ve_tab[i] = VExpert{v.x, v.y, v.z, v.w};
     }
     for (int i = lane; i < p.ld_slots; i += 32) slot_tab[i] = __ldcg(p.slots_sorted + i);
   }
-  sp = make_space<KIND>(p);
+  sp = make_space<KIND>(p, V);
   if (!route_ok) sp.total = 0;  // no pieces: straight to the end marker
   __syncwarp();
 
@@ -995,7 +999,7 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
       }
       __nanosleep(64);
     }
-    if (!ok) atomicOr(p.err, 1 << ERR_WAIT_ROUTE);
+    if (!ok) atomicOr(p.err, 1 << ERR_WAIT_DEP);
     sm_flag[0] = ok ? 1 : 0;
   }
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads

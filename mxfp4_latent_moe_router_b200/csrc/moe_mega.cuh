@@ -63,18 +63,19 @@ __device__ __forceinline__ void mega_wait_deps(const MegaParams& mp, const MegaP
 __device__ __forceinline__ void mega_route(const MegaParams& mp, MegaProd& st, VExpert* ve_tab,
                                            int* slot_tab, int lane) {
   const Params& pe = mp.k[KIND_EGU];
-  const bool ok = wait_flag(pe.route_ready, pe.err, ERR_WAIT_ROUTE, lane);
+  const bool ok = wait_flag(pe.route_ready, pe.err, ERR_WAIT_DEP, lane);
   st.V = 0;
   if (ok) {
-    // L2 reads: the tables were written by another CTA of this launch
+    // L2 reads, all in one round trip: the tables and the count were written
+    // by another CTA of this launch
+    st.V = __ldcg(pe.nve);
     for (int i = lane; i < pe.ve_max; i += 32) {
       const int4 v = __ldcg(reinterpret_cast<const int4*>(pe.ve + i));
       ve_tab[i] = VExpert{v.x, v.y, v.z, v.w};
     }
     for (int i = lane; i < pe.ld_slots; i += 32) slot_tab[i] = __ldcg(pe.slots_sorted + i);
-    st.V = __ldcg(pe.nve);
-    st.sp[KIND_EGU] = make_space<KIND_EGU>(pe);
-    st.sp[KIND_EDN] = make_space<KIND_EDN>(mp.k[KIND_EDN]);
+    st.sp[KIND_EGU] = make_space<KIND_EGU>(pe, st.V);
+    st.sp[KIND_EDN] = make_space<KIND_EDN>(mp.k[KIND_EDN], st.V);
   } else {
     st.sp[KIND_EGU].total = st.sp[KIND_EDN].total = 0;
     st.sp[KIND_EGU].ppr = st.sp[KIND_EDN].ppr = 1;
@@ -290,7 +291,7 @@ __device__ __forceinline__ bool mega_piece(const Params& p, MegaCons& cs, uint8_
     // The resident activation reads y, the combine weights and h_s: acquire
     // the phases that wrote them (the producer has already seen them done).
     if (tid == 0) {
-      wait_flag(p.route_ready, p.err, ERR_WAIT_ROUTE, lane);  // combine weights, nve
+      wait_flag(p.route_ready, p.err, ERR_WAIT_DEP, lane);  // combine weights, nve
       const int V = __ldcg(p.nve);
       wait_count(p.done + 3, V * p.need_rb_edn, p.err, lane);
       wait_count(p.done + 1, p.need_rb_sh, p.err, lane);
