@@ -209,8 +209,8 @@ MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
  *   11..13 producer cycles waiting for a free stage / issuing / stages issued,
  *   14 the SM the CTA ran on, 15..18 fused slot: ns of the consumers' first
  *   stage of each phase (the routing CTA: top-k phase stamps in 16..18),
- *   19 ns the router logits of a row block were published, 20..22 routing CTA:
- *   rehearsal end, slice selection end, merge end.
+ *   19 ns the router logits of a row block were published, 21..22 routing
+ *   CTA: slice selection end, merge end.
  * Synchronises the device.
  */
 MOE_API moe_status moe_debug_trace(moe_plan p, uint64_t *host, int64_t count);

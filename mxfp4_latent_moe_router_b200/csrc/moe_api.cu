@@ -413,7 +413,6 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
 
   TRY(alloc(p, &v, sizeof(float) * maxB * E, false));
   p->logits = (float*)v;
-  CUDA_TRY(cudaMemset(v, 0, sizeof(float) * maxB * E));  // read by the top-k rehearsal
   TRY(alloc(p, &v, (size_t)maxB * ceil_div(L, kMxChunkK) * kActRecBytes, false));
   p->z_mx = (uint8_t*)v;
   TRY(alloc(p, &v, sizeof(float) * (size_t)ceil_div(std::max(Is, 1), 64) * maxB * 64, false));

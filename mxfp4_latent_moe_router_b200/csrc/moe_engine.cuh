@@ -74,8 +74,6 @@ struct KindTraits {
   static constexpr bool kMx = (KIND == KIND_EGU || KIND == KIND_EDN);
   static constexpr int kTileBytes = kMx ? kMxTileBytes : kDenseTileBytes;
   static constexpr int kChunkK = kMx ? kMxChunkK : kDenseChunkK;
-  // every kind streams one ring of weight tiles before its dependency resolves
-  static constexpr bool kPrefetchWeights = true;
   static constexpr bool kDynamicSpace = (KIND == KIND_EGU || KIND == KIND_EDN);
 };
 
@@ -261,13 +259,10 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   int stage = 0;
   uint32_t ephase = 1;  // empty barriers start "released"
   Space sp;
-  int prefetched = 0;  // stages filled with weights only, waiting for pdl_wait
+  // every kind streams up to one ring of weight tiles before its dependency
+  // resolves (stages filled with weights only, their activations pending)
+  int prefetched = 0;
   bool waited = false;
-  if (!KindTraits<KIND>::kPrefetchWeights) {
-    pdl_wait();
-    pdl_trigger();
-    waited = true;
-  }
   // routing tables in shared memory: the per-stage lookups then cost no
   // global round trip (they are visible to the consumers through the first
   // full-barrier completion).  The whole capacity is copied so that these
@@ -729,7 +724,7 @@ __device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int wa
 }
 
 __device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
-                                          int* wtot, int tid, int warp, int lane, bool dry);
+                                          int* wtot, int tid, int warp, int lane);
 
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
@@ -836,11 +831,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
 // top-k routing and per-expert token lists (one CTA, 256 threads); the
 // per-token selection is warp_topk (topk.cuh).
 
-// dry: the same instructions with every global store skipped (a rehearsal
-// that brings the code into the instruction cache while the logits are not
-// ready yet; its shared-memory results are discarded)
 __device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
-                                          int* wtot, int tid, int warp, int lane, bool dry) {
+                                          int* wtot, int tid, int warp, int lane) {
   const int E = p.E, K = p.topk, B = p.B;
   const int tg = p.tg > 0 ? p.tg : 1;
   int* cnt = reinterpret_cast<int*>(scratch);  // [E] slots per expert
@@ -864,10 +856,8 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
       warp_topk(p.logits + (long long)b * E, E, K, p.score_fn, bias, p.renorm, p.routed_scale,
                 lane, sel_id, sel_w);
       if (lane < K) {
-        if (!dry) {
-          p.ids[b * K + lane] = sel_id;
-          p.wts[b * K + lane] = sel_w;
-        }
+        p.ids[b * K + lane] = sel_id;
+        p.wts[b * K + lane] = sel_w;
         ids_s[b * K + lane] = sel_id;
         atomicAdd(&cnt[sel_id], 1);
       }
@@ -897,10 +887,8 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
                       p.routed_scale, lane, sel_id, sel_w);
       if (tr) tr[22] = global_ns();
       if (lane < K) {
-        if (!dry) {
-          p.ids[b * K + lane] = sel_id;
-          p.wts[b * K + lane] = sel_w;
-        }
+        p.ids[b * K + lane] = sel_id;
+        p.wts[b * K + lane] = sel_w;
         ids_s[b * K + lane] = sel_id;
         atomicAdd(&cnt[sel_id], 1);
       }
@@ -950,19 +938,19 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
         ve.start = bc + gi * tg;
         ve.count = min(tg, c[i] - gi * tg);
         ve.pad = 0;
-        if (!dry && bg + gi < p.ve_max) p.ve[bg + gi] = ve;
+        if (bg + gi < p.ve_max) p.ve[bg + gi] = ve;
       }
     }
     bc += c[i];
     bg += gsz[i];
   }
-  if (!dry && tid == kConsumerThreads - 1) *p.nve = bg < p.ve_max ? bg : p.ve_max;
+  if (tid == kConsumerThreads - 1) *p.nve = bg < p.ve_max ? bg : p.ve_max;
   named_sync(1, kConsumerThreads);
   if (tr) tr[18] = global_ns();
   for (int s = tid; s < B * K; s += kConsumerThreads) {
     const int e = ids_s[s];
     const int pos = off[e] + atomicAdd(&fill[e], 1);
-    if (!dry) p.slots_sorted[pos] = s;
+    p.slots_sorted[pos] = s;
   }
   named_sync(1, kConsumerThreads);
 }
@@ -985,11 +973,6 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
     bias = bias_s;
   }
   named_sync(1, kConsumerThreads);
-  // Selection is a short serial program run once per forward: cold, every
-  // instruction fetch would miss and queue behind the HBM stream.  Rehearse
-  // it on whatever the logits buffer holds while the router rows stream.
-  route_tokens(p, bias, scratch, sm_flag + 16, tid, warp, lane, true);
-  if (tr && tid == 0) tr[20] = global_ns();
   if (tid == 0) {
     bool ok = false;
     for (uint32_t i = 0; i < (1u << 22); ++i) {
@@ -1005,7 +988,7 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
   if (!sm_flag[0]) return;
   if (tr && tid == 0) tr[4] = global_ns();
-  route_tokens(p, bias, scratch, sm_flag + 16, tid, warp, lane, false);  // ends with a barrier
+  route_tokens(p, bias, scratch, sm_flag + 16, tid, warp, lane);  // ends with a barrier
   if (tid == 0) {
     if (tr) tr[5] = global_ns();
     *p.router_done = 0;
