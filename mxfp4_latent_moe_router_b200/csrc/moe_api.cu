@@ -282,8 +282,12 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   }
 }
 
+// Price of a split-K piece end in stages: partial sums out and the
+// finalising sums back in both grow with the piece's token tiles.
+int split_cost_for(int nt) { return g_split_cost * std::max(1, nt); }
+
 // split-K factor of a kind whose row-block count the host knows
-int ppr_for(int mats, int C, int ctas) { return best_ppr(mats, C, ctas, g_split_cost); }
+int ppr_for(int mats, int C, int ctas, int nt) { return best_ppr(mats, C, ctas, split_cost_for(nt)); }
 
 // Router row blocks are the first pieces handed out and the routing waits
 // for all of them: they get pieces of at most ~C/12 chunks.
@@ -299,18 +303,18 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     const KindGeom& g = p->g[kind];
     if (kind == KIND_FRONT) {
       nt = f.nt_front;
-      const int ppr = ppr_for(g.RB, g.C, f.front_workers);
+      const int ppr = ppr_for(g.RB, g.C, f.front_workers, nt);
       pieces = (size_t)p->RB_router * router_ppr(ppr, g.C) + (size_t)(g.RB - p->RB_router) * ppr;
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      pieces = (size_t)passes * g.RB * ppr_for(g.RB * passes, g.C, f.tail_grid);
+      pieces = (size_t)passes * g.RB * ppr_for(g.RB * passes, g.C, f.tail_grid, nt);
     } else {
       nt = f.nt_e;
       // the split depends on the routing: take the largest over every
       // possible count of virtual experts
       for (int V = 1; V <= p->ve_max; ++V)
-        pieces = std::max(pieces, (size_t)V * g.RB * ppr_for(V * g.RB, g.C, f.expert_grid));
+        pieces = std::max(pieces, (size_t)V * g.RB * ppr_for(V * g.RB, g.C, f.expert_grid, nt));
     }
     best = std::max(best, pieces * (size_t)nt * 1024);
   }
@@ -515,12 +519,12 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
     q.need_rb_edn = p->g[KIND_EDN].RB;
     q.need_rb_sh = p->g[KIND_FRONT].RB - p->RB_router - p->RB_lat;
     if (k == KIND_FRONT) {
-      q.PPR = ppr_for(q.RB, q.C, f.front_workers);
+      q.PPR = ppr_for(q.RB, q.C, f.front_workers, 1);
       q.PPR_r = router_ppr(q.PPR, q.C);
       mp.n_front = p->RB_router * q.PPR_r + (q.RB - p->RB_router) * q.PPR;
     } else if (k == KIND_EGU || k == KIND_EDN) {
       q.piece_ctas = f.expert_grid;
-      q.split_cost = g_split_cost;
+      q.split_cost = split_cost_for(1);
     } else {
       if (res_bytes) {
         q.res_off = kStageOff + table_bytes;
@@ -528,7 +532,7 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
         q.res_k = res_k;
       }
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid);
+      q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid, 1);
     }
     mp.k[k] = q;
   }
@@ -562,7 +566,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     Params q = base;
     const SmemGeom sm = smem_geom(KIND_FRONT, f.nt_front, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_FRONT, sm);
-    q.PPR = ppr_for(q.RB, q.C, f.front_workers);
+    q.PPR = ppr_for(q.RB, q.C, f.front_workers, f.nt_front);
     q.PPR_r = router_ppr(q.PPR, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_FRONT, f.nt_front, q, f.front_grid, sm.total, s, p->use_pdl));
@@ -573,7 +577,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EGU, sm);
     q.piece_ctas = f.expert_grid;
-    q.split_cost = g_split_cost;
+    q.split_cost = split_cost_for(f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
@@ -583,7 +587,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
     set_kind(q, p, KIND_EDN, sm);
     q.piece_ctas = f.expert_grid;
-    q.split_cost = g_split_cost;
+    q.split_cost = split_cost_for(f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
@@ -602,7 +606,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       q.res_k = res_k;
     }
     const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-    q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid);
+    q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid, f.nt_tail);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][1], s));

@@ -426,7 +426,12 @@ __device__ __forceinline__ void mma_dense_x(const Params& p, const Hdr& h, const
         const uint32_t A0[4] = {a[b][0].x, a[b][0].y, a[b][0].z, a[b][0].w};
         const uint32_t A1[4] = {a[b][1].x, a[b][1].y, a[b][1].z, a[b][1].w};
         mma_bf16(acc[t], A0, bv[b].x, bv[b].y);
-        mma_bf16(acc2[t], A1, bv[b].z, bv[b].w);
+        // four or more tiles give the tensor pipe independent MMAs already:
+        // one accumulator set, half the registers
+        if constexpr (NT >= 4)
+          mma_bf16(acc[t], A1, bv[b].z, bv[b].w);
+        else
+          mma_bf16(acc2[t], A1, bv[b].z, bv[b].w);
       }
     }
   }
@@ -449,9 +454,76 @@ __device__ __forceinline__ float e8m0_byte_to_float(uint32_t word, int j) {
   return __uint_as_float(t & 0x7F800000u);
 }
 
+// Several token tiles (a virtual expert of up to 8*NT tokens): the 32-wide
+// blocks are decoded four at a time (codes and scales into registers) and
+// each decoded half serves every tile that holds tokens of this piece; tiles
+// past ceil(ntok/8) are skipped (the test is uniform over the CTA), so an
+// expert chosen by 2 tokens costs one tile.  A tile's shared-memory loads are
+// issued together before its MMAs, as in the one-tile loop below.  (Halves,
+// not all eight blocks at once: 288 threads leave 168 registers a thread.)
+template <int NT>
+__device__ __forceinline__ void mma_mx_tiles(const Params& p, const Hdr& h, const uint8_t* tile,
+                                             const uint8_t* act, float (&acc)[NT][4], int warp,
+                                             int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+  const int nact = (h.ntok + 7) >> 3;
+  const uint4 sc = lds128(tile + kMxCodeBytes + (warp * 8 + g) * 16);
+  const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+  const bool full = h.nb == 8;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    if (!full && 4 * hf >= h.nb) break;
+    uint32_t A[4][2][4];
+    float sw[4][2];
+    const uint4 c0 = lds128(tile + (warp * 4 + 2 * hf) * 512 + lane * 16);
+    const uint4 c1 = lds128(tile + (warp * 4 + 2 * hf + 1) * 512 + lane * 16);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 w4 = (i >> 1) ? c1 : c0;
+      e2m1x8_to_f16x2x4((i & 1) ? w4.z : w4.x, A[i][0]);
+      e2m1x8_to_f16x2x4((i & 1) ? w4.w : w4.y, A[i][1]);
+      sw[i][0] = e8m0_byte_to_float(scw[hf], i);
+      sw[i][1] = e8m0_byte_to_float(scw[2 + hf], i);
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      if (t >= nact) break;
+      const int tok = 8 * t + g;
+      const int cc = 8 * t + 2 * tig;
+      const uint8_t* arow = act + (tok < h.ntok ? tok : 0) * p.act_stride + tig * 16 + hf * 256;
+      const float* s0 = reinterpret_cast<const float*>(act + (cc < h.ntok ? cc : 0) * p.act_stride + 512) + 4 * hf;
+      const float* s1 =
+          reinterpret_cast<const float*>(act + (cc + 1 < h.ntok ? cc + 1 : 0) * p.act_stride + 512) + 4 * hf;
+      uint4 bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bv[i] = lds128(arow + i * 64);
+      const float4 s0v = *reinterpret_cast<const float4*>(s0);
+      const float4 s1v = *reinterpret_cast<const float4*>(s1);
+      const float sa0[4] = {s0v.x, s0v.y, s0v.z, s0v.w};
+      const float sa1[4] = {s1v.x, s1v.y, s1v.z, s1v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (full || 4 * hf + i < h.nb) {
+          float tmp[4];
+          mma_f16_zc(tmp, A[i][0], bv[i].x, bv[i].y);
+          mma_f16(tmp, A[i][1], bv[i].z, bv[i].w);
+          acc[t][0] = fmaf(sw[i][0] * sa0[i], tmp[0], acc[t][0]);
+          acc[t][1] = fmaf(sw[i][0] * sa1[i], tmp[1], acc[t][1]);
+          acc[t][2] = fmaf(sw[i][1] * sa0[i], tmp[2], acc[t][2]);
+          acc[t][3] = fmaf(sw[i][1] * sa1[i], tmp[3], acc[t][3]);
+        }
+      }
+    }
+  }
+}
+
 template <int NT>
 __device__ __forceinline__ void mma_mx(const Params& p, const Hdr& h, const uint8_t* tile,
                                        const uint8_t* act, float (&acc)[NT][4], int warp, int lane) {
+  if constexpr (NT > 1) {
+    mma_mx_tiles<NT>(p, h, tile, act, acc, warp, lane);
+    return;
+  }
   const int g = lane >> 2, tig = lane & 3;
   const uint4 sc = lds128(tile + kMxCodeBytes + (warp * 8 + g) * 16);
   const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
@@ -724,7 +796,8 @@ __device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int wa
 }
 
 __device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
-                                          int* wtot, int tid, int warp, int lane);
+                                          float* lg_s, int lg_cap, int* wtot, int tid, int warp,
+                                          int lane);
 
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
@@ -831,8 +904,47 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
 // top-k routing and per-expert token lists (one CTA, 256 threads); the
 // per-token selection is warp_topk (topk.cuh).
 
+// Copy n floats that other CTAs wrote (read past L1) into shared memory, with
+// eight 16-byte loads (or sixteen 4-byte ones) in flight per thread.
+__device__ __forceinline__ void stage_floats(const float* src, int n, float* dst, int tid) {
+  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (n & 3) == 0) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    float4* d4 = reinterpret_cast<float4*>(dst);
+    const int n4 = n >> 2;
+    for (int i0 = tid; i0 < n4; i0 += kConsumerThreads * 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kConsumerThreads;
+        v[u] = i < n4 ? __ldcg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kConsumerThreads;
+        if (i < n4) d4[i] = v[u];
+      }
+    }
+  } else {
+    for (int i0 = tid; i0 < n; i0 += kConsumerThreads * 16) {
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + u * kConsumerThreads;
+        v[u] = i < n ? __ldcg(src + i) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + u * kConsumerThreads;
+        if (i < n) dst[i] = v[u];
+      }
+    }
+  }
+}
+
+// lg_s: shared memory for lg_cap floats of logits (at least E).
 __device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
-                                          int* wtot, int tid, int warp, int lane) {
+                                          float* lg_s, int lg_cap, int* wtot, int tid, int warp,
+                                          int lane) {
   const int E = p.E, K = p.topk, B = p.B;
   const int tg = p.tg > 0 ? p.tg : 1;
   int* cnt = reinterpret_cast<int*>(scratch);  // [E] slots per expert
@@ -847,20 +959,37 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
   named_sync(1, kConsumerThreads);
   if (tr) tr[16] = global_ns();
   // Few tokens: P warps share a token (each selects within a slice of the
-  // experts, one warp merges); 8 or more tokens: one warp per token.
+  // experts, one warp merges); 8 or more tokens: one warp per token, the
+  // logits of as many tokens as lg_s holds first copied there together (one
+  // round trip for all of them instead of one per token and warp).
   const int P = B >= kConsumerWarps ? 1 : kConsumerWarps / B;  // B * P <= 8 warps
   if (P == 1) {
-    for (int b = warp; b < B; b += kConsumerWarps) {
-      int sel_id;
-      float sel_w;
-      warp_topk(p.logits + (long long)b * E, E, K, p.score_fn, bias, p.renorm, p.routed_scale,
-                lane, sel_id, sel_w);
-      if (lane < K) {
-        p.ids[b * K + lane] = sel_id;
-        p.wts[b * K + lane] = sel_w;
-        ids_s[b * K + lane] = sel_id;
-        atomicAdd(&cnt[sel_id], 1);
+    const bool staged = lg_cap >= E;  // (the ring always holds a token's logits)
+    const int chunk = staged ? min(B, lg_cap / E) : B;
+    for (int b0 = 0; b0 < B; b0 += chunk) {
+      const int nb = min(chunk, B - b0);
+      if (staged) {
+        stage_floats(p.logits + (long long)b0 * E, nb * E, lg_s, tid);
+        named_sync(1, kConsumerThreads);
       }
+      for (int bl = warp; bl < nb; bl += kConsumerWarps) {
+        const int b = b0 + bl;
+        int sel_id;
+        float sel_w;
+        if (staged)
+          warp_topk<true>(lg_s + bl * E, E, K, p.score_fn, bias, p.renorm, p.routed_scale, lane,
+                          sel_id, sel_w);
+        else
+          warp_topk<false>(p.logits + (long long)b * E, E, K, p.score_fn, bias, p.renorm,
+                           p.routed_scale, lane, sel_id, sel_w);
+        if (lane < K) {
+          p.ids[b * K + lane] = sel_id;
+          p.wts[b * K + lane] = sel_w;
+          ids_s[b * K + lane] = sel_id;
+          atomicAdd(&cnt[sel_id], 1);
+        }
+      }
+      named_sync(1, kConsumerThreads);  // every warp is done with lg_s
     }
   } else {
     // candidates after the token table: [B][P][K] TopkCand, then [B][P] partials
@@ -988,7 +1117,11 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
   if (!sm_flag[0]) return;
   if (tr && tid == 0) tr[4] = global_ns();
-  route_tokens(p, bias, scratch, sm_flag + 16, tid, warp, lane);  // ends with a barrier
+  // the rest of the idle ring holds staged logits
+  const int bias_floats = (p.E + 31) & ~31;
+  const int ring_floats = p.nstages * p.stage_bytes / 4;
+  route_tokens(p, bias, scratch, bias_s + bias_floats, ring_floats - bias_floats, sm_flag + 16,
+               tid, warp, lane);  // ends with a barrier
   if (tid == 0) {
     if (tr) tr[5] = global_ns();
     *p.router_done = 0;
@@ -1017,80 +1150,81 @@ __device__ __forceinline__ void write_partial(const Params& p, int piece, int nt
     }
 }
 
-// Sum the row block's pieces in piece order (the same order whatever CTA ran
-// them, so the result is deterministic).
-template <int NT>
-__device__ __forceinline__ void sum_partials(const Params& p, const Hdr& h, float (&acc)[NT][4],
-                                             int warp, int lane) {
-  const int g = lane >> 2, tig = lane & 3;
-  const long long first = h.p0;
-  const long long stride = NT * 8 * kRowsPerBlock;
+// Sum of ppr pieces' partials for n4 groups of four consecutive floats:
+// thread tid owns groups tid + 256 j (j < JG) and keeps JG * PB 16-byte loads
+// in flight.  Pieces are added in piece order.
+template <int JG, int PB>
+__device__ __forceinline__ void sum_groups(const float* base, long long stride, int ppr, int n4,
+                                           float* rs, int tid) {
+  float4 s[JG];
 #pragma unroll
-  for (int t = 0; t < NT; ++t)
+  for (int j = 0; j < JG; ++j) s[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int pr = 0; pr < ppr; pr += PB) {
+    float4 v[JG][PB];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int col = 8 * t + 2 * tig + (q & 1);
-      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
-      float sum = 0.f;
-      if (col < h.ntok) {
-        const float* src = p.partials + first * stride + col * kRowsPerBlock + row;
-        int pr = 0;
-        for (; pr + 8 <= h.ppr; pr += 8) {
-          float v[8];
+    for (int j = 0; j < JG; ++j)
 #pragma unroll
-          for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (pr + u) * stride);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) sum += v[u];
-        }
-        for (; pr < h.ppr; ++pr) sum += __ldcg(src + pr * stride);
+      for (int u = 0; u < PB; ++u) {
+        const int i = tid + j * kConsumerThreads;
+        v[j][u] = (i < n4 && pr + u < ppr)
+                      ? __ldcg(reinterpret_cast<const float4*>(base + (pr + u) * stride) + i)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      acc[t][q] = sum;
-    }
+#pragma unroll
+    for (int j = 0; j < JG; ++j)
+#pragma unroll
+      for (int u = 0; u < PB; ++u) {
+        s[j].x += v[j][u].x;
+        s[j].y += v[j][u].y;
+        s[j].z += v[j][u].z;
+        s[j].w += v[j][u].w;
+      }
+  }
+#pragma unroll
+  for (int j = 0; j < JG; ++j) {
+    const int i = tid + j * kConsumerThreads;
+    if (i < n4) reinterpret_cast<float4*>(rs)[i] = s[j];
+  }
 }
 
-// Same sums for up to 32 token columns, spread over all consumer threads
-// (one (column, row) value each, 16 loads in flight) and handed back through
-// shared memory.
+// Sum the row block's pieces in piece order (the same order whatever CTA ran
+// them, so the result is deterministic).  All consumer threads share the
+// loads and hand the sums back through shared memory, 32 token columns
+// (16 KB of scratch) at a time: up to 8 columns one group of four rows a
+// thread with 16 pieces in flight, more columns four groups a thread with 4
+// pieces in flight.
 template <int NT>
-__device__ __forceinline__ void sum_partials_wide(const Params& p, const Hdr& h, float (&acc)[NT][4],
-                                                  float* rs, int tid, int warp, int lane) {
-  const long long first = h.p0;
+__device__ __forceinline__ void sum_partials(const Params& p, const Hdr& h, float (&acc)[NT][4],
+                                             float* rs, int tid, int warp, int lane) {
   const long long stride = NT * 8 * kRowsPerBlock;
-  const int n = h.ntok * kRowsPerBlock;
-  for (int i = tid; i < n; i += kConsumerThreads) {
-    const float* src = p.partials + first * stride + i;  // i = col * 128 + row
-    float sum = 0.f;
-    int pr = 0;
-    for (; pr + 16 <= h.ppr; pr += 16) {
-      float v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = __ldcg(src + (pr + u) * stride);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) sum += v[u];
-    }
-    for (; pr < h.ppr; ++pr) sum += __ldcg(src + pr * stride);
-    rs[i] = sum;
-  }
-  named_sync(1, kConsumerThreads);
+  const float* base = p.partials + (long long)h.p0 * stride;
   const int g = lane >> 2, tig = lane & 3;
+  for (int c0 = 0; c0 < h.ntok; c0 += 32) {
+    const int ncol = min(32, h.ntok - c0);
+    const int n4 = ncol * (kRowsPerBlock / 4);
+    if (ncol <= 8)
+      sum_groups<1, 16>(base + c0 * kRowsPerBlock, stride, h.ppr, n4, rs, tid);
+    else
+      sum_groups<4, 4>(base + c0 * kRowsPerBlock, stride, h.ppr, n4, rs, tid);
+    named_sync(1, kConsumerThreads);
 #pragma unroll
-  for (int t = 0; t < NT; ++t)
+    for (int t = 0; t < NT; ++t) {
+      if (8 * t < c0 || 8 * t >= c0 + 32) continue;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int col = 8 * t + 2 * tig + (q & 1);
-      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
-      acc[t][q] = col < h.ntok ? rs[col * kRowsPerBlock + row] : 0.f;
+      for (int q = 0; q < 4; ++q) {
+        const int col = 8 * t + 2 * tig + (q & 1);
+        const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+        acc[t][q] = col < h.ntok ? rs[(col - c0) * kRowsPerBlock + row] : 0.f;
+      }
     }
-  named_sync(1, kConsumerThreads);
+    named_sync(1, kConsumerThreads);
+  }
 }
 
 template <int KIND, int NT>
 __device__ __forceinline__ void finalize(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
                          int* sm_flag, const int* slot_tab, int tid, int warp, int lane) {
-  if (h.ntok <= 32)
-    sum_partials_wide<NT>(p, h, acc, reinterpret_cast<float*>(scratch), tid, warp, lane);
-  else
-    sum_partials<NT>(p, h, acc, warp, lane);
+  sum_partials<NT>(p, h, acc, reinterpret_cast<float*>(scratch), tid, warp, lane);
   if (tid == 0) p.counters[h.v * p.RB + h.rb] = 0;  // ready for the next launch
   epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
 }

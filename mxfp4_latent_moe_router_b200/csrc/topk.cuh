@@ -44,8 +44,10 @@ constexpr uint32_t kNoExpert = 0xffffffffu;
 // Top-K of experts [e0, e1) of one token (K <= 16, e1 - e0 <= 32 * EPL).
 // On return lane r < K holds the r-th best candidate (key-descending), and
 // every lane holds the slice's logit maximum and sum of exp(logit - max)
-// (softmax scoring only; they normalise the probabilities).
-template <int EPL>
+// (softmax scoring only; they normalise the probabilities).  The logits are
+// in global memory, read past L1 (other CTAs wrote them), or with kSmem in
+// this CTA's shared memory.
+template <int EPL, bool kSmem = false>
 __device__ __forceinline__ void warp_topk_slice(const float* logits, const float* bias, int e0, int e1,
                                              int K, int score_fn, int lane, TopkCand& out,
                                              float& smax, float& ssum) {
@@ -56,7 +58,7 @@ __device__ __forceinline__ void warp_topk_slice(const float* logits, const float
   for (int j = 0; j < EPL; ++j) {
     const int e = e0 + lane + 32 * j;
     const bool in = e < e1;
-    lg[j] = in ? __ldcg(logits + e) : 0.f;
+    lg[j] = in ? (kSmem ? logits[e] : __ldcg(logits + e)) : 0.f;
     bs[j] = (in && bias) ? bias[e] : 0.f;  // (global or shared memory)
   }
   float mx = -INFINITY;
@@ -124,22 +126,23 @@ __device__ __forceinline__ void warp_topk_slice(const float* logits, const float
 }
 
 // Pick an EPL bound for a slice of n experts.
+template <bool kSmem = false>
 __device__ __forceinline__ void warp_topk_slice_any(const float* logits, const float* bias, int e0,
                                                     int e1, int K, int score_fn, int lane,
                                                     TopkCand& out, float& smax, float& ssum) {
   const int n = e1 - e0;
   if (n <= 32)
-    warp_topk_slice<1>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
+    warp_topk_slice<1, kSmem>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
   else if (n <= 64)
-    warp_topk_slice<2>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
+    warp_topk_slice<2, kSmem>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
   else if (n <= 128)
-    warp_topk_slice<4>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
+    warp_topk_slice<4, kSmem>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
   else if (n <= 256)
-    warp_topk_slice<8>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
+    warp_topk_slice<8, kSmem>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
   else if (n <= 384)
-    warp_topk_slice<12>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
+    warp_topk_slice<12, kSmem>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);
   else
-    warp_topk_slice<16>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);  // n <= 512
+    warp_topk_slice<16, kSmem>(logits, bias, e0, e1, K, score_fn, lane, out, smax, ssum);  // n <= 512
 }
 
 // K rounds over two candidates per lane (candidate slots lane and lane + 32):
@@ -211,17 +214,18 @@ __device__ __forceinline__ void warp_topk_merge(const TopkCand* cand, const floa
 
 // Whole selection for one token on one warp: one slice of up to 512 experts,
 // or two slices whose candidates are merged in registers (E <= 1024).
+template <bool kSmem = false>
 __device__ __forceinline__ void warp_topk(const float* logits, int E, int K, int score_fn,
                                           const float* bias, int renorm, float routed_scale,
                                           int lane, int& sel_id, float& sel_w) {
   const int split = E > 512 ? (E + 1) / 2 : E;
   TopkCand c0, c1;
   float m0, s0, m1 = -INFINITY, s1 = 0.f;
-  warp_topk_slice_any(logits, bias, 0, split, K, score_fn, lane, c0, m0, s0);
+  warp_topk_slice_any<kSmem>(logits, bias, 0, split, K, score_fn, lane, c0, m0, s0);
   c1.key = -INFINITY;
   c1.id = 0x7fffffff;
   c1.logit = 0.f;
-  if (split < E) warp_topk_slice_any(logits, bias, split, E, K, score_fn, lane, c1, m1, s1);
+  if (split < E) warp_topk_slice_any<kSmem>(logits, bias, split, E, K, score_fn, lane, c1, m1, s1);
   const float mx = fmaxf(m0, m1);
   float den = 1.f;
   if (score_fn == 0) den = s0 * __expf(m0 - mx) + (split < E ? s1 * __expf(m1 - mx) : 0.f);
