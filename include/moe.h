@@ -210,7 +210,9 @@ MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
  *   14 the SM the CTA ran on, 15..18 fused slot: ns of the consumers' first
  *   stage of each phase (the routing CTA: top-k phase stamps in 16..18),
  *   19 ns the router logits of a row block were published, 21..22 routing
- *   CTA: slice selection end, merge end.
+ *   CTA: slice selection end, merge end (8 or more tokens: logits staged,
+ *   first token selected; 20: the first warp's tokens of the first staged
+ *   group selected).
  * Synchronises the device.
  */
 MOE_API moe_status moe_debug_trace(moe_plan p, uint64_t *host, int64_t count);

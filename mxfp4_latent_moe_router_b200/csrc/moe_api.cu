@@ -32,8 +32,17 @@ constexpr int kFused = KIND_COUNT;
 // largest batch the fused single launch takes (one 8-column token tile)
 constexpr int kFusedMaxTokens = 8;
 constexpr int kTailTg = 16;
-constexpr int kExpertTg = 32;
+// Tokens per virtual expert (an expert's slots are cut into groups of at most
+// this many).  Up to 64 tokens an expert rarely holds more than 8 of them:
+// groups of 8 keep the expert kernels at one token tile, where two CTAs share
+// an SM.  Beyond that (skewed batches of 128) groups of 32, so a popular
+// expert's weights are streamed once per 32 tokens rather than per 8.
+constexpr int kExpertTgSmall = 8, kExpertTgLarge = 32, kExpertSmallMaxB = 64;
+int expert_tg(int B) { return B <= kExpertSmallMaxB ? kExpertTgSmall : kExpertTgLarge; }
 constexpr int kBigSmem = 227 * 1024;
+// two CTAs of the one-tile expert kernels share an SM (228 KB, 1 KB reserved
+// per CTA): twice the warps to hide the MXFP4 loop's latencies
+constexpr int kHalfSmem = 113 * 1024;
 
 struct KindGeom {
   int RB = 0, C = 0, KL = 0;
@@ -93,6 +102,7 @@ struct moe_plan_s {
   // split-K piece end in the split choice, whether kernels chain with
   // programmatic dependent launch, and whether small batches run fused
   int split_cost = 2;
+  int expert_per_sm_max = 2;  // environment MOE_EXPERT_CTAS_PER_SM
   bool use_pdl = true;
   // one launch per forward for B <= kFusedMaxTokens (environment MOE_FUSED=1);
   // off by default: measured slower than the four-launch chain at B = 1
@@ -146,27 +156,6 @@ moe_status alloc(moe_plan p, void** out, size_t bytes, bool packed) {
 
 bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
 
-// token geometry of one forward
-struct FwdGeom {
-  int nt_front, nt_e, nt_tail, tail_tg;
-  int front_grid, front_workers, tail_grid, expert_grid;
-};
-
-FwdGeom fwd_geom(const moe_plan_s* p, int B) {
-  FwdGeom f;
-  f.nt_front = pow2_at_least((B + 7) / 8);
-  f.nt_e = pow2_at_least((std::min(B, kExpertTg) + 7) / 8);
-  f.tail_tg = p->tail_tg;
-  f.nt_tail = pow2_at_least((std::min(B, p->tail_tg) + 7) / 8);
-  // every kernel takes every SM (one CTA each); the front kernel's last CTA
-  // is the routing CTA and streams nothing
-  f.front_grid = p->num_sms;
-  f.front_workers = p->num_sms - 1;
-  f.tail_grid = p->num_sms;
-  f.expert_grid = p->num_sms;
-  return f;
-}
-
 int g_max_stages = 5;  // ring depth cap (environment MOE_MAX_STAGES)
 
 struct SmemGeom {
@@ -179,7 +168,7 @@ constexpr int kResidentMax = 72 * 1024;
 int resident_stride(int res_k) { return res_k * 4 + 64; }
 
 SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int slots,
-                   int res_bytes = 0) {
+                   int res_bytes = 0, int budget = kBigSmem) {
   SmemGeom s;
   // routing tables (virtual experts + expert-sorted slots) for the expert kernels
   s.table_bytes = 0;
@@ -201,18 +190,47 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int 
   const int tile = (kind == KIND_EGU || kind == KIND_EDN) ? kMxTileBytes : kDenseTileBytes;
   s.act_off = kHdr + tile;
   s.stage_bytes = ((kHdr + tile + act) + 127) / 128 * 128;
-  // one CTA per SM: a running kernel and the next one, launched early by
-  // programmatic dependent launch, never share an SM, and the whole shared
-  // memory goes to the ring
-  const int budget = kBigSmem;
+  // one CTA per SM (the whole shared memory for the ring): a running kernel
+  // and the next one, launched early by programmatic dependent launch, never
+  // share an SM; with the half budget, two CTAs of one expert kernel do
   // enough bytes in flight to saturate HBM (about 6 x 16 KB per SM); more only
   // lengthens the queues every other memory request waits behind
   s.nstages = std::max(2, std::min(g_max_stages, (budget - stage_off) / s.stage_bytes));
   s.stage_off = stage_off;
   s.total = (size_t)stage_off + (size_t)s.nstages * s.stage_bytes;
   // more than half of the SM's shared memory: never two CTAs on one SM
-  s.total = std::max(s.total, (size_t)(116 * 1024));
+  // (unless the budget is the half that two CTAs share)
+  if (budget > kHalfSmem) s.total = std::max(s.total, (size_t)(116 * 1024));
   return s;
+}
+
+// token geometry of one forward
+struct FwdGeom {
+  int nt_front, nt_e, nt_tail, tail_tg;
+  int front_grid, front_workers, tail_grid, expert_grid;
+  int expert_per_sm;  // CTAs of each expert kernel per SM (1 or 2)
+};
+
+FwdGeom fwd_geom(const moe_plan_s* p, int B) {
+  FwdGeom f;
+  f.nt_front = pow2_at_least((B + 7) / 8);
+  f.nt_e = pow2_at_least((std::min(B, expert_tg(B)) + 7) / 8);
+  f.tail_tg = p->tail_tg;
+  f.nt_tail = pow2_at_least((std::min(B, p->tail_tg) + 7) / 8);
+  // every kernel takes every SM (one CTA each; the one-tile expert kernels
+  // two, when half the shared memory still holds a ring of 3 stages); the
+  // front kernel's last CTA is the routing CTA and streams nothing
+  f.front_grid = p->num_sms;
+  f.front_workers = p->num_sms - 1;
+  f.tail_grid = p->num_sms;
+  f.expert_per_sm = 1;
+  if (f.nt_e == 1 && p->expert_per_sm_max >= 2) {
+    const int slots = B * p->cfg.top_k;
+    const SmemGeom h = smem_geom(KIND_EGU, 1, 1, p->cfg.top_k, p->ve_max, slots, 0, kHalfSmem);
+    if (h.nstages >= 3 && h.total <= (size_t)kHalfSmem) f.expert_per_sm = 2;
+  }
+  f.expert_grid = p->num_sms * f.expert_per_sm;
+  return f;
 }
 
 int g_split_cost = 2;  // split-K piece-end price in stages (environment MOE_SPLIT_COST)
@@ -258,7 +276,7 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   q.C = p->g[kind].C;
   q.KL = p->g[kind].KL;
   q.ctl = p->ctl + kind;
-  q.trace = p->trace ? p->trace + (size_t)kind * p->num_sms * 24 : nullptr;
+  q.trace = p->trace ? p->trace + (size_t)kind * 2 * p->num_sms * 24 : nullptr;
   q.counters = p->counters[kind];
   q.partials = p->partials[kind];
   q.nstages = s.nstages;
@@ -271,20 +289,21 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   switch (kind) {
     case KIND_FRONT:  // its routing CTA groups expert tokens by tg
       q.wt = p->w_front;
-      q.tg = kExpertTg;
+      q.tg = expert_tg(q.B);
       q.RB_router = p->RB_router;
       q.RB_lat = p->RB_lat;
       q.route_cta = 1;
       break;
-    case KIND_EGU: q.wt = p->w_egu; q.tg = kExpertTg; break;
-    case KIND_EDN: q.wt = p->w_edn; q.tg = kExpertTg; break;
+    case KIND_EGU: q.wt = p->w_egu; q.tg = expert_tg(q.B); break;
+    case KIND_EDN: q.wt = p->w_edn; q.tg = expert_tg(q.B); break;
     default: q.wt = p->w_tail; q.tg = p->tail_tg; break;
   }
 }
 
 // Price of a split-K piece end in stages: partial sums out and the
-// finalising sums back in both grow with the piece's token tiles.
-int split_cost_for(int nt) { return g_split_cost * std::max(1, nt); }
+// finalising sums back in grow with the piece's token tiles, but more slowly
+// than a stage's own work does (a stage of 16 tiles costs about 2x one of 1).
+int split_cost_for(int nt) { return g_split_cost * (1 + std::max(1, nt) / 4); }
 
 // split-K factor of a kind whose row-block count the host knows
 int ppr_for(int mats, int C, int ctas, int nt) { return best_ppr(mats, C, ctas, split_cost_for(nt)); }
@@ -361,6 +380,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   if (prop.major != 10) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
   p->num_sms = prop.multiProcessorCount;
   if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
   if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
   if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
   if (const char* e = getenv("MOE_MAX_STAGES")) g_max_stages = std::max(2, std::min(8, atoi(e)));
@@ -401,7 +421,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
 
   const int maxB = c.max_tokens, K = c.top_k;
   const int slots = maxB * K;
-  p->ve_max = std::min(E, slots) + ceil_div(slots, kExpertTg) + 1;
+  p->ve_max = std::min(E, slots) + ceil_div(slots, kExpertTgSmall) + 1;  // any group size
 
   void* v;
   TRY(alloc(p, &v, fr.weight_bytes, true));
@@ -452,9 +472,10 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
     p->partials[k] = (float*)v;
   }
   if (getenv("MOE_TRACE")) {
-    TRY(alloc(p, &v, sizeof(unsigned long long) * kSlots * p->num_sms * 24, false));
+    // rows for up to two CTAs per SM in every slot
+    TRY(alloc(p, &v, sizeof(unsigned long long) * kSlots * 2 * p->num_sms * 24, false));
     p->trace = (unsigned long long*)v;
-    CUDA_TRY(cudaMemset(v, 0, sizeof(unsigned long long) * kSlots * p->num_sms * 24));
+    CUDA_TRY(cudaMemset(v, 0, sizeof(unsigned long long) * kSlots * 2 * p->num_sms * 24));
   }
   TRY(alloc(p, &v, sizeof(uint16_t) * (size_t)maxB * H, false));
   p->x_stage = (uint16_t*)v;
@@ -514,7 +535,7 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
     q.stage_off = stage_off;
     q.table_off = kStageOff;
     q.ctl = p->ctl + kFused;
-    q.trace = p->trace ? p->trace + (size_t)kFused * p->num_sms * 24 : nullptr;
+    q.trace = p->trace ? p->trace + (size_t)kFused * 2 * p->num_sms * 24 : nullptr;
     q.done = p->done;
     q.need_rb_edn = p->g[KIND_EDN].RB;
     q.need_rb_sh = p->g[KIND_FRONT].RB - p->RB_router - p->RB_lat;
@@ -574,7 +595,8 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
+    const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, 0,
+                                  f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
     set_kind(q, p, KIND_EGU, sm);
     q.piece_ctas = f.expert_grid;
     q.split_cost = split_cost_for(f.nt_e);
@@ -584,7 +606,8 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
+    const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, 0,
+                                  f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
     set_kind(q, p, KIND_EDN, sm);
     q.piece_ctas = f.expert_grid;
     q.split_cost = split_cost_for(f.nt_e);
@@ -894,7 +917,12 @@ moe_status moe_debug_trace(moe_plan p, uint64_t* host, int64_t count) {
   if (count != n) return MOE_ERR_INVALID_ARG;
   DeviceGuard g(p->device);
   CUDA_TRY(cudaDeviceSynchronize());
-  CUDA_TRY(cudaMemcpy(host, p->trace, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost));
+  // the first num_sms CTAs of each slot (a grid of two CTAs per SM traces
+  // its second half into rows that are not returned)
+  const size_t row = (size_t)p->num_sms * 24;
+  for (int k = 0; k < kSlots; ++k)
+    CUDA_TRY(cudaMemcpy(host + k * row, p->trace + (size_t)k * 2 * row, sizeof(uint64_t) * row,
+                        cudaMemcpyDeviceToHost));
   return MOE_OK;
 }
 

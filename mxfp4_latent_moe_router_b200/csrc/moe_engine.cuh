@@ -198,10 +198,93 @@ __device__ __forceinline__ const uint8_t* weight_src(const Params& p, const Hdr&
   return p.wt + tile * kDenseTileBytes;
 }
 
+// A stage's activation rows are one bulk copy each, but the copy engine takes
+// bulk copies one at a time: past 8 rows (64 rows of 128 bytes at B = 64)
+// issuing them outlasts the stage's own weight tile.  Such stages copy their
+// rows in 16-byte pieces from all producer lanes instead; their full barrier
+// then expects only the weight tile's bytes and completes once the lanes'
+// copies have landed and lane 0 has arrived.
+constexpr int kBulkRowsMax = 8;
+template <int KIND>
+__device__ __forceinline__ bool rows_async(const Hdr& h) {
+  return (KIND == KIND_FRONT || KIND == KIND_EGU || KIND == KIND_EDN) && h.ntok > kBulkRowsMax;
+}
+
+// Lane 0: a stage's header, its barrier expectation and its weight tile.
+template <int KIND>
+__device__ __forceinline__ void stage_begin(const Params& p, const Hdr& h, uint8_t* sb, uint64_t* bar) {
+  constexpr int kTile = KindTraits<KIND>::kTileBytes;
+  *reinterpret_cast<Hdr*>(sb) = h;
+  // a slot whose activations once came in 16-byte copies may now take a bulk
+  // copy: order the two proxies' writes
+  if ((KIND == KIND_FRONT || KIND == KIND_EGU || KIND == KIND_EDN) && p.B > kBulkRowsMax)
+    fence_proxy_async_smem();
+  if (rows_async<KIND>(h))
+    mbar_expect_tx(bar, kTile);  // lane 0 arrives once the rows are issued
+  else
+    mbar_arrive_expect_tx(bar, kTile + h.act_bytes);
+  bulk_g2s(sb + kHdrBytes, weight_src<KIND>(p, h), kTile, bar);
+}
+
+// The lanes' 16-byte copies are done; let the barrier track them and arrive.
+__device__ __forceinline__ void rows_async_done(uint64_t* bar, int lane) {
+  cp_async_mbar_arrive(bar);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
+// Front: token rows of x, 2^lg_per 16-byte pieces each, rows ld bytes apart.
+__device__ __forceinline__ void copy_x_rows_async(uint8_t* act, int stride, int nrows, int lg_per,
+                                                  const uint8_t* src, long long ld, uint64_t* bar,
+                                                  int lane) {
+  for (int i = lane; i < (nrows << lg_per); i += 32) {
+    const int r = i >> lg_per, q = i & ((1 << lg_per) - 1);
+    cp_async16(act + r * stride + q * 16, src + r * ld + q * 16);
+  }
+  rows_async_done(bar, lane);
+}
+
+// Expert kernels: nrows activation records (kActRecBytes each).  Gathered
+// rows (nrows <= 32) come from lane r's row pointer; otherwise the records
+// are consecutive from src.
+__device__ __forceinline__ void copy_records_async(uint8_t* act, int stride, int nrows,
+                                                   const uint8_t* src, bool gathered,
+                                                   uint64_t* bar, int lane) {
+  constexpr int kPer = kActRecBytes / 16;
+  const int n = nrows * kPer;
+  for (int i0 = 0; i0 < n; i0 += 32) {  // the whole warp in every round (shuffles)
+    const int i = i0 + lane;
+    const int r = min(i / kPer, nrows - 1), q = i - r * kPer;
+    const uint8_t* row =
+        gathered ? reinterpret_cast<const uint8_t*>(
+                       __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(src), r))
+                 : src + (long long)r * kActRecBytes;
+    if (i < n) cp_async16(act + r * stride + q * 16, row + q * 16);
+  }
+  rows_async_done(bar, lane);
+}
+
 // Issue this stage's activation copies (all 32 producer lanes).
 template <int KIND>
 __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t* act, uint64_t* bar,
                                           int lane, const int* slot_tab) {
+  if (rows_async<KIND>(h)) {
+    if (KIND == KIND_FRONT) {
+      const uint8_t* x = reinterpret_cast<const uint8_t*>(p.x + h.chunk * kDenseChunkK);
+      copy_x_rows_async(act, p.act_stride, h.ntok, h.nb == 2 ? 3 : 2, x, (long long)p.H * 2, bar, lane);
+    } else if (KIND == KIND_EGU) {
+      // lane r: token row of slot r (a virtual expert holds at most 32 slots)
+      const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
+      const uint8_t* mine = p.z_mx + (long long)h.chunk * kActRecBytes;
+      if (lane < h.ntok) mine += (long long)(slot_tab[h.tok0 + lane] / p.topk) * cz * kActRecBytes;
+      copy_records_async(act, p.act_stride, h.ntok, mine, true, bar, lane);
+    } else {
+      copy_records_async(act, p.act_stride, h.ntok,
+                         p.h_mx + ((long long)h.chunk * p.ld_slots + h.tok0) * kActRecBytes, false,
+                         bar, lane);
+    }
+    return;
+  }
   if (KIND == KIND_FRONT) {
     const int bytes = h.nb * 64;
     for (int r = lane; r < h.ntok; r += 32)
@@ -332,11 +415,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
       Hdr h = ph;
       chunk_header<KIND>(p, c, c_first, c_last, h);
-      if (lane == 0) {
-        *reinterpret_cast<Hdr*>(sb) = h;
-        mbar_arrive_expect_tx(&full[stage], KindTraits<KIND>::kTileBytes + h.act_bytes);
-        bulk_g2s(sb + kHdrBytes, weight_src<KIND>(p, h), KindTraits<KIND>::kTileBytes, &full[stage]);
-      }
+      if (lane == 0) stage_begin<KIND>(p, h, sb, &full[stage]);
       __syncwarp();
       if (waited)
         issue_act<KIND>(p, h, sb + p.act_off, &full[stage], lane, slot_tab);
@@ -972,6 +1051,7 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
         stage_floats(p.logits + (long long)b0 * E, nb * E, lg_s, tid);
         named_sync(1, kConsumerThreads);
       }
+      if (tr && b0 == 0) tr[21] = global_ns();
       for (int bl = warp; bl < nb; bl += kConsumerWarps) {
         const int b = b0 + bl;
         int sel_id;
@@ -988,7 +1068,9 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
           ids_s[b * K + lane] = sel_id;
           atomicAdd(&cnt[sel_id], 1);
         }
+        if (tr && b0 == 0 && bl == 0) tr[22] = global_ns();
       }
+      if (tr && b0 == 0) tr[20] = global_ns();
       named_sync(1, kConsumerThreads);  // every warp is done with lg_s
     }
   } else {
@@ -1377,7 +1459,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
 // ---------------------------------------------------------------------------
 
 template <int KIND, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, (KIND == KIND_EGU || KIND == KIND_EDN) && NT == 1 ? 2 : 1)
     moe_kernel(const __grid_constant__ Params p) {
   // shared memory: [0,128) full barriers, [128,256) empty barriers,
   // [256,512) flags, [scratch_off, ...) scratch, [table_off, ...) routing

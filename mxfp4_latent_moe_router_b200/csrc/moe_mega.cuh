@@ -159,11 +159,7 @@ __device__ __forceinline__ int mega_issue_piece(const MegaParams& mp, MegaProd& 
       next = mega_next(st, ctl, workers, lane);
       h.next_kind = mega_kind_of(mp, st, next);
     }
-    if (lane == 0) {
-      *reinterpret_cast<Hdr*>(sb) = h;
-      mbar_arrive_expect_tx(&full[st.stage], KindTraits<KIND>::kTileBytes + h.act_bytes);
-      bulk_g2s(sb + kHdrBytes, weight_src<KIND>(p, h), KindTraits<KIND>::kTileBytes, &full[st.stage]);
-    }
+    if (lane == 0) stage_begin<KIND>(p, h, sb, &full[st.stage]);
     __syncwarp();
     if (st.dep_ok[KIND])
       issue_act<KIND>(p, h, sb + p.act_off, &full[st.stage], lane, slot_tab);
