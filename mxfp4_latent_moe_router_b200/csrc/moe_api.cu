@@ -33,12 +33,16 @@ constexpr int kFused = KIND_COUNT;
 constexpr int kFusedMaxTokens = 8;
 constexpr int kTailTg = 16;
 // Tokens per virtual expert (an expert's slots are cut into groups of at most
-// this many).  Up to 64 tokens an expert rarely holds more than 8 of them:
-// groups of 8 keep the expert kernels at one token tile, where two CTAs share
-// an SM.  Beyond that (skewed batches of 128) groups of 32, so a popular
-// expert's weights are streamed once per 32 tokens rather than per 8.
-constexpr int kExpertTgSmall = 8, kExpertTgLarge = 32, kExpertSmallMaxB = 64;
-int expert_tg(int B) { return B <= kExpertSmallMaxB ? kExpertTgSmall : kExpertTgLarge; }
+// this many).  Groups of 8 keep the expert kernels at one token tile, where
+// two CTAs share an SM.  That wins even for 128 Zipf-skewed tokens (675 vs
+// 772 us per step), although a popular expert's weights are then read once
+// per 8 tokens: its groups are adjacent in the piece order and tend to run
+// at about the same time, so most re-reads can hit L2.  Groups of 32 (four
+// tiles, one CTA per SM) remain for batches above the environment variable
+// MOE_EXPERT_SMALL_MAX_B.
+constexpr int kExpertTgSmall = 8, kExpertTgLarge = 32;
+int g_expert_small_max_b = 128;
+int expert_tg(int B) { return B <= g_expert_small_max_b ? kExpertTgSmall : kExpertTgLarge; }
 constexpr int kBigSmem = 227 * 1024;
 // two CTAs of the one-tile expert kernels share an SM (228 KB, 1 KB reserved
 // per CTA): twice the warps to hide the MXFP4 loop's latencies
@@ -381,6 +385,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->num_sms = prop.multiProcessorCount;
   if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
+  if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) g_expert_small_max_b = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
   if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
   if (const char* e = getenv("MOE_MAX_STAGES")) g_max_stages = std::max(2, std::min(8, atoi(e)));
