@@ -131,6 +131,21 @@ typedef struct moe_plan_info {
  * and workspace.  *out receives the plan.
  * Errors: INVALID_ARG (null, bad shape), UNSUPPORTED (no sm_100 device, shape
  * beyond the limits above), OOM, CUDA.
+ *
+ * Environment variables read here (measurement and tuning; every default is
+ * the measured best, and none changes a result beyond rounding order):
+ *   MOE_TRACE               keep the per-CTA timeline (moe_debug_trace)
+ *   MOE_LOG                 print the plan's geometry to stderr
+ *   MOE_FUSED=1             one launch per forward for B <= 8 (slower)
+ *   MOE_NO_PDL=1            no programmatic dependent launch between kernels
+ *   MOE_MAX_STAGES=n        ring depth cap, 2..8 (default 5)
+ *   MOE_SPLIT_COST=n        split-K piece-end price in stages (default 2)
+ *   MOE_EXPERT_CTAS_PER_SM=1  one CTA per SM for the expert kernels (default
+ *                           2 at one token tile)
+ *   MOE_EXPERT_SMALL_MAX_B=n  largest B with 8-token virtual experts (default
+ *                           128; above it, 32-token groups)
+ *   MOE_FAIL_ALLOC_AFTER=n  fail the (n+1)-th allocation with MOE_ERR_OOM
+ *                           (tests of the error path)
  */
 MOE_API moe_status moe_plan_create(const moe_config *cfg, int device, moe_plan *out);
 
