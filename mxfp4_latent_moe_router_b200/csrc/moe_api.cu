@@ -41,8 +41,6 @@ constexpr int kTailTg = 16;
 // tiles, one CTA per SM) remain for batches above the environment variable
 // MOE_EXPERT_SMALL_MAX_B.
 constexpr int kExpertTgSmall = 8, kExpertTgLarge = 32;
-int g_expert_small_max_b = 128;
-int expert_tg(int B) { return B <= g_expert_small_max_b ? kExpertTgSmall : kExpertTgLarge; }
 constexpr int kBigSmem = 227 * 1024;
 // two CTAs of the one-tile expert kernels share an SM (228 KB, 1 KB reserved
 // per CTA): twice the warps to hide the MXFP4 loop's latencies
@@ -106,7 +104,8 @@ struct moe_plan_s {
   // split-K piece end in the split choice, whether kernels chain with
   // programmatic dependent launch, and whether small batches run fused
   int split_cost = 2;
-  int expert_per_sm_max = 2;  // environment MOE_EXPERT_CTAS_PER_SM
+  int expert_per_sm_max = 2;     // environment MOE_EXPERT_CTAS_PER_SM
+  int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
   bool use_pdl = true;
   // one launch per forward for B <= kFusedMaxTokens (environment MOE_FUSED=1);
   // off by default: measured slower than the four-launch chain at B = 1
@@ -119,6 +118,11 @@ struct moe_plan_s {
   double prof_ms[kSlots] = {};
   int prof_count = 0;
 };
+
+// tokens per virtual expert for a forward of B tokens
+int expert_tg(const moe_plan_s* p, int B) {
+  return B <= p->expert_small_max_b ? kExpertTgSmall : kExpertTgLarge;
+}
 
 namespace {
 
@@ -218,7 +222,7 @@ struct FwdGeom {
 FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   FwdGeom f;
   f.nt_front = pow2_at_least((B + 7) / 8);
-  f.nt_e = pow2_at_least((std::min(B, expert_tg(B)) + 7) / 8);
+  f.nt_e = pow2_at_least((std::min(B, expert_tg(p, B)) + 7) / 8);
   f.tail_tg = p->tail_tg;
   f.nt_tail = pow2_at_least((std::min(B, p->tail_tg) + 7) / 8);
   // every kernel takes every SM (one CTA each; the one-tile expert kernels
@@ -293,13 +297,13 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   switch (kind) {
     case KIND_FRONT:  // its routing CTA groups expert tokens by tg
       q.wt = p->w_front;
-      q.tg = expert_tg(q.B);
+      q.tg = expert_tg(p, q.B);
       q.RB_router = p->RB_router;
       q.RB_lat = p->RB_lat;
       q.route_cta = 1;
       break;
-    case KIND_EGU: q.wt = p->w_egu; q.tg = expert_tg(q.B); break;
-    case KIND_EDN: q.wt = p->w_edn; q.tg = expert_tg(q.B); break;
+    case KIND_EGU: q.wt = p->w_egu; q.tg = expert_tg(p, q.B); break;
+    case KIND_EDN: q.wt = p->w_edn; q.tg = expert_tg(p, q.B); break;
     default: q.wt = p->w_tail; q.tg = p->tail_tg; break;
   }
 }
@@ -385,7 +389,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->num_sms = prop.multiProcessorCount;
   if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
-  if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) g_expert_small_max_b = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
   if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
   if (const char* e = getenv("MOE_MAX_STAGES")) g_max_stages = std::max(2, std::min(8, atoi(e)));

@@ -1,7 +1,7 @@
 """Edge cases of the CUDA path against the CPU oracle: the largest expert count
 and top-k the library takes, the largest batch, sigmoid scoring without a
-selection bias, and the fused single launch with a tail activation too large
-to keep in shared memory."""
+selection bias, the fused single launch with a tail activation too large to
+keep in shared memory, and 32-token virtual experts."""
 import numpy as np
 import pytest
 
@@ -77,3 +77,16 @@ def test_fused_launch_with_staged_tail(monkeypatch):
     w = synth.make_weights(shape)
     monkeypatch.setenv("MOE_FUSED", "1")
     _check(shape, w, synth.make_x(shape), max_tokens=8)
+
+
+@pytest.mark.parametrize("B,E,k", [(24, 8, 4), (48, 4, 3)])
+def test_thirty_two_token_expert_groups(B, E, k, monkeypatch):
+    # with 8-token groups switched off, an expert's slots form groups of up to
+    # 32 tokens: ~12 per expert in one group, or 36 per expert in groups of
+    # 32 and 4.  The expert kernels run four token tiles at one CTA per SM
+    # and gather more than 8 activation rows per stage with 16-byte copies.
+    monkeypatch.setenv("MOE_EXPERT_SMALL_MAX_B", "0")
+    shape = synth.custom_shape("tg32", B, 256, 256, E, k, 256, 64, synth.SCORE_SOFTMAX,
+                               seed=101 + B, scale_exp_lo=-5, scale_exp_hi=-2)
+    w = synth.make_weights(shape)
+    _check(shape, w, synth.make_x(shape), max_tokens=B)
