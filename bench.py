@@ -12,13 +12,14 @@ Timed region: a CUDA graph of exactly K layer steps, each step one
 rotation (4 x 206 MB touched per rotation at B=1, far above the 126 MB L2, so
 no step reuses weights from L2).  Barrier + synchronize on both sides, CUDA
 events on the launching stream, max over ranks.  N>1 runs independent replicas
-(the layer does not shard).
+(the layer runs whole on each GPU, with no collective).
 
 Also measured: per-kernel durations (CUDA events around each kernel on its
 own stream, a separate eager pass) for the dominant kernel's roofline; the same
 metric end to end through ``moe_forward_host`` with pinned host buffers
 (copies inside the timed region); the CPU oracle on the host cores on a
-bounded sample; SM clocks during the timed region.
+bounded sample; SM clocks during the timed region; the spread of the timed
+graph over five more replays (``step_spread``).
 """
 from __future__ import annotations
 
@@ -332,6 +333,23 @@ def run_ours(args):
     torch.cuda.synchronize()
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     us_step = ms_total * 1e3 / args.steps
+
+    # spread: the same graph replayed five more times after the timed region
+    # (this rank's own device time; the reported value is the timed replay)
+    try:
+        reps = [e0.elapsed_time(e1) * 1e3 / args.steps]
+        for _ in range(5):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                a0.record(stream)
+                g.replay()
+                a1.record(stream)
+            stream.synchronize()
+            reps.append(a0.elapsed_time(a1) * 1e3 / args.steps)
+        spread = {"replays": len(reps), "median_us": float(np.median(reps)),
+                  "p10_us": float(np.percentile(reps, 10)), "p90_us": float(np.percentile(reps, 90))}
+    except Exception as exc:  # the spread is context only; never lose the line for it
+        spread = {"error": type(exc).__name__}
     del g
 
     # routing of each input on instance 0..3 -> distinct touched experts per step
@@ -438,6 +456,7 @@ def run_ours(args):
             "clocks": clk,
             "plan": {"front_ctas": info.front_ctas, "expert_ctas": info.expert_ctas},
             "parity_spot_check": spot,
+            "step_spread": spread,
         }
         print(json.dumps(line), flush=True)
     for p in plans:
