@@ -103,7 +103,8 @@ struct moe_plan_s {
   // tuning knobs read once at plan creation (environment): the price of a
   // split-K piece end in the split choice, whether kernels chain with
   // programmatic dependent launch, and whether small batches run fused
-  int split_cost = 2;
+  int split_cost = 2;  // split-K piece-end price in stages (environment MOE_SPLIT_COST)
+  int max_stages = 5;  // ring depth cap (environment MOE_MAX_STAGES)
   int expert_per_sm_max = 2;     // environment MOE_EXPERT_CTAS_PER_SM
   int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
   bool use_pdl = true;
@@ -164,7 +165,6 @@ moe_status alloc(moe_plan p, void** out, size_t bytes, bool packed) {
 
 bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
 
-int g_max_stages = 5;  // ring depth cap (environment MOE_MAX_STAGES)
 
 struct SmemGeom {
   int stage_bytes, nstages, act_off, act_stride, table_bytes, stage_off, res_bytes;
@@ -175,8 +175,9 @@ struct SmemGeom {
 constexpr int kResidentMax = 72 * 1024;
 int resident_stride(int res_k) { return res_k * 4 + 64; }
 
-SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int slots,
+SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int slots,
                    int res_bytes = 0, int budget = kBigSmem) {
+  const int topk = p->cfg.top_k, ve_max = p->ve_max;
   SmemGeom s;
   // routing tables (virtual experts + expert-sorted slots) for the expert kernels
   s.table_bytes = 0;
@@ -203,7 +204,7 @@ SmemGeom smem_geom(int kind, int nt, int tail_tg_eff, int topk, int ve_max, int 
   // share an SM; with the half budget, two CTAs of one expert kernel do
   // enough bytes in flight to saturate HBM (about 6 x 16 KB per SM); more only
   // lengthens the queues every other memory request waits behind
-  s.nstages = std::max(2, std::min(g_max_stages, (budget - stage_off) / s.stage_bytes));
+  s.nstages = std::max(2, std::min(p->max_stages, (budget - stage_off) / s.stage_bytes));
   s.stage_off = stage_off;
   s.total = (size_t)stage_off + (size_t)s.nstages * s.stage_bytes;
   // more than half of the SM's shared memory: never two CTAs on one SM
@@ -234,14 +235,13 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   f.expert_per_sm = 1;
   if (f.nt_e == 1 && p->expert_per_sm_max >= 2) {
     const int slots = B * p->cfg.top_k;
-    const SmemGeom h = smem_geom(KIND_EGU, 1, 1, p->cfg.top_k, p->ve_max, slots, 0, kHalfSmem);
+    const SmemGeom h = smem_geom(p, KIND_EGU, 1, 1, slots, 0, kHalfSmem);
     if (h.nstages >= 3 && h.total <= (size_t)kHalfSmem) f.expert_per_sm = 2;
   }
   f.expert_grid = p->num_sms * f.expert_per_sm;
   return f;
 }
 
-int g_split_cost = 2;  // split-K piece-end price in stages (environment MOE_SPLIT_COST)
 
 Params base_params(const moe_plan_s* p, int B) {
   Params q;
@@ -311,10 +311,12 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
 // Price of a split-K piece end in stages: partial sums out and the
 // finalising sums back in grow with the piece's token tiles, but more slowly
 // than a stage's own work does (a stage of 16 tiles costs about 2x one of 1).
-int split_cost_for(int nt) { return g_split_cost * (1 + std::max(1, nt) / 4); }
+int split_cost_for(const moe_plan_s* p, int nt) { return p->split_cost * (1 + std::max(1, nt) / 4); }
 
 // split-K factor of a kind whose row-block count the host knows
-int ppr_for(int mats, int C, int ctas, int nt) { return best_ppr(mats, C, ctas, split_cost_for(nt)); }
+int ppr_for(const moe_plan_s* p, int mats, int C, int ctas, int nt) {
+  return best_ppr(mats, C, ctas, split_cost_for(p, nt));
+}
 
 // Router row blocks are the first pieces handed out and the routing waits
 // for all of them: they get pieces of at most ~C/12 chunks.
@@ -330,18 +332,18 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     const KindGeom& g = p->g[kind];
     if (kind == KIND_FRONT) {
       nt = f.nt_front;
-      const int ppr = ppr_for(g.RB, g.C, f.front_workers, nt);
+      const int ppr = ppr_for(p, g.RB, g.C, f.front_workers, nt);
       pieces = (size_t)p->RB_router * router_ppr(ppr, g.C) + (size_t)(g.RB - p->RB_router) * ppr;
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      pieces = (size_t)passes * g.RB * ppr_for(g.RB * passes, g.C, f.tail_grid, nt);
+      pieces = (size_t)passes * g.RB * ppr_for(p, g.RB * passes, g.C, f.tail_grid, nt);
     } else {
       nt = f.nt_e;
       // the split depends on the routing: take the largest over every
       // possible count of virtual experts
       for (int V = 1; V <= p->ve_max; ++V)
-        pieces = std::max(pieces, (size_t)V * g.RB * ppr_for(V * g.RB, g.C, f.expert_grid, nt));
+        pieces = std::max(pieces, (size_t)V * g.RB * ppr_for(p, V * g.RB, g.C, f.expert_grid, nt));
     }
     best = std::max(best, pieces * (size_t)nt * 1024);
   }
@@ -392,8 +394,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
   if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
-  if (const char* e = getenv("MOE_MAX_STAGES")) g_max_stages = std::max(2, std::min(8, atoi(e)));
-  g_split_cost = p->split_cost;
+  if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -527,12 +528,12 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
   SmemGeom g[KIND_COUNT];
   int stage_bytes = 0;
   for (int k = 0; k < KIND_COUNT; ++k) {
-    g[k] = smem_geom(k, 1, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, k == KIND_TAIL ? res_bytes : 0);
+    g[k] = smem_geom(p, k, 1, tail_tg_eff, B * c.top_k, k == KIND_TAIL ? res_bytes : 0);
     stage_bytes = std::max(stage_bytes, g[k].stage_bytes);
   }
   const int table_bytes = g[KIND_EGU].table_bytes;
   const int stage_off = kStageOff + table_bytes + res_bytes;
-  const int nstages = std::max(2, std::min(g_max_stages, (kBigSmem - stage_off) / stage_bytes));
+  const int nstages = std::max(2, std::min(p->max_stages, (kBigSmem - stage_off) / stage_bytes));
   const size_t total = std::max((size_t)stage_off + (size_t)nstages * stage_bytes, (size_t)(116 * 1024));
   MegaParams mp;
   std::memset(&mp, 0, sizeof(mp));
@@ -549,12 +550,12 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
     q.need_rb_edn = p->g[KIND_EDN].RB;
     q.need_rb_sh = p->g[KIND_FRONT].RB - p->RB_router - p->RB_lat;
     if (k == KIND_FRONT) {
-      q.PPR = ppr_for(q.RB, q.C, f.front_workers, 1);
+      q.PPR = ppr_for(p, q.RB, q.C, f.front_workers, 1);
       q.PPR_r = router_ppr(q.PPR, q.C);
       mp.n_front = p->RB_router * q.PPR_r + (q.RB - p->RB_router) * q.PPR;
     } else if (k == KIND_EGU || k == KIND_EDN) {
       q.piece_ctas = f.expert_grid;
-      q.split_cost = split_cost_for(1);
+      q.split_cost = split_cost_for(p, 1);
     } else {
       if (res_bytes) {
         q.res_off = kStageOff + table_bytes;
@@ -562,7 +563,7 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
         q.res_k = res_k;
       }
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid, 1);
+      q.PPR = ppr_for(p, q.RB * passes, q.C, f.tail_grid, 1);
     }
     mp.k[k] = q;
   }
@@ -582,7 +583,6 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
 
 moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStream_t s) {
   const moe_config& c = p->cfg;
-  g_split_cost = p->split_cost;
   const FwdGeom f = fwd_geom(p, B);
   const int tail_tg_eff = std::min(B, p->tail_tg);
   Params base = base_params(p, B);
@@ -594,9 +594,9 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   //   front (router, latent, shared gate/up) -> expert gate/up -> expert down -> tail.
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_FRONT, f.nt_front, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k);
+    const SmemGeom sm = smem_geom(p, KIND_FRONT, f.nt_front, tail_tg_eff, B * c.top_k);
     set_kind(q, p, KIND_FRONT, sm);
-    q.PPR = ppr_for(q.RB, q.C, f.front_workers, f.nt_front);
+    q.PPR = ppr_for(p, q.RB, q.C, f.front_workers, f.nt_front);
     q.PPR_r = router_ppr(q.PPR, q.C);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_FRONT, f.nt_front, q, f.front_grid, sm.total, s, p->use_pdl));
@@ -604,22 +604,22 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_EGU, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, 0,
+    const SmemGeom sm = smem_geom(p, KIND_EGU, f.nt_e, tail_tg_eff, B * c.top_k, 0,
                                   f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
     set_kind(q, p, KIND_EGU, sm);
     q.piece_ctas = f.expert_grid;
-    q.split_cost = split_cost_for(f.nt_e);
+    q.split_cost = split_cost_for(p, f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
   }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(KIND_EDN, f.nt_e, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, 0,
+    const SmemGeom sm = smem_geom(p, KIND_EDN, f.nt_e, tail_tg_eff, B * c.top_k, 0,
                                   f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
     set_kind(q, p, KIND_EDN, sm);
     q.piece_ctas = f.expert_grid;
-    q.split_cost = split_cost_for(f.nt_e);
+    q.split_cost = split_cost_for(p, f.nt_e);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
@@ -630,7 +630,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     const int res_bytes =
         (B * resident_stride(res_k) <= kResidentMax) ? B * resident_stride(res_k) : 0;
     const SmemGeom sm =
-        smem_geom(KIND_TAIL, f.nt_tail, tail_tg_eff, c.top_k, p->ve_max, B * c.top_k, res_bytes);
+        smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * c.top_k, res_bytes);
     set_kind(q, p, KIND_TAIL, sm);
     if (res_bytes) {
       q.res_off = kStageOff + sm.table_bytes;
@@ -638,7 +638,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       q.res_k = res_k;
     }
     const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-    q.PPR = ppr_for(q.RB * passes, q.C, f.tail_grid, f.nt_tail);
+    q.PPR = ppr_for(p, q.RB * passes, q.C, f.tail_grid, f.nt_tail);
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][1], s));
