@@ -233,6 +233,34 @@ MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
 MOE_API moe_status moe_debug_trace(moe_plan p, uint64_t *host, int64_t count);
 MOE_API moe_status moe_get_profile(moe_plan p, float *ms, int32_t *count);
 
+/* Launch geometry of one kernel kind, as moe_forward would choose it. */
+typedef struct moe_geometry {
+  int32_t kind;               /* 0 dense front, 1 expert gate/up, 2 expert down, 3 latent tail */
+  int32_t grid;               /* CTAs launched */
+  int32_t ctas_per_sm;        /* 1, or 2 for the one-tile expert kernels */
+  int32_t token_tiles;        /* 8-column token tiles the kernel is instantiated for */
+  int32_t max_piece_tokens;   /* most tokens one piece can hold */
+  int32_t stages;             /* ring depth */
+  int32_t stage_bytes;        /* bytes of one ring stage */
+  int32_t pieces_per_row_block; /* split-K factor (expert kinds: at the most virtual experts) */
+  int64_t smem_bytes;         /* dynamic shared memory per CTA */
+  int64_t partial_floats_needed;   /* split-K partial sums this forward can write */
+  int64_t partial_floats_capacity; /* what a plan allocates (largest over every B) */
+  int32_t route_logit_floats; /* front: logits the routing CTA can stage at once (else 0) */
+  int32_t resident_tail_bytes; /* tail: shared-memory bytes of the resident activation (0: staged) */
+} moe_geometry;
+
+/*
+ * The geometry moe_forward(num_tokens) would use on a device with num_sms
+ * SMs, for the 4 kinds (out[0..3]), with the default settings (environment
+ * variables are not read).  Host only: needs no device and allocates no
+ * device memory, so the planner can be checked anywhere.
+ * Errors: INVALID_ARG (null, bad shape, num_sms < 2, num_tokens outside
+ * 1..max_tokens), UNSUPPORTED (shape beyond the limits above), OOM.
+ */
+MOE_API moe_status moe_debug_geometry(const moe_config *cfg, int32_t num_sms, int32_t num_tokens,
+                                      moe_geometry *out);
+
 /*
  * Router scores and top-k for callers that cannot allocate device memory.
  * The source pages have no counterpart to this call; it exists for code that

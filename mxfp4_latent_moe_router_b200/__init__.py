@@ -26,10 +26,11 @@ MOE_DBG_LOGITS, MOE_DBG_Z, MOE_DBG_H, MOE_DBG_Y, MOE_DBG_HS = range(5)
 ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forward_host",
                "moe_last_routing", "moe_debug_fetch", "moe_sync_status", "moe_get_plan_info",
                "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile",
-               "moe_route_noalloc", "moe_debug_trace"]
-# launch slots: the four kernels a forward of more than 8 tokens runs (the
-# dense front kernel streams the router, latent-projection and shared-expert
-# gate/up rows and runs top-k), then the single fused launch of smaller ones
+               "moe_route_noalloc", "moe_debug_trace", "moe_debug_geometry"]
+# launch slots: the four kernels a forward runs (the dense front kernel
+# streams the router, latent-projection and shared-expert gate/up rows and
+# runs top-k), then the single fused launch that MOE_FUSED=1 selects for
+# forwards of at most 8 tokens
 KERNEL_NAMES = ["dense_front", "expert_gate_up", "expert_down", "latent_tail", "fused_block"]
 
 
@@ -61,6 +62,16 @@ class moe_plan_info(ctypes.Structure):
                 ("kernels_per_forward", ctypes.c_int32)]
 
 
+class moe_geometry(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("grid", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
+                ("token_tiles", ctypes.c_int32), ("max_piece_tokens", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("stage_bytes", ctypes.c_int32),
+                ("pieces_per_row_block", ctypes.c_int32), ("smem_bytes", ctypes.c_int64),
+                ("partial_floats_needed", ctypes.c_int64),
+                ("partial_floats_capacity", ctypes.c_int64),
+                ("route_logit_floats", ctypes.c_int32), ("resident_tail_bytes", ctypes.c_int32)]
+
+
 _lib = None
 
 
@@ -89,6 +100,8 @@ def load_library():
     lib.moe_set_profiling.argtypes = [P, ctypes.c_int32]
     lib.moe_debug_trace.argtypes = [P, P, ctypes.c_int64]
     lib.moe_get_profile.argtypes = [P, P, P]
+    lib.moe_debug_geometry.argtypes = [ctypes.POINTER(moe_config), ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.POINTER(moe_geometry)]
     lib.moe_status_str.argtypes = [ctypes.c_int]
     lib.moe_status_str.restype = ctypes.c_char_p
     for n in ABI_SYMBOLS:
@@ -193,6 +206,15 @@ def moe_debug_trace(plan: int, num_sms: int):
     a = np.zeros((len(KERNEL_NAMES), num_sms, 24), np.uint64)
     _check(load_library().moe_debug_trace(plan, a.ctypes.data, a.size), "moe_debug_trace")
     return a
+
+
+def moe_debug_geometry(cfg: moe_config, num_sms: int, num_tokens: int) -> list:
+    """Launch geometry of the four kernels for a forward of num_tokens tokens on
+    num_sms SMs, with default settings (host only: no device needed)."""
+    out = (moe_geometry * 4)()
+    _check(load_library().moe_debug_geometry(ctypes.byref(cfg), num_sms, num_tokens, out),
+           "moe_debug_geometry")
+    return [{f[0]: getattr(g, f[0]) for f in moe_geometry._fields_} for g in out]
 
 
 def moe_plan_destroy(plan: int) -> None:

@@ -377,30 +377,11 @@ moe_status check_cfg(const moe_config* c) {
   return MOE_OK;
 }
 
-moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
-  p->cfg = *cfg;
-  p->device = device;
-  int ndev = 0;
-  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
-    cudaGetLastError();
-    return MOE_ERR_UNSUPPORTED;
-  }
-  cudaDeviceProp prop;
-  CUDA_TRY(cudaGetDeviceProperties(&prop, device));
-  if (prop.major != 10) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
-  p->num_sms = prop.multiProcessorCount;
-  if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
-  if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
-  if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
-  if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
-  if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
-  if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
-  if (set_smem_limits(kBigSmem) != 0) {
-    cudaGetLastError();
-    return MOE_ERR_CUDA;
-  }
-
-  const moe_config& c = *cfg;
+// Row blocks, chunks and packed sizes of every kind, the tail's token group
+// and the routing-table bound: everything about a plan that follows from its
+// shape alone (no device involved).
+void plan_shape(moe_plan_s* p) {
+  const moe_config& c = p->cfg;
   const int H = c.hidden, L = c.latent, E = c.num_experts, I = c.expert_inter, Is = c.shared_inter;
   // the front kernel's row blocks: router (first, so the routing starts
   // early), latent projection, shared expert gate/up (64 + 64 rows a block)
@@ -432,6 +413,40 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   const int maxB = c.max_tokens, K = c.top_k;
   const int slots = maxB * K;
   p->ve_max = std::min(E, slots) + ceil_div(slots, kExpertTgSmall) + 1;  // any group size
+}
+
+moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
+  p->cfg = *cfg;
+  p->device = device;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return MOE_ERR_UNSUPPORTED;
+  }
+  cudaDeviceProp prop;
+  CUDA_TRY(cudaGetDeviceProperties(&prop, device));
+  if (prop.major != 10) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
+  p->num_sms = prop.multiProcessorCount;
+  if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
+  if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
+  if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
+  if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
+  if (set_smem_limits(kBigSmem) != 0) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+
+  const moe_config& c = *cfg;
+  const int H = c.hidden, L = c.latent, E = c.num_experts, I = c.expert_inter, Is = c.shared_inter;
+  plan_shape(p);
+  KindGeom& fr = p->g[KIND_FRONT];
+  KindGeom& eg = p->g[KIND_EGU];
+  KindGeom& ed = p->g[KIND_EDN];
+  KindGeom& tl = p->g[KIND_TAIL];
+  const int maxB = c.max_tokens, K = c.top_k;
+  const int slots = maxB * K;
 
   void* v;
   TRY(alloc(p, &v, fr.weight_bytes, true));
@@ -949,6 +964,73 @@ moe_status moe_get_profile(moe_plan p, float* ms, int32_t* count) {
   }
   *count = p->prof_count;
   p->prof_count = 0;
+  return MOE_OK;
+}
+
+moe_status moe_debug_geometry(const moe_config* cfg, int32_t num_sms, int32_t num_tokens,
+                              moe_geometry* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  const moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (num_sms < 2 || num_tokens < 1 || num_tokens > cfg->max_tokens) return MOE_ERR_INVALID_ARG;
+  moe_plan_s* p = new (std::nothrow) moe_plan_s();
+  if (!p) return MOE_ERR_OOM;
+  p->cfg = *cfg;
+  p->num_sms = num_sms;
+  plan_shape(p);
+  const moe_config& c = p->cfg;
+  const int B = num_tokens, K = c.top_k;
+  const FwdGeom f = fwd_geom(p, B);
+  const int tail_tg_eff = std::min(B, p->tail_tg);
+  for (int k = 0; k < KIND_COUNT; ++k) {
+    moe_geometry& o = out[k];
+    std::memset(&o, 0, sizeof(o));
+    o.kind = k;
+    o.partial_floats_capacity = (int64_t)partial_floats(p, k);
+    const KindGeom& g = p->g[k];
+    SmemGeom sm;
+    if (k == KIND_FRONT) {
+      sm = smem_geom(p, KIND_FRONT, f.nt_front, tail_tg_eff, B * K);
+      const int ppr = ppr_for(p, g.RB, g.C, f.front_workers, f.nt_front);
+      const int pieces = p->RB_router * router_ppr(ppr, g.C) + (g.RB - p->RB_router) * ppr;
+      o.grid = f.front_grid;
+      o.ctas_per_sm = 1;
+      o.token_tiles = f.nt_front;
+      o.max_piece_tokens = B;
+      o.pieces_per_row_block = ppr;
+      o.partial_floats_needed = (int64_t)pieces * f.nt_front * 1024;
+      o.route_logit_floats = sm.nstages * sm.stage_bytes / 4 - ((c.num_experts + 31) & ~31);
+    } else if (k == KIND_EGU || k == KIND_EDN) {
+      sm = smem_geom(p, k, f.nt_e, tail_tg_eff, B * K, 0, f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
+      o.grid = f.expert_grid;
+      o.ctas_per_sm = f.expert_per_sm;
+      o.token_tiles = f.nt_e;
+      o.max_piece_tokens = std::min(B, expert_tg(p, B));
+      o.pieces_per_row_block = ppr_for(p, p->ve_max * g.RB, g.C, f.expert_grid, f.nt_e);
+      int64_t most = 0;
+      for (int V = 1; V <= p->ve_max; ++V)
+        most = std::max(most, (int64_t)V * g.RB * ppr_for(p, V * g.RB, g.C, f.expert_grid, f.nt_e));
+      o.partial_floats_needed = most * f.nt_e * 1024;
+    } else {
+      const int res_k = g.C * kDenseChunkK;
+      const int res_bytes =
+          (B * resident_stride(res_k) <= kResidentMax) ? B * resident_stride(res_k) : 0;
+      sm = smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * K, res_bytes);
+      const int passes = (B + p->tail_tg - 1) / p->tail_tg;
+      const int ppr = ppr_for(p, g.RB * passes, g.C, f.tail_grid, f.nt_tail);
+      o.grid = f.tail_grid;
+      o.ctas_per_sm = 1;
+      o.token_tiles = f.nt_tail;
+      o.max_piece_tokens = tail_tg_eff;
+      o.pieces_per_row_block = ppr;
+      o.partial_floats_needed = (int64_t)passes * g.RB * ppr * f.nt_tail * 1024;
+      o.resident_tail_bytes = res_bytes;
+    }
+    o.stages = sm.nstages;
+    o.stage_bytes = sm.stage_bytes;
+    o.smem_bytes = (int64_t)sm.total;
+  }
+  delete p;
   return MOE_OK;
 }
 
