@@ -165,7 +165,6 @@ moe_status alloc(moe_plan p, void** out, size_t bytes, bool packed) {
 
 bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
 
-
 struct SmemGeom {
   int stage_bytes, nstages, act_off, act_stride, table_bytes, stage_off, res_bytes;
   size_t total;
@@ -241,7 +240,6 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   f.expert_grid = p->num_sms * f.expert_per_sm;
   return f;
 }
-
 
 Params base_params(const moe_plan_s* p, int B) {
   Params q;
