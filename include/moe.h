@@ -118,7 +118,8 @@ typedef struct moe_plan_info {
   int32_t device;
   int32_t num_sms;
   int32_t front_ctas;       /* CTAs streaming the router / latent / shared gate-up rows */
-  int32_t expert_ctas;      /* CTAs of each routed-expert kernel */
+  int32_t expert_ctas;      /* CTAs of each routed-expert kernel for max_tokens tokens
+                               (two per SM when a piece holds one token tile) */
   int64_t packed_bytes;     /* library-owned packed weights */
   int64_t workspace_bytes;  /* library-owned activations, routing metadata, partial sums */
   int64_t dense_weight_bytes;      /* bf16 bytes one forward streams regardless of routing */
