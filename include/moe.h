@@ -19,9 +19,10 @@
  *     kernel, saving one launch and one intermediate write + re-read: page
  *     "Kimi K3 在 vLLM 中的性能优化", section 延迟 MXFP4 最终化 ("deferred MXFP4
  *     finalize");
- *   - decode batch 1-64 and the 16 x 8 speculative-verify shape: page 1 intro
- *     and page "Kimi K3 vLLM 优化：NVIDIA 解码速度提升 1.68×", section
- *     上游测试实际展示了什么.
+ *   - decode batch 1-64 and the 16 x 8 speculative-verify shape: page
+ *     "Hyper Optimizing Kimi K3 in vLLM: Moving Fast and Responsibly",
+ *     introduction, and page "Kimi K3 vLLM 优化：NVIDIA 解码速度提升 1.68×",
+ *     section 上游测试实际展示了什么.
  *   MXFP4 encodings follow the OCP Microscaling (MX) v1.0 specification.
  *
  * Conventions for every call:

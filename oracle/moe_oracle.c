@@ -28,7 +28,8 @@
  *       "deferred MXFP4 finalize": the top-k weighted combine of the MXFP4
  *       expert outputs feeds the latent-tail up-projection.)
  *   7. shared   h_s = silu(x . W_sg) * (x . W_su),  o_s = h_s . W_sd
- *      (page 1, same section: the shared expert is independent of routing.)
+ *      (page "Hyper Optimizing Kimi K3 in vLLM: Moving Fast and Responsibly",
+ *       section 从算子之间找时间: the shared expert is independent of routing.)
  *   8. output   out[n] = sum_l c[l] * W_out[l][n] + o_s[n]
  *
  * Readings where the pages are silent:
