@@ -1,7 +1,8 @@
 """Edge cases of the CUDA path against the CPU oracle: the largest expert count
 and top-k the library takes, the largest batch, sigmoid scoring without a
 selection bias, the fused single launch with a tail activation too large to
-keep in shared memory, and 32-token virtual experts."""
+keep in shared memory, 32-token virtual experts, and raw (unrenormalised)
+scores with a routed scale."""
 import numpy as np
 import pytest
 
@@ -90,3 +91,13 @@ def test_thirty_two_token_expert_groups(B, E, k, monkeypatch):
                                seed=101 + B, scale_exp_lo=-5, scale_exp_hi=-2)
     w = synth.make_weights(shape)
     _check(shape, w, synth.make_x(shape), max_tokens=B)
+
+
+@pytest.mark.parametrize("score_fn", [synth.SCORE_SOFTMAX, synth.SCORE_SIGMOID])
+def test_raw_scores_with_routed_scale(score_fn):
+    # renormalisation off and a routed scale: each combine weight is the
+    # chosen expert's raw score times 2.5
+    shape = synth.custom_shape("raw", 5, 256, 128, 24, 3, 64, 64, score_fn, seed=111 + score_fn,
+                               renormalize=0, routed_scale=2.5)
+    w = synth.make_weights(shape)
+    _check(shape, w, synth.make_x(shape), max_tokens=8)

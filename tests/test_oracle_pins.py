@@ -233,11 +233,17 @@ def _dense_reference(shape, w, x):
     return out, logits, sel_all
 
 
-@pytest.mark.parametrize("score_fn,k", [(synth.SCORE_SOFTMAX, 2), (synth.SCORE_SIGMOID, 3),
-                                        (synth.SCORE_SIGMOID, 1)])
-def test_block_matches_dense_enumeration(score_fn, k):
+@pytest.mark.parametrize("score_fn,k,renorm,scale", [(synth.SCORE_SOFTMAX, 2, 1, 1.0),
+                                                     (synth.SCORE_SIGMOID, 3, 1, 1.0),
+                                                     (synth.SCORE_SIGMOID, 1, 1, 1.0),
+                                                     (synth.SCORE_SIGMOID, 3, 0, 2.5),
+                                                     (synth.SCORE_SOFTMAX, 2, 0, 0.5)])
+def test_block_matches_dense_enumeration(score_fn, k, renorm, scale):
+    # also without renormalisation and with a routed scale: the combine weight
+    # is then the raw score times the scale
     shape = synth.custom_shape("enum", 3, 96, 64, 6, k, 64, 32, score_fn, seed=11 + k,
-                               scale_exp_lo=-5, scale_exp_hi=-2)
+                               scale_exp_lo=-5, scale_exp_hi=-2, renormalize=renorm,
+                               routed_scale=scale)
     w = synth.make_weights(shape)
     x = synth.make_x(shape)
     r = oracle.forward(shape, w, x)
