@@ -226,7 +226,8 @@ __device__ __forceinline__ void stage_begin(const Params& p, const Hdr& h, uint8
   bulk_g2s(sb + kHdrBytes, weight_src<KIND>(p, h), kTile, bar);
 }
 
-// The lanes' 16-byte copies are done; let the barrier track them and arrive.
+// The lanes' 16-byte copies are issued: the barrier now tracks their
+// completion, and lane 0 adds its arrival once every lane has registered.
 __device__ __forceinline__ void rows_async_done(uint64_t* bar, int lane) {
   cp_async_mbar_arrive(bar);
   __syncwarp();
