@@ -1,8 +1,9 @@
 """Edge cases of the CUDA path against the CPU oracle: the largest expert count
 and top-k the library takes, the largest batch, sigmoid scoring without a
 selection bias, the fused single launch with a tail activation too large to
-keep in shared memory, 32-token virtual experts, and raw (unrenormalised)
-scores with a routed scale."""
+keep in shared memory, 32-token virtual experts, raw (unrenormalised)
+scores with a routed scale, and the host-side geometry query against a real
+plan."""
 import numpy as np
 import pytest
 
@@ -101,3 +102,18 @@ def test_raw_scores_with_routed_scale(score_fn):
                                renormalize=0, routed_scale=2.5)
     w = synth.make_weights(shape)
     _check(shape, w, synth.make_x(shape), max_tokens=8)
+
+
+def test_geometry_query_matches_the_plan():
+    # the host-only geometry query and a plan on this device choose alike
+    shape = synth.SHAPES["tiny"]
+    for B in (1, 16):
+        cfg = moe.config_from_shape(shape, max_tokens=B)
+        plan = moe.MoePlan(cfg)
+        try:
+            info = plan.info()
+            front, egu, edn, tail = moe.moe_debug_geometry(cfg, info.num_sms, B)
+            assert front["grid"] == info.front_ctas + 1  # + the routing CTA
+            assert egu["grid"] == edn["grid"] == info.expert_ctas
+        finally:
+            plan.close()
