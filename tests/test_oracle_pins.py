@@ -83,11 +83,13 @@ def test_e8m0_matches_torch_decoder():
 def test_bf16_decoder_exhaustive():
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     ref = _bf16_torch(bits)
-    got = np.array([oracle.bf16_value(int(b)) for b in bits[::97]])
-    r = ref[::97]
-    nan = np.isnan(r)
+    # every one of the 65536 patterns
+    got = np.array([oracle.bf16_value(int(b)) for b in bits])
+    nan = np.isnan(ref)
     assert np.array_equal(np.isnan(got), nan)
-    np.testing.assert_array_equal(got[~nan], r[~nan])
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    # signed zeros keep their sign
+    assert math.copysign(1.0, oracle.bf16_value(0x8000)) == -1.0
 
 
 def test_dequant_exhaustive_codes_and_scales():
@@ -357,3 +359,107 @@ def test_hand_computed_tiny_case():
     expect[0] = -0.5 * sig(1)
     np.testing.assert_allclose(r["out"][0], expect, rtol=1e-14, atol=1e-15)
     np.testing.assert_allclose(r["h_s"][0][4], 0.5 * sig(1), rtol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# the selection margin and the router-only entry point
+#
+# The margin (k-th minus (k+1)-th selection key) decides which tokens the GPU
+# parity tests hold to exact ids, so it is pinned on its own: hand cases whose
+# keys are closed forms, and the dense numpy/scipy route at non-zero input.
+
+
+def _one_hot_router(logit_row, k, score_fn, bias=None, renorm=1, scale=1.0):
+    """x = e0, W_r row 0 = logit_row: the logits are exactly logit_row."""
+    E = len(logit_row)
+    shape = synth.custom_shape("margin", 1, 32, 32, E, k, 32, 0, score_fn, renormalize=renorm,
+                               routed_scale=scale)
+    w = synth.make_weights(shape)
+    Wr = np.zeros((32, E), np.float32)
+    Wr[0] = logit_row
+    w["router_w"] = _bf(Wr)
+    w["router_bias"] = None if bias is None else np.asarray(bias, np.float32)
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0] = 1.0
+    return shape, w, _bf(x)
+
+
+def test_margin_softmax_hand_case():
+    # logits (1, 0.5, 2, -1, 0.25), top-2: experts 2 then 0; the next is 1.
+    # margin = p_0 - p_1 = (e^1 - e^0.5) / sum_e e^{l_e}
+    lg = [1.0, 0.5, 2.0, -1.0, 0.25]
+    shape, w, x = _one_hot_router(lg, 2, synth.SCORE_SOFTMAX)
+    den = sum(math.exp(v) for v in lg)
+    for r in (oracle.route(shape, w, x), oracle.forward(shape, w, x, intermediates=False)):
+        assert r["ids"][0].tolist() == [2, 0]
+        assert r["margin"][0] == pytest.approx((math.exp(1.0) - math.exp(0.5)) / den, rel=1e-14)
+        e2, e0 = math.exp(2.0) / den, math.exp(1.0) / den
+        np.testing.assert_allclose(r["weights"][0], [e2 / (e2 + e0), e0 / (e2 + e0)], rtol=1e-14)
+
+
+def test_margin_sigmoid_with_bias_hand_case():
+    # keys s_e + b_e with s = sigmoid(logit).  Logits (0, 2, -1, 1), biases
+    # (0.25, -0.5, 0.5, 0): keys 0.75, sig(2)-0.5 = 0.3808, sig(-1)+0.5 = 0.7689,
+    # sig(1) = 0.7311.  Top-2: experts 2 and 0; the next is 3.
+    sig = lambda t: 1.0 / (1.0 + math.exp(-t))
+    lg, bias = [0.0, 2.0, -1.0, 1.0], [0.25, -0.5, 0.5, 0.0]
+    shape, w, x = _one_hot_router(lg, 2, synth.SCORE_SIGMOID, bias=bias)
+    for r in (oracle.route(shape, w, x), oracle.forward(shape, w, x, intermediates=False)):
+        assert r["ids"][0].tolist() == [2, 0]
+        assert r["margin"][0] == pytest.approx((sig(0.0) + 0.25) - sig(1.0), rel=1e-14)
+        # weights come from the unbiased scores
+        np.testing.assert_allclose(r["weights"][0],
+                                   [sig(-1.0) / (sig(-1.0) + 0.5), 0.5 / (sig(-1.0) + 0.5)], rtol=1e-14)
+
+
+def test_margin_is_infinite_when_every_expert_is_chosen():
+    shape, w, x = _one_hot_router([0.5, -0.25, 1.0], 3, synth.SCORE_SIGMOID, bias=[0.0, 0.1, -0.1])
+    for r in (oracle.route(shape, w, x), oracle.forward(shape, w, x, intermediates=False)):
+        assert math.isinf(r["margin"][0]) and r["margin"][0] > 0
+        assert sorted(r["ids"][0].tolist()) == [0, 1, 2]
+
+
+def test_margin_of_exact_tie_is_zero():
+    # two experts tie at the k-th place: the lower index is taken, margin 0
+    shape, w, x = _one_hot_router([1.0, 0.5, 0.5, -2.0], 2, synth.SCORE_SOFTMAX)
+    r = oracle.route(shape, w, x)
+    assert r["ids"][0].tolist() == [0, 1]
+    assert r["margin"][0] == 0.0
+
+
+@pytest.mark.parametrize("score_fn,k,renorm,scale", [(synth.SCORE_SOFTMAX, 2, 1, 1.0),
+                                                     (synth.SCORE_SIGMOID, 3, 1, 1.0),
+                                                     (synth.SCORE_SIGMOID, 4, 0, 2.5),
+                                                     (synth.SCORE_SOFTMAX, 3, 0, 0.5)])
+def test_route_matches_dense_route_at_nonzero_input(score_fn, k, renorm, scale):
+    """The router-only entry point at random (non-zero) input: logits, ids,
+    weights and margins against numpy/scipy, with the selection from a sort
+    of the dense keys; and the same values as the full forward."""
+    shape = synth.custom_shape("route", 7, 96, 64, 12, k, 64, 0, score_fn, seed=31 + k,
+                               renormalize=renorm, routed_scale=scale)
+    w = synth.make_weights(shape)
+    if score_fn == synth.SCORE_SIGMOID:
+        w["router_bias"] = (np.random.default_rng(5).standard_normal(12) * 0.05).astype(np.float32)
+    x = synth.make_x(shape)
+    r = oracle.route(shape, w, x)
+    f = oracle.forward(shape, w, x, intermediates=False)
+    xf = _bf16_torch(x).reshape(7, 96)
+    logits = xf @ _bf16_torch(w["router_w"]).reshape(96, 12)
+    if score_fn == synth.SCORE_SOFTMAX:
+        src = scipy.special.softmax(logits, axis=1)
+        keys = src
+    else:
+        src = scipy.special.expit(logits)
+        keys = src + w["router_bias"].astype(np.float64)
+    np.testing.assert_allclose(r["logits"], logits, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(r["keys"], keys, rtol=1e-12, atol=1e-14)
+    for b in range(7):
+        order = np.lexsort((np.arange(12), -keys[b]))     # key descending, index ascending
+        sel = order[:k]
+        assert r["ids"][b].tolist() == sel.tolist()
+        assert r["margin"][b] == pytest.approx(keys[b][order[k - 1]] - keys[b][order[k]], rel=1e-9,
+                                               abs=1e-14)
+        tot = src[b][sel].sum() if renorm else 1.0
+        np.testing.assert_allclose(r["weights"][b], src[b][sel] / tot * scale, rtol=1e-12)
+    for key in ("logits", "ids", "weights", "margin"):
+        np.testing.assert_array_equal(r[key], f[key])
