@@ -254,21 +254,36 @@ def _measured_traffic(workload: str) -> dict:
     return {k[len("bytes."):]: float(v) for k, v in kv.items() if k.startswith("bytes.")}
 
 
-def run_ours(args):
+def _step_bytes(shape, distinct):
+    """Algorithmic bytes of one layer step: every dense weight once, plus the
+    MXFP4 tensors of each distinct routed expert once."""
+    from mxfp4_latent_moe_router_b200 import synth
+    wb = synth.weight_bytes(shape)
+    return wb["dense"] + distinct * wb["per_expert"]
+
+
+def _kernel_bytes(shape, distinct):
+    H, L, E, I, Is = shape.hidden, shape.latent, shape.num_experts, shape.expert_inter, shape.shared_inter
+    per_expert_gu = 2 * I * L // 2 + 2 * I * L // 32
+    per_expert_dn = L * I // 2 + L * I // 32
+    kb = {"dense_front": 2 * H * (E + L + 2 * Is),
+          "expert_gate_up": distinct * per_expert_gu,
+          "expert_down": distinct * per_expert_dn,
+          "latent_tail": 2 * L * H + 2 * Is * H}
+    kb["fused_block"] = sum(kb.values())  # one launch streams them all
+    return kb
+
+
+def measure_workload(name, args, rank, local, dist, headline):
+    """Device-timed layer steps of one workload (K steps in one CUDA graph,
+    4 resident weight instances rotating), per-kernel event times, the same
+    metric end to end through moe_forward_host, and, for the headline
+    workload, the clocks during the timed region and a parity spot check."""
     import torch
     import mxfp4_latent_moe_router_b200 as moe
     from mxfp4_latent_moe_router_b200 import synth
 
-    ws, rank, local = _dist()
-    torch.cuda.set_device(local)
-    dist = None
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    shape = synth.SHAPES[args.workload]
+    shape = synth.SHAPES[name]
     B = shape.tokens
     INSTANCES = args.instances
     stream = torch.cuda.Stream()
@@ -293,9 +308,9 @@ def run_ours(args):
         for k in range(max(3, args.warmup)):
             step(k)
     stream.synchronize()
-    # parity spot check of instance 0 against the oracle (one token)
     spot = None
-    if rank == 0 and not args.no_check:
+    if headline and rank == 0 and not args.no_check:
+        # parity spot check of instance 0 against the oracle (one token)
         import oracle
         from tests.helpers import bf16_to_f32, rel_errors  # noqa
         xin = synth.make_x(shape, step=0)
@@ -315,19 +330,20 @@ def run_ours(args):
         g.replay()  # graph warm-up
     stream.synchronize()
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local) if headline else None
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
     with torch.cuda.stream(stream):
         e0.record(stream)
         g.replay()
         e1.record(stream)
     stream.synchronize()
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks else None
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -360,10 +376,8 @@ def run_ours(args):
         ids, _ = plans[k].routing(B)
         distinct.append(len(np.unique(ids)))
     info = plans[0].info()
-    dense_b = info.dense_weight_bytes
-    exp_b = info.expert_weight_bytes
     mean_distinct = float(np.mean(distinct))
-    step_bytes = dense_b + mean_distinct * exp_b
+    step_bytes = _step_bytes(shape, mean_distinct)
     hbm_peak, peak_src = _peaks()
     achieved_step = step_bytes / (us_step * 1e-6) / 1e9
 
@@ -384,16 +398,9 @@ def run_ours(args):
             tot[n] += ms[n]
         cnt += c
     kern_us = {n: tot[n] * 1e3 / max(cnt, 1) for n in tot if tot[n] > 0}
-    H, L, E, I, Is = shape.hidden, shape.latent, shape.num_experts, shape.expert_inter, shape.shared_inter
-    per_expert_gu = 2 * I * L // 2 + 2 * I * L // 32
-    per_expert_dn = L * I // 2 + L * I // 32
-    kern_bytes = {"dense_front": 2 * H * (E + L + 2 * Is),
-                  "expert_gate_up": mean_distinct * per_expert_gu,
-                  "expert_down": mean_distinct * per_expert_dn,
-                  "latent_tail": 2 * L * H + 2 * Is * H}
-    kern_bytes["fused_block"] = sum(kern_bytes.values())  # one launch streams them all
+    kern_bytes = _kernel_bytes(shape, mean_distinct)
     dom = max(kern_us, key=lambda n: kern_us[n])
-    traffic = _measured_traffic(args.workload)
+    traffic = _measured_traffic(name)
     ach = kern_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9 if kern_us[dom] > 0 else 0.0
     roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
             "frac": ach / hbm_peak, "traffic": traffic.get(dom), "peak_source": peak_src,
@@ -404,7 +411,7 @@ def run_ours(args):
 
     # end to end through the host-buffer entry point (pinned host memory)
     xh = [x.cpu().pin_memory() for x in xs]
-    oh = [torch.empty_like(x) .pin_memory() for x in xh]
+    oh = [torch.empty_like(x).pin_memory() for x in xh]
     with torch.cuda.stream(stream):
         for k in range(3):
             plans[k % INSTANCES].forward_host(xh[k % INPUT_POOL], oh[k % INPUT_POOL], stream=stream)
@@ -418,49 +425,119 @@ def run_ours(args):
             plans[k % INSTANCES].forward_host(xh[k % INPUT_POOL], oh[k % INPUT_POOL], stream=stream)
         f1.record(stream)
     stream.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
-    e2e_us = e2e_ms * 1e3 / args.steps
+    e2e_us = max_over_ranks(f0.elapsed_time(f1)) * 1e3 / args.steps
+    for p in plans:
+        p.close()
+    del plans
+    torch.cuda.empty_cache()
+    return {"shape": shape, "us_step": us_step, "step_bytes": step_bytes, "distinct": distinct,
+            "achieved": achieved_step, "peak": hbm_peak, "peak_src": peak_src, "roof": roof,
+            "e2e_us": e2e_us, "clk": clk, "spot": spot, "spread": spread, "info": info,
+            "host_w0": host_w0, "kern_us": kern_us}
 
-    # CPU oracle baseline (rank 0, one GPU only)
+
+def cpu_baselines(shape, w, all_tokens, one_tokens):
+    """The oracle as it stands, timed on the host cores: its token loop over
+    all OpenMP threads, and on one thread.  Returns per-layer-step µs."""
+    import oracle
+    nthr = oracle.num_threads()
+    us_all, cores, steps = oracle_sample(shape, w, all_tokens)
+    res = {"value": us_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+           "sample": "%g layer steps (%d tokens) of this workload on instance-0 weights, fp64 "
+                     "oracle, tokens spread over %d threads" % (steps, all_tokens, cores)}
+    if one_tokens:
+        oracle.set_threads(1)
+        try:
+            us1, _, steps1 = oracle_sample(shape, w, one_tokens)
+        finally:
+            oracle.set_threads(nthr)
+        res["one_thread"] = {"value": us1, "unit": UNIT, "cores": 1,
+                             "sample": "%g layer steps (%d tokens) on one thread" % (steps1, one_tokens)}
+    return res
+
+
+def run_ours(args):
+    import torch
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    head = measure_workload(args.workload, args, rank, local, dist, headline=True)
+    shape = head["shape"]
+    B, H = shape.tokens, shape.hidden
+    us_step = head["us_step"]
+
+    # every other workload, at N = 1 in the default run: the same
+    # measurement, summarised (the headline stays the workload above)
+    others = {}
+    if ws == 1 and args.all_workloads:
+        from mxfp4_latent_moe_router_b200 import synth
+        for name in synth.SHAPE_ORDER:
+            if name == args.workload:
+                continue
+            r = measure_workload(name, args, rank, local, dist, headline=False)
+            others[name] = r
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
         import oracle
-        n = max(4, min(2 * oracle.num_threads(), 64)) * B
-        us_cpu, cores, steps = oracle_sample(shape, host_w0, n)
-        cpu = {"value": us_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": "%d layer steps (%d tokens) of this workload on instance-0 weights, "
-                         "fp64 oracle, tokens spread over %d threads" % (steps, n, cores)}
+        n_all = max(4, min(2 * oracle.num_threads(), 64)) * B
+        cpu = cpu_baselines(shape, head["host_w0"], n_all, max(1, 3 // B) * B if B <= 8 else 0)
+        for name, r in others.items():
+            sh = r["shape"]
+            # a bounded token sample of the workload (every token costs about
+            # the same: the dense weights plus k experts); tiny takes more
+            n = 256 if sh.name == "tiny" else 16
+            us, cores, steps = oracle_sample(sh, r["host_w0"], n)
+            r["cpu"] = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
+                        "sample": "%d tokens (%g layer steps) of this workload, %d threads" % (n, steps, cores)}
 
     if rank == 0:
+        workloads = {}
+        for name, r in [(args.workload, head)] + list(others.items()):
+            sh = r["shape"]
+            workloads[name] = {
+                "us_per_step": r["us_step"], "tokens_per_s": sh.tokens / (r["us_step"] * 1e-6),
+                "distinct_experts": r["distinct"], "bytes_per_step": r["step_bytes"],
+                "weight_stream_gbs": r["achieved"], "hbm_frac": r["achieved"] / r["peak"],
+                "e2e_us_per_step": r["e2e_us"], "per_kernel_us": r["kern_us"],
+                "step_spread": r["spread"],
+                "cpu_baseline_us_per_step": (r.get("cpu") or {}).get("value")}
+        info = head["info"]
         line = {
             "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f16 MMA on bf16 + MXFP4 weights, fp32 accumulate",
             "data": "synthetic",
             "config": {"workload": _workload_desc(shape), "tokens_per_step": B,
-                       "weight_instances": INSTANCES,
+                       "weight_instances": args.instances,
                        "l2": "inputs larger than L2: %d weight instances rotate, %.0f MB touched per step"
-                             % (INSTANCES, step_bytes / 1e6),
+                             % (args.instances, head["step_bytes"] / 1e6),
                        "parallelism": "replicas" if ws > 1 else "single GPU"},
             "tokens_per_s": ws * B / (us_step * 1e-6),
-            "weight_stream_gbs": achieved_step,
-            "step_roofline": {"bound": "hbm", "achieved": achieved_step, "peak": hbm_peak,
-                              "unit": "GB/s", "frac": achieved_step / hbm_peak,
-                              "bytes_per_step": step_bytes, "peak_source": peak_src,
-                              "distinct_experts": distinct},
-            "roofline": roof,
+            "weight_stream_gbs": head["achieved"],
+            "step_roofline": {"bound": "hbm", "achieved": head["achieved"], "peak": head["peak"],
+                              "unit": "GB/s", "frac": head["achieved"] / head["peak"],
+                              "bytes_per_step": head["step_bytes"], "peak_source": head["peak_src"],
+                              "distinct_experts": head["distinct"]},
+            "roofline": head["roof"],
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": B * H * 2,
+            "e2e": {"value": head["e2e_us"], "unit": UNIT, "h2d_bytes_per_step": B * H * 2,
                     "d2h_bytes_per_step": B * H * 2},
             "gpu_launches": args.steps * info.kernels_per_forward,
-            "clocks": clk,
+            "clocks": head["clk"],
             "plan": {"front_ctas": info.front_ctas, "expert_ctas": info.expert_ctas},
-            "parity_spot_check": spot,
-            "step_spread": spread,
+            "parity_spot_check": head["spot"],
+            "step_spread": head["spread"],
+            "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
-    for p in plans:
-        p.close()
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -478,6 +555,9 @@ def main():
                     help="resident weight instances rotated per step (4 keeps every step out of L2)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-check", action="store_true")
+    ap.add_argument("--only", dest="all_workloads", action="store_false",
+                    help="measure only --workload (default at N=1: every workload, the "
+                         "chosen one as the headline)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -79,7 +79,8 @@ typedef struct moe_config {
 } moe_config;
 
 /*
- * Weights in canonical layout, all DEVICE pointers, row-major, 16-byte aligned.
+ * Weights in canonical layout, all DEVICE pointers, row-major, 16-byte aligned
+ * (router_bias: 4-byte aligned).
  * bf16 tensors are in "x . W" orientation [in][out]; MXFP4 tensors are
  * output-row-major with K (the reduction index) contiguous:
  *   router_w   bf16 [H][E]
@@ -146,8 +147,9 @@ typedef struct moe_plan_info {
  *                           2 at one token tile)
  *   MOE_EXPERT_SMALL_MAX_B=n  largest B with 8-token virtual experts (default
  *                           128; above it, 32-token groups)
- *   MOE_FAIL_ALLOC_AFTER=n  fail the (n+1)-th allocation with MOE_ERR_OOM
- *                           (tests of the error path)
+ *   MOE_FAIL_ALLOC_AFTER=n  fail this plan's (n+1)-th device allocation with
+ *                           MOE_ERR_OOM (tests of the error path; everything
+ *                           allocated before it is released)
  */
 MOE_API moe_status moe_plan_create(const moe_config *cfg, int device, moe_plan *out);
 
@@ -194,9 +196,24 @@ enum {
 };
 MOE_API moe_status moe_debug_fetch(moe_plan p, int32_t what, int32_t num_tokens, float *host, int64_t count);
 
-/* Synchronise the plan's streams and report a device-side error word
- * (MOE_ERR_TIMEOUT if a bounded wait gave up), then clear it. */
+/* Synchronise the device and report the plan's device-side error word
+ * (MOE_ERR_TIMEOUT if a bounded wait gave up), then clear it.  After a
+ * timeout the plan's scheduling state (split-K tickets, piece cursors, the
+ * routing flag and counts) is also cleared, so the next forward starts as on
+ * a fresh plan; the output of the forward that timed out is undefined. */
 MOE_API moe_status moe_sync_status(moe_plan p);
+
+/*
+ * Test of the timeout path, for tests only.  Enqueues on `stream` one thread
+ * that leaves the plan's scheduling state as a forward cut short by an
+ * expired wait could (a router row block counted, a split-K ticket taken, a
+ * piece cursor advanced, the routing flag raised), then runs the kernels'
+ * bounded flag wait on a flag that nothing sets, giving up after
+ * limit_polls polls (1..2^22; 1000 polls take well under a millisecond).
+ * The next moe_sync_status returns MOE_ERR_TIMEOUT and clears that state.
+ * Errors: INVALID_ARG, CUDA.
+ */
+MOE_API moe_status moe_debug_expire_wait(moe_plan p, int32_t limit_polls, void* stream);
 
 MOE_API moe_status moe_get_plan_info(moe_plan p, moe_plan_info *info);
 

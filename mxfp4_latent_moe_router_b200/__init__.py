@@ -26,7 +26,8 @@ MOE_DBG_LOGITS, MOE_DBG_Z, MOE_DBG_H, MOE_DBG_Y, MOE_DBG_HS = range(5)
 ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forward_host",
                "moe_last_routing", "moe_debug_fetch", "moe_sync_status", "moe_get_plan_info",
                "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile",
-               "moe_route_noalloc", "moe_debug_trace", "moe_debug_geometry"]
+               "moe_route_noalloc", "moe_debug_trace", "moe_debug_geometry",
+               "moe_debug_expire_wait"]
 # launch slots: the four kernels a forward runs (the dense front kernel
 # streams the router, latent-projection and shared-expert gate/up rows and
 # runs top-k), then the single fused launch that MOE_FUSED=1 selects for
@@ -91,6 +92,7 @@ def load_library():
     lib.moe_last_routing.argtypes = [P, P, P, ctypes.c_int32]
     lib.moe_debug_fetch.argtypes = [P, ctypes.c_int32, ctypes.c_int32, P, ctypes.c_int64]
     lib.moe_sync_status.argtypes = [P]
+    lib.moe_debug_expire_wait.argtypes = [P, ctypes.c_int32, P]
     lib.moe_get_plan_info.argtypes = [P, ctypes.POINTER(moe_plan_info)]
     lib.moe_plan_destroy.argtypes = [P]
     lib.moe_plan_destroy.restype = None
@@ -170,6 +172,11 @@ def moe_debug_fetch(plan: int, what: int, num_tokens: int, host) -> None:
 
 def moe_sync_status(plan: int) -> int:
     return load_library().moe_sync_status(plan)
+
+
+def moe_debug_expire_wait(plan: int, limit_polls: int, stream=None) -> int:
+    """Test of the timeout path: a bounded wait that runs out (see include/moe.h)."""
+    return load_library().moe_debug_expire_wait(plan, limit_polls, _stream_ptr(stream))
 
 
 def moe_get_plan_info(plan: int) -> moe_plan_info:

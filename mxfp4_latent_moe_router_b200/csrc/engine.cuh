@@ -119,6 +119,8 @@ struct MegaParams {
 int launch_kind(int kind, int nt, const Params& p, int grid, size_t smem, void* stream, bool pdl);
 int launch_mega(const MegaParams& mp, int grid, size_t smem, void* stream, bool pdl);
 int max_smem_optin();
+int launch_expire_wait(int* never, int* err, int* router_done, int* ticket, Ctl* ctl,
+                       int* route_ready, unsigned limit, void* stream);
 int set_smem_limits(size_t bytes);
 
 int launch_pack_dense(const void* src, int K, int N, int layout, int RB, int C, int rows_valid,

@@ -91,6 +91,7 @@ struct moe_plan_s {
   Ctl* ctl = nullptr;  // [kSlots]
   int* done = nullptr;  // [4] phase completion counts of the fused launch
   int* counters[KIND_COUNT] = {};
+  size_t counter_n[KIND_COUNT] = {};  // tickets per kind
   int* router_done = nullptr;
   int* route_ready = nullptr;
   float* partials[KIND_COUNT] = {};
@@ -108,6 +109,7 @@ struct moe_plan_s {
   int expert_per_sm_max = 2;     // environment MOE_EXPERT_CTAS_PER_SM
   int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
   bool use_pdl = true;
+  int fail_alloc_after = -1;     // environment MOE_FAIL_ALLOC_AFTER (tests only)
   // one launch per forward for B <= kFusedMaxTokens (environment MOE_FUSED=1);
   // off by default: measured slower than the four-launch chain at B = 1
   bool use_fused = false;
@@ -147,11 +149,9 @@ int pow2_at_least(int v) {
 moe_status alloc(moe_plan p, void** out, size_t bytes, bool packed) {
   void* d = nullptr;
   if (bytes == 0) bytes = 16;
-  if (getenv("MOE_FAIL_ALLOC_AFTER")) {  // fault injection for the OOM path (host side only)
-    static int left = -1;
-    if (left < 0) left = atoi(getenv("MOE_FAIL_ALLOC_AFTER"));
-    if (left-- == 0) return MOE_ERR_OOM;
-  }
+  // injected failure for tests of the OOM path (host side only): the plan's
+  // countdown comes from MOE_FAIL_ALLOC_AFTER at plan creation
+  if (p->fail_alloc_after >= 0 && p->fail_alloc_after-- == 0) return MOE_ERR_OOM;
   cudaError_t e = cudaMalloc(&d, bytes);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -413,6 +413,17 @@ void plan_shape(moe_plan_s* p) {
   p->ve_max = std::min(E, slots) + ceil_div(slots, kExpertTgSmall) + 1;  // any group size
 }
 
+// The control block (routing count, router-row count, error word, routing
+// flag, phase counts, per-kind piece cursors) and every kind's split-K
+// tickets back to zero, as a fresh plan has them.  Synchronous.
+constexpr size_t kControlBytes = 1024 + sizeof(Ctl) * kSlots;
+moe_status reset_control(moe_plan p) {
+  CUDA_TRY(cudaMemset(p->nve, 0, kControlBytes));
+  for (int k = 0; k < KIND_COUNT; ++k) CUDA_TRY(cudaMemset(p->counters[k], 0, sizeof(int) * p->counter_n[k]));
+  CUDA_TRY(cudaDeviceSynchronize());
+  return MOE_OK;
+}
+
 moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->cfg = *cfg;
   p->device = device;
@@ -431,6 +442,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
   if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
   if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
+  if (const char* e = getenv("MOE_FAIL_ALLOC_AFTER")) p->fail_alloc_after = std::max(0, atoi(e));
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -477,16 +489,17 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   TRY(alloc(p, &v, sizeof(VExpert) * p->ve_max, false));
   p->ve = (VExpert*)v;
   // small control block: nve, router_done, err, Ctl[KIND_COUNT]
-  TRY(alloc(p, &v, 1024 + sizeof(Ctl) * kSlots, false));
+  TRY(alloc(p, &v, kControlBytes, false));
   p->nve = (int*)v;
   p->router_done = p->nve + 1;
   p->err = p->nve + 2;
   p->done = p->nve + 8;
   p->route_ready = p->nve + 3;
   p->ctl = reinterpret_cast<Ctl*>((uint8_t*)v + 1024);
-  CUDA_TRY(cudaMemset(v, 0, 1024 + sizeof(Ctl) * kSlots));
+  CUDA_TRY(cudaMemset(v, 0, kControlBytes));
   const int cnt_n[KIND_COUNT] = {fr.RB, p->ve_max * eg.RB, p->ve_max * ed.RB, maxB * tl.RB};
   for (int k = 0; k < KIND_COUNT; ++k) {
+    p->counter_n[k] = cnt_n[k];
     TRY(alloc(p, &v, sizeof(int) * cnt_n[k], false));
     p->counters[k] = (int*)v;
     CUDA_TRY(cudaMemset(v, 0, sizeof(int) * cnt_n[k]));
@@ -742,6 +755,9 @@ moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
     for (const void* q : sh)
       if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
   }
+  // the selection bias is copied as floats: 4-byte alignment is all it needs
+  const bool use_bias = w->router_bias && c.score_fn == MOE_SCORE_SIGMOID;
+  if (use_bias && (reinterpret_cast<uintptr_t>(w->router_bias) & 3)) return MOE_ERR_INVALID_ARG;
   DeviceGuard g(p->device);
   cudaStream_t s = (cudaStream_t)stream;
   p->loaded = false;
@@ -769,8 +785,7 @@ moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
   const KindGeom& ed = p->g[KIND_EDN];
   CUDA_TRY((cudaError_t)launch_pack_mx(w->dn_codes, w->dn_scales, E, L, I, 0, ed.RB, ed.C,
                                        p->w_edn, p->err, s));
-  if (w->router_bias && c.score_fn == MOE_SCORE_SIGMOID) {
-    if (!aligned16(w->router_bias)) return MOE_ERR_INVALID_ARG;
+  if (use_bias) {
     CUDA_TRY(cudaMemcpyAsync(p->bias, w->router_bias, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
   } else {
     CUDA_TRY(cudaMemsetAsync(p->bias, 0, sizeof(float) * E, s));
@@ -821,9 +836,26 @@ moe_status moe_sync_status(moe_plan p) {
   CUDA_TRY(cudaMemcpy(&err, p->err, sizeof(int), cudaMemcpyDeviceToHost));
   if (err) {
     CUDA_TRY(cudaMemset(p->err, 0, sizeof(int)));
-    if (err & ((1 << ERR_WAIT_FULL) | (1 << ERR_WAIT_EMPTY) | (1 << ERR_WAIT_DEP))) return MOE_ERR_TIMEOUT;
+    if (err & ((1 << ERR_WAIT_FULL) | (1 << ERR_WAIT_EMPTY) | (1 << ERR_WAIT_DEP))) {
+      // A forward whose wait gave up may have left partial counts behind
+      // (router row blocks, split-K tickets, piece cursors, the routing flag,
+      // the fused launch's phase counts).  Nothing runs after the
+      // synchronisation above, so they are cleared here and the next forward
+      // starts from the state a fresh plan has.
+      TRY(reset_control(p));
+      return MOE_ERR_TIMEOUT;
+    }
     return MOE_ERR_RANGE;
   }
+  return MOE_OK;
+}
+
+moe_status moe_debug_expire_wait(moe_plan p, int32_t limit_polls, void* stream) {
+  if (!p || limit_polls < 1 || limit_polls > (1 << 22)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  CUDA_TRY((cudaError_t)launch_expire_wait(p->nve + 4, p->err, p->router_done, p->counters[KIND_FRONT],
+                                           p->ctl + KIND_FRONT, p->route_ready,
+                                           (unsigned)limit_polls, stream));
   return MOE_OK;
 }
 

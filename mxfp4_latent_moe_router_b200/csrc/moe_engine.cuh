@@ -315,10 +315,12 @@ __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t
   }
 }
 
-// Bounded wait (about a second) until *flag != 0, with acquire semantics for
-// the calling thread; false (and an error bit) if it never is.
-__device__ __forceinline__ bool wait_flag(const int* flag, int* err, int err_bit, int lane) {
-  for (uint32_t i = 0; i < (1u << 22); ++i) {
+// Bounded wait (about a second at the default limit of 2^22 polls) until
+// *flag != 0, with acquire semantics for the calling thread; false (and an
+// error bit) if it never is.
+__device__ __forceinline__ bool wait_flag(const int* flag, int* err, int err_bit, int lane,
+                                          uint32_t limit = 1u << 22) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (ld_acquire(flag) != 0) return true;
     __nanosleep(256);
   }

@@ -112,6 +112,9 @@ extern "C" moe_status moe_route_noalloc(const void* x, const void* router_w,
   if (score_fn != MOE_SCORE_SOFTMAX && score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(router_w)) & 1)
     return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ids) | reinterpret_cast<uintptr_t>(weights) |
+       reinterpret_cast<uintptr_t>(router_bias)) & 3)
+    return MOE_ERR_INVALID_ARG;
   // sizes beyond the static scratch
   if (num_tokens > kStaticMaxTokens || num_experts > kStaticMaxExperts || top_k > 16)
     return MOE_ERR_UNSUPPORTED;
@@ -123,13 +126,25 @@ extern "C" moe_status moe_route_noalloc(const void* x, const void* router_w,
   float* logits = nullptr;
   moe_status st = scratch_for(dev, &logits);
   if (st != MOE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  static_router_logits<<<(num_experts + 63) / 64, 256, 0, s>>>(
-      static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(router_w), num_tokens, hidden,
-      num_experts, logits);
-  static_topk<<<(num_tokens + 7) / 8, 256, 0, s>>>(
-      logits, num_tokens, num_experts, top_k, score_fn,
-      score_fn == MOE_SCORE_SIGMOID ? router_bias : nullptr, renormalize, routed_scale, ids, weights);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  // each launch's own status (an error left behind by unrelated earlier work
+  // on this thread is neither reported nor cleared here)
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.gridDim = dim3((num_experts + 63) / 64);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, static_router_logits, static_cast<const uint16_t*>(x),
+                                     static_cast<const uint16_t*>(router_w), (int)num_tokens,
+                                     (int)hidden, (int)num_experts, logits);
+  if (e == cudaSuccess) {
+    cfg.gridDim = dim3((num_tokens + 7) / 8);
+    e = cudaLaunchKernelEx(&cfg, static_topk, static_cast<const float*>(logits), (int)num_tokens,
+                           (int)num_experts, (int)top_k, (int)score_fn,
+                           score_fn == MOE_SCORE_SIGMOID ? router_bias : nullptr, (int)renormalize,
+                           routed_scale, ids, weights);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // this call's launch error: report it, leave no trace behind
+    return MOE_ERR_CUDA;
+  }
   return MOE_OK;
 }

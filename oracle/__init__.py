@@ -73,6 +73,8 @@ def _load():
         lib.oracle_bf16_value.restype = ctypes.c_double
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = None
         _lib = lib
     return _lib
 
@@ -97,6 +99,11 @@ def _weights(w: dict):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads of the oracle's token loop (for timing; results do not change)."""
+    _load().oracle_set_threads(int(n))
 
 
 def e2m1_value(code: int) -> float:

@@ -199,6 +199,16 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads of the token loops from here on (timing only; results do not
+ * depend on it: every token is computed by one thread in the same order). */
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* Full block for B tokens.  x: bf16 [B][H]. */
 int oracle_forward(const oracle_cfg *cfg, const oracle_weights *w, const uint16_t *x,
                    int32_t B, oracle_outputs *o) {

@@ -233,13 +233,14 @@ def test_fused_launch_matches_multi_kernel_path(tiny, B, monkeypatch):
 
 
 # ---------------------------------------------------------------------------
-# full-size decode shapes (H=7168, L=2048, E=384, k=8, I=2048, I_s=2048)
+# full-size decode shapes (H=7168, L=2048, E=384, k=8, I=2048, I_s=2048), each
+# with the seeded weights the benchmark loads for it (instance 0 of that
+# workload), in a plan of 128 tokens as the benchmark creates
 
 
 @pytest.fixture(scope="module")
 def full_weights():
-    shape = synth.SHAPES["b1"]
-    return synth.make_weights(shape)
+    return synth.make_weights(synth.SHAPES["b1"], 0)
 
 
 @pytest.fixture(scope="module")
@@ -256,31 +257,40 @@ def test_b1_full_size(full_block):
     print("b1: max_rel %.3g mean_rel %.3g near-ties %s" % (mx, mn, near))
 
 
-@pytest.mark.parametrize("name,sample", [("b8", None), ("b64", [0, 9, 31, 63]),
-                                         ("b128", [0, 5, 64, 127])])
-def test_batched_full_size(full_block, full_weights, name, sample):
+# sampled tokens for the whole-block check at B = 64 and 128 (every token's
+# routing is checked): spread over the batch, both ends included
+SAMPLES = {"b8": None,
+           "b64": [0, 5, 9, 17, 22, 31, 38, 44, 50, 57, 61, 63],
+           "b128": [0, 5, 13, 22, 31, 40, 47, 64, 71, 80, 95, 101, 110, 119, 127]}
+
+
+@pytest.mark.parametrize("name", ["b8", "b64", "b128"])
+def test_batched_full_size_as_benchmarked(name):
     shape = synth.SHAPES[name]
-    w = full_weights
-    if shape.routing == "zipf":
-        # the speculative-verify shape: skewed popularity through the bias
-        w = dict(full_weights)
-        w["router_bias"] = synth.make_weights(synth.custom_shape(
-            "bias-only", 1, 32, 32, shape.num_experts, 1, 32, 0, synth.SCORE_SIGMOID,
-            routing="zipf", seed=shape.seed))["router_bias"]
-        blk = GpuBlock(shape, w, max_tokens=128)
-    else:
-        blk = full_block
-    x = synth.make_x(shape)
-    out = blk.run(x)
-    # routing of every token, with the cheap router-only oracle
-    r = oracle.route(shape, w, x)
-    ids, wts = blk.plan.routing(x.shape[0])
-    logits = blk.plan.fetch(moe.MOE_DBG_LOGITS, x.shape[0])
-    near = check_routing(shape, w, x, ids, wts, logits, r)
-    # whole block on sampled tokens
-    sel = np.arange(x.shape[0]) if sample is None else np.array(sample)
-    sel = np.array([b for b in sel if b not in near])
-    orc = oracle.forward(shape, w, x[sel], intermediates=False)
-    assert_close(bf16_to_f32(out[sel]), orc["out"], name + " out")
-    distinct = len(np.unique(ids))
-    print("%s: distinct experts %d, near ties %s" % (name, distinct, near))
+    w = synth.make_weights(shape, 0)
+    blk = GpuBlock(shape, w, max_tokens=128)
+    try:
+        x = synth.make_x(shape)
+        out = blk.run(x)
+        # routing of every token, with the cheap router-only oracle
+        r = oracle.route(shape, w, x)
+        ids, wts = blk.plan.routing(x.shape[0])
+        logits = blk.plan.fetch(moe.MOE_DBG_LOGITS, x.shape[0])
+        near = check_routing(shape, w, x, ids, wts, logits, r)
+        # whole block on sampled tokens
+        sample = SAMPLES[name]
+        sel = np.arange(x.shape[0]) if sample is None else np.array(sample)
+        sel = np.array([b for b in sel if b not in near])
+        orc = oracle.forward(shape, w, x[sel], intermediates=False)
+        mx, mn = assert_close(bf16_to_f32(out[sel]), orc["out"], name + " out")
+        distinct = len(np.unique(ids))
+        print("%s: distinct experts %d, near ties %s, max_rel %.3g mean_rel %.3g"
+              % (name, distinct, near, mx, mn))
+        if shape.routing == "zipf":
+            # the Zipf bias concentrates the tokens: far fewer experts than
+            # uniform routing would touch (about 358 of 384 at B = 128)
+            assert distinct < 200, distinct
+    finally:
+        blk.plan.close()
+        del blk
+        torch.cuda.empty_cache()
