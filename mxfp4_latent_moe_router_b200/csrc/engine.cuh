@@ -105,6 +105,9 @@ struct Params {
   int need_rb_edn, need_rb_sh;
   float* partials;
   int* err;
+  // ns a producer (consumer) warp sleeps after a failed poll of a ring
+  // barrier before polling again
+  int prod_sleep, cons_sleep;
 };
 
 // The single-launch path (few tokens): one Params per phase, all with the

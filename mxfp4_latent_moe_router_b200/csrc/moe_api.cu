@@ -110,6 +110,7 @@ struct moe_plan_s {
   int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
   bool use_pdl = true;
   int fail_alloc_after = -1;     // environment MOE_FAIL_ALLOC_AFTER (tests only)
+  int prod_sleep = 200, cons_sleep = 32;  // environment MOE_PROD_SLEEP / MOE_CONS_SLEEP (ns)
   // one launch per forward for B <= kFusedMaxTokens (environment MOE_FUSED=1);
   // off by default: measured slower than the four-launch chain at B = 1
   bool use_fused = false;
@@ -271,6 +272,8 @@ Params base_params(const moe_plan_s* p, int B) {
   q.router_done = p->router_done;
   q.route_ready = p->route_ready;
   q.err = p->err;
+  q.prod_sleep = p->prod_sleep;
+  q.cons_sleep = p->cons_sleep;
   q.C_lat = p->C_lat;
   q.KS = c.shared_inter;
   q.scratch_off = kScratchOff;
@@ -443,6 +446,8 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
   if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
   if (const char* e = getenv("MOE_FAIL_ALLOC_AFTER")) p->fail_alloc_after = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_PROD_SLEEP")) p->prod_sleep = std::max(0, std::min(2000, atoi(e)));
+  if (const char* e = getenv("MOE_CONS_SLEEP")) p->cons_sleep = std::max(0, std::min(2000, atoi(e)));
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
     return MOE_ERR_CUDA;

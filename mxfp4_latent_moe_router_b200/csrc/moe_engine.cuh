@@ -412,7 +412,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
         }
       }
       const long long tw0 = clock64();
-      if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, 200)) return;
+      if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, p.prod_sleep)) return;
       const long long tw1 = clock64();
       pw += tw1 - tw0;
       uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
@@ -463,7 +463,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
     tr[13] = (unsigned long long)nst;
   }
   // end marker
-  if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, 200)) return;
+  if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, p.prod_sleep)) return;
   if (lane == 0) {
     uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
     reinterpret_cast<Hdr*>(sb)->flags = HDR_END;
@@ -1351,7 +1351,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   int n_pieces = 0, n_fin = 0;
   long long c_wait = 0, c_comp = 0, c_end = 0, t_a = clock64();
   while (true) {
-    if (!mbar_wait_bounded(&full[stage], phase, p.err, ERR_WAIT_FULL)) break;
+    if (!mbar_wait_bounded(&full[stage], phase, p.err, ERR_WAIT_FULL, p.cons_sleep)) break;
     long long t_b = clock64();
     c_wait += t_b - t_a;
     uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;

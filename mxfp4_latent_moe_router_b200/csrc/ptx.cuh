@@ -38,14 +38,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait: poll, sleeping `sleep_ns` after each failed poll so a waiting
 // warp gives its scheduler's issue slots to the warps doing work; gives up
-// after 2^22 polls (about a second with the sleeps), sets bit `err_bit` of
-// *err and returns false.
+// after 2^22 polls or about a second of the global timer, whichever comes
+// first, sets bit `err_bit` of *err and returns false.
+__device__ __forceinline__ unsigned long long timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
                                                   int err_bit, uint32_t sleep_ns = 32) {
-  const uint32_t limit = 1u << 22;
-  for (uint32_t i = 0; i < limit; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = timer_ns();
+  for (uint32_t i = 1; i < (1u << 22); ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
-    __nanosleep(sleep_ns);
+    if ((i & 63) == 0 && timer_ns() - t0 > 1000000000ull) break;
   }
   atomicOr(err, 1 << err_bit);
   return false;
