@@ -48,6 +48,16 @@ struct Params {
   int piece_ctas;     // EGU/EDN: CTAs taking pieces (for the split-K choice)
   int split_cost;     // EGU/EDN: price of a split-K piece end, in stages
   int C_lat;          // TAIL: chunks covering L; chunks >= C_lat cover I_s
+  // TAIL, shared part first (0: one split over all C chunks): pieces over
+  // the I_s chunks come first in the schedule and need nothing from the
+  // routed experts (h_s is complete before this kernel starts), so CTAs that
+  // land while the expert kernels finish stream them at once; the latent
+  // pieces follow.  ppr_sh + ppr_lat == PPR pieces per row block.
+  int tail_split, ppr_lat, ppr_sh;
+  // EGU: the latent row blocks' finalisations count up here (release); the
+  // expert gate/up kernel reads z once it reaches RB_lat instead of waiting
+  // for the whole front grid (whose last CTAs stream shared-expert rows)
+  int* z_done;
   int RB_router;      // FRONT: leading row blocks holding router rows
   int RB_lat;         // FRONT: row blocks of the latent projection (after the router's);
                       // the shared expert's gate/up row blocks follow

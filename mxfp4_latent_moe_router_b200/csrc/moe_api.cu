@@ -111,6 +111,13 @@ struct moe_plan_s {
   bool use_pdl = true;
   int fail_alloc_after = -1;     // environment MOE_FAIL_ALLOC_AFTER (tests only)
   int prod_sleep = 200, cons_sleep = 32;  // environment MOE_PROD_SLEEP / MOE_CONS_SLEEP (ns)
+  // the tail streams its shared-expert part first, without waiting for the
+  // routed experts (environment MOE_TAIL_SPLIT=0 turns it off)
+  bool tail_split = true;
+  // expert gate/up waits for the latent row blocks' count, not the whole
+  // front grid (environment MOE_Z_FLAG=0 turns it off)
+  bool z_flag = true;
+  int* z_done = nullptr;
   // one launch per forward for B <= kFusedMaxTokens (environment MOE_FUSED=1);
   // off by default: measured slower than the four-launch chain at B = 1
   bool use_fused = false;
@@ -272,6 +279,8 @@ Params base_params(const moe_plan_s* p, int B) {
   q.router_done = p->router_done;
   q.route_ready = p->route_ready;
   q.err = p->err;
+  q.z_done = p->z_flag ? p->z_done : nullptr;
+  q.RB_lat = p->RB_lat;
   q.prod_sleep = p->prod_sleep;
   q.cons_sleep = p->cons_sleep;
   q.C_lat = p->C_lat;
@@ -323,6 +332,26 @@ int ppr_for(const moe_plan_s* p, int mats, int C, int ctas, int nt) {
 // for all of them: they get pieces of at most ~C/12 chunks.
 int router_ppr(int ppr, int C) { return std::max(1, std::min(C, std::max(ppr, 12))); }
 
+// The tail's pieces per row block with its shared part first: ppr pieces
+// split between the latent chunks and the shared-expert chunks in proportion
+// (at least one each, at most one chunk a piece); without a shared expert,
+// or with the split off, one split over all chunks (ppr_sh = 0).
+struct TailSplit {
+  int ppr_lat, ppr_sh;
+};
+TailSplit tail_split_for(const moe_plan_s* p, int ppr) {
+  const int C = p->g[KIND_TAIL].C, C_lat = p->C_lat, C_sh = C - p->C_lat;
+  if (!p->tail_split || C_sh <= 0) return {ppr, 0};
+  int lat = (int)std::lround((double)ppr * C_lat / C);
+  lat = std::max(1, std::min(C_lat, lat));
+  const int sh = std::max(1, std::min(C_sh, ppr - lat));
+  return {lat, sh};
+}
+int tail_ppr(const moe_plan_s* p, int ppr) {
+  const TailSplit t = tail_split_for(p, ppr);
+  return t.ppr_lat + t.ppr_sh;
+}
+
 // largest number of partial-sum floats a kind can need for B <= maxB
 size_t partial_floats(const moe_plan_s* p, int kind) {
   size_t best = 0;
@@ -338,7 +367,7 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      pieces = (size_t)passes * g.RB * ppr_for(p, g.RB * passes, g.C, f.tail_grid, nt);
+      pieces = (size_t)passes * g.RB * tail_ppr(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, nt));
     } else {
       nt = f.nt_e;
       // the split depends on the routing: take the largest over every
@@ -447,6 +476,8 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
   if (const char* e = getenv("MOE_FAIL_ALLOC_AFTER")) p->fail_alloc_after = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_PROD_SLEEP")) p->prod_sleep = std::max(0, std::min(2000, atoi(e)));
+  if (const char* e = getenv("MOE_TAIL_SPLIT")) p->tail_split = atoi(e) != 0;
+  if (const char* e = getenv("MOE_Z_FLAG")) p->z_flag = atoi(e) != 0;
   if (const char* e = getenv("MOE_CONS_SLEEP")) p->cons_sleep = std::max(0, std::min(2000, atoi(e)));
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
@@ -500,6 +531,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->err = p->nve + 2;
   p->done = p->nve + 8;
   p->route_ready = p->nve + 3;
+  p->z_done = p->nve + 5;  // (nve + 4: a flag nothing sets, for the expiring-wait test)
   p->ctl = reinterpret_cast<Ctl*>((uint8_t*)v + 1024);
   CUDA_TRY(cudaMemset(v, 0, kControlBytes));
   const int cnt_n[KIND_COUNT] = {fr.RB, p->ve_max * eg.RB, p->ve_max * ed.RB, maxB * tl.RB};
@@ -576,6 +608,7 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
     q.stage_off = stage_off;
     q.table_off = kStageOff;
     q.ctl = p->ctl + kFused;
+    q.z_done = nullptr;  // the single launch counts phases in `done`
     q.trace = p->trace ? p->trace + (size_t)kFused * 2 * p->num_sms * 24 : nullptr;
     q.done = p->done;
     q.need_rb_edn = p->g[KIND_EDN].RB;
@@ -669,7 +702,11 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       q.res_k = res_k;
     }
     const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-    q.PPR = ppr_for(p, q.RB * passes, q.C, f.tail_grid, f.nt_tail);
+    const TailSplit ts = tail_split_for(p, ppr_for(p, q.RB * passes, q.C, f.tail_grid, f.nt_tail));
+    q.PPR = ts.ppr_lat + ts.ppr_sh;
+    q.tail_split = ts.ppr_sh > 0;
+    q.ppr_lat = ts.ppr_lat;
+    q.ppr_sh = ts.ppr_sh;
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
     CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, p->use_pdl));
     if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][1], s));
@@ -1052,7 +1089,7 @@ moe_status moe_debug_geometry(const moe_config* cfg, int32_t num_sms, int32_t nu
           (B * resident_stride(res_k) <= kResidentMax) ? B * resident_stride(res_k) : 0;
       sm = smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * K, res_bytes);
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      const int ppr = ppr_for(p, g.RB * passes, g.C, f.tail_grid, f.nt_tail);
+      const int ppr = tail_ppr(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, f.nt_tail));
       o.grid = f.tail_grid;
       o.ctas_per_sm = 1;
       o.token_tiles = f.nt_tail;

@@ -63,7 +63,9 @@ struct Hdr {
   int piece, v, rb;
   int chunk, nb, ntok, tok0;
   int expert, ppr, act_bytes;
-  int p0;  // first piece of this row block (its partial sums are p0 .. p0 + ppr - 1)
+  int p0;  // first partial slot of this row block (its partial sums are p0 .. p0 + ppr - 1)
+  int c_first, c_last;  // chunks of this piece
+  int dep;              // 1: its activations need the kernel's dependency resolved
   // fused single-launch path: this piece's kind, and on its last stage the
   // kind of the piece the producer streams next (-1: none)
   int kind, next_kind;
@@ -104,7 +106,7 @@ __device__ __forceinline__ Space make_space(const Params& p, int V = 0) {
   } else if (KIND == KIND_TAIL) {
     const int passes = (p.B + p.tg - 1) / p.tg;
     s.ppr = p.PPR;
-    s.total = passes * p.RB * p.PPR;
+    s.total = passes * p.RB * p.PPR;  // (split or not: ppr_sh + ppr_lat == PPR)
   } else {
     // FRONT: the router row blocks come first, in pieces of their own size
     s.ppr = p.PPR;
@@ -143,6 +145,39 @@ __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, i
                                              const VExpert* ve_tab) {
   h.piece = piece;
   h.expert = 0;
+  h.dep = 1;
+  if (KIND == KIND_TAIL && p.tail_split) {
+    // shared-expert pieces of every (pass, row block) first, then the latent
+    // ones; a row block's partial slots stay contiguous (latent j, then
+    // shared ppr_lat + j) so the finalising sum keeps one fixed order
+    const int n_sh = sp.total / p.PPR * p.ppr_sh;
+    int q, pp, cb, cn, slot0;
+    if (piece < n_sh) {
+      q = piece / p.ppr_sh;
+      pp = piece % p.ppr_sh;
+      cb = p.C_lat;
+      cn = p.C - p.C_lat;
+      slot0 = p.ppr_lat;
+      h.dep = 0;
+    } else {
+      q = (piece - n_sh) / p.ppr_lat;
+      pp = (piece - n_sh) % p.ppr_lat;
+      cb = 0;
+      cn = p.C_lat;
+      slot0 = 0;
+    }
+    const int pieces_here = h.dep ? p.ppr_lat : p.ppr_sh;
+    h.v = q / p.RB;
+    h.rb = q % p.RB;
+    h.ppr = p.PPR;
+    h.p0 = q * p.PPR;
+    h.piece = h.p0 + slot0 + pp;
+    h.c_first = cb + (pp * cn) / pieces_here;
+    h.c_last = cb + ((pp + 1) * cn) / pieces_here;
+    h.tok0 = h.v * p.tg;
+    h.ntok = min(p.tg, p.B - h.tok0);
+    return;
+  }
   const int nr = KIND == KIND_FRONT ? p.RB_router * p.PPR_r : 0;
   if (piece < nr) {  // router row blocks (smaller pieces, so the logits are summed early)
     h.v = 0;
@@ -172,6 +207,9 @@ __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, i
     h.tok0 = ve.start;
     h.ntok = ve.count;
   }
+  const int pr = h.piece - h.p0;
+  h.c_first = (pr * p.C) / h.ppr;
+  h.c_last = ((pr + 1) * p.C) / h.ppr;
 }
 
 // Per chunk: flags, block count and activation bytes.
@@ -339,6 +377,29 @@ __device__ __forceinline__ bool wait_count(const int* counter, int target, int* 
   return false;
 }
 
+// The producer's dependency: what its activation copies must wait for.
+//   FRONT, EDN, TAIL: the previous kernel of the stream, complete
+//                     (griddepcontrol.wait);
+//   EGU with z_done:  only the latent row blocks of the front kernel (z), by
+//                     their release count -- the front's last CTAs stream
+//                     shared-expert rows this kernel never reads.  Its
+//                     dependents may launch at once; each CTA still waits for
+//                     the front grid before it exits, so that this grid's
+//                     completion implies the front's (the tail reads h_s and
+//                     the combine weights after waiting only for its own
+//                     predecessor).
+template <int KIND>
+__device__ __forceinline__ bool producer_dep_wait(const Params& p, int lane) {
+  if (KIND == KIND_EGU && p.z_done) {
+    const bool ok = wait_count(p.z_done, p.RB_lat, p.err, lane);
+    fence_proxy_async_global();  // the z records are read by bulk copies
+    return ok;
+  }
+  pdl_wait();
+  pdl_trigger();
+  return true;
+}
+
 template <int KIND>
 __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t* tables,
                          uint64_t* full, uint64_t* empty, int lane) {
@@ -346,9 +407,15 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   uint32_t ephase = 1;  // empty barriers start "released"
   Space sp;
   // every kind streams up to one ring of weight tiles before its dependency
-  // resolves (stages filled with weights only, their activations pending)
-  int prefetched = 0;
+  // resolves (stages filled with weights only, their activations pending:
+  // always the last `prefetched` stages issued, from ring slot pend_first on)
+  int prefetched = 0, pend_first = 0;
   bool waited = false;
+  // The tail with its shared part first: those pieces need no dependency, so
+  // CTAs take pieces (and keep a grab in flight) from the start; the first
+  // latent piece they hold waits for it.
+  const bool free_start = KIND == KIND_TAIL && p.tail_split;
+  if (KIND == KIND_EGU && p.z_done) pdl_trigger();
   // routing tables in shared memory: the per-stage lookups then cost no
   // global round trip (they are visible to the consumers through the first
   // full-barrier completion).  The whole capacity is copied so that these
@@ -376,19 +443,32 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   if (!route_ok) sp.total = 0;  // no pieces: straight to the end marker
   __syncwarp();
 
+  // Resolve the dependency and issue the pending stages' activations.
+  auto resolve = [&]() {
+    if (!producer_dep_wait<KIND>(p, lane)) sp.total = 0;  // gave up: no further pieces
+    waited = true;
+    for (int j = 0; j < prefetched; ++j) {
+      const int s = (pend_first + j) % p.nstages;
+      uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
+      const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
+      issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
+    }
+    prefetched = 0;
+  };
+
   // every CTA starts on piece blockIdx.x (no round trip before the first
   // tile); later pieces come from the cursor, offset by the number of
   // piece-taking CTAs.  Lane 0 keeps one grab in flight and reads its result
-  // one piece later -- but only once the dependency has resolved: CTAs that
-  // land early (while the previous kernel's last CTAs still run) would
-  // otherwise take several pieces each before the late ones can start, and
-  // finish last.
+  // one piece later -- but only once the dependency has resolved (or from the
+  // start where the first pieces need none): CTAs that land early (while the
+  // previous kernel's last CTAs still run) would otherwise take several
+  // pieces each before the late ones can start, and finish last.
   long long pw = 0, pi = 0, nst = 0;
   int grabbed = 0;
   bool in_flight = false;
   const int workers = (int)gridDim.x - (KIND == KIND_FRONT ? p.route_cta : 0);
   int piece = blockIdx.x;
-  if (waited && piece < sp.total) {
+  if ((waited || free_start) && piece < sp.total) {
     if (lane == 0) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
     in_flight = true;
   }
@@ -396,21 +476,11 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
     if (piece >= sp.total) break;
     Hdr ph;
     piece_header<KIND>(p, sp, piece, ph, ve_tab);
-    const int pr = piece - ph.p0;
-    const int c_first = (pr * p.C) / ph.ppr;
-    const int c_last = ((pr + 1) * p.C) / ph.ppr;
+    const int c_first = ph.c_first, c_last = ph.c_last;
     for (int c = c_first; c < c_last; ++c) {
-      // before the dependency resolves, fill at most one ring of weight-only stages
-      if (!waited && prefetched == p.nstages) {
-        pdl_wait();
-        pdl_trigger();
-        waited = true;
-        for (int s = 0; s < prefetched; ++s) {
-          uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
-          const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
-          issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
-        }
-      }
+      // before the dependency resolves, fill at most one ring of weight-only
+      // stages: the slot to reuse next would otherwise be a pending one
+      if (!waited && prefetched == p.nstages) resolve();
       const long long tw0 = clock64();
       if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, p.prod_sleep)) return;
       const long long tw1 = clock64();
@@ -420,10 +490,12 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       chunk_header<KIND>(p, c, c_first, c_last, h);
       if (lane == 0) stage_begin<KIND>(p, h, sb, &full[stage]);
       __syncwarp();
-      if (waited)
+      if (waited || !h.dep) {
         issue_act<KIND>(p, h, sb + p.act_off, &full[stage], lane, slot_tab);
-      else
+      } else {
+        if (prefetched == 0) pend_first = stage;
         ++prefetched;
+      }
       if (++stage == p.nstages) {
         stage = 0;
         ephase ^= 1;
@@ -431,31 +503,14 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       pi += clock64() - tw1;
       ++nst;
     }
-    if (!waited) {
-      // first piece issued and still no dependency: stop prefetching here
-      pdl_wait();
-      pdl_trigger();
-      waited = true;
-      for (int s = 0; s < prefetched; ++s) {
-        uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
-        const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
-        issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
-      }
-    }
+    // a piece issued with pending activations: stop prefetching here
+    if (!waited && (prefetched > 0 || !free_start)) resolve();
     if (!in_flight && lane == 0) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
     piece = __shfl_sync(0xffffffffu, grabbed, 0);
     in_flight = piece < sp.total;
     if (lane == 0 && in_flight) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
   }
-  if (!waited) {
-    pdl_wait();
-    pdl_trigger();
-    for (int s = 0; s < prefetched; ++s) {
-      uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
-      const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
-      issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
-    }
-  }
+  if (!waited && (prefetched > 0 || !free_start)) resolve();
   if (p.trace && lane == 0) {
     unsigned long long* tr = p.trace + (size_t)blockIdx.x * kTraceStride;
     tr[11] = (unsigned long long)pw;
@@ -653,11 +708,15 @@ __device__ __forceinline__ void mma_mx(const Params& p, const Hdr& h, const uint
 // TAIL, few tokens: form every token's whole activation once per CTA.  Token
 // b's record holds bf16 hi values for k in [0, res_k), then the lo parts.
 // k < C_lat*64 is the combine c = sum_j w_j y_j (zero past L); the rest is h_s.
-__device__ __forceinline__ void build_resident(const Params& p, uint8_t* res, int tid) {
+// Only the groups of eight k in [kbeg, kend) are formed (multiples of 8): the
+// h_s part can be built before the routed experts finish, the combine after.
+__device__ __forceinline__ void build_resident(const Params& p, uint8_t* res, int tid, int kbeg,
+                                               int kend) {
   const int K = p.topk, KR = p.res_k, klat = p.C_lat * 64;
-  const int groups = p.B * (KR / 8);
+  const int n8 = (kend - kbeg) / 8;
+  const int groups = p.B * n8;
   for (int gi = tid; gi < groups; gi += kConsumerThreads) {
-    const int b = gi / (KR / 8), k0 = (gi % (KR / 8)) * 8;
+    const int b = gi / n8, k0 = kbeg + (gi % n8) * 8;
     float v[8];
     if (k0 < klat) {
       // K <= 16: compile-time slots keep everything in registers, loads first
@@ -919,6 +978,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
     store_f16mx<NT, 2>(val, warp, lane, 2, p.B, reinterpret_cast<float*>(scratch), rec, idx,
                        l0 < p.L, l0 + 8 < p.L);  // ends with a barrier
     if (p.done && tid == 0) red_release_add(p.done + 0, 1);
+    // every thread's records precede the release (barrier cumulativity)
+    if (p.z_done && tid == 0) red_release_add(p.z_done, 1);
   } else if (KIND == KIND_FRONT) {
     // shared expert gate/up rows (64 gate + 64 up per block) -> h_s
     const int i = 64 * (h.rb - p.RB_router - p.RB_lat) + 8 * warp + g;
@@ -1334,18 +1395,43 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   int ticket = 0;
   int* tflag = sm_flag + 4;  // two alternating slots
   int tslot = 0;
-  // activations, routing tables and partial sums of the previous kernel are
+  // Activations, routing tables and partial sums of the previous kernel are
   // read only after the dependency has resolved; the next kernel may then be
-  // scheduled (it cannot overtake this one's own predecessor)
-  pdl_wait();
-  pdl_trigger();
-  // Past this wait every earlier kernel of the forward has finished, so no
-  // reader of the routing flag is left: clear it for the next forward.
-  if (KIND == KIND_TAIL && blockIdx.x == 0 && tid == 0) *p.route_ready = 0;
+  // scheduled (it cannot overtake this one's own predecessor).  Two kinds
+  // wait elsewhere:
+  //   - the tail with its shared part first waits when its first latent
+  //     stage arrives (the shared part reads h_s, complete before this
+  //     kernel starts, and the stages the producer filled);
+  //   - the expert gate/up kernel with a z count reads nothing of the front
+  //     kernel but what its producer copies after that count; it waits for
+  //     the front grid only before exiting.
+  const bool lazy = KIND == KIND_TAIL && p.tail_split;
+  const bool late = KIND == KIND_EGU && p.z_done;
   uint8_t* res = stage_base - p.stage_off + p.res_off;  // shared-memory base + offset
-  if (KIND == KIND_TAIL && p.res_off) {
-    build_resident(p, res, tid);
-    named_sync(1, kConsumerThreads);
+  const int klat = p.C_lat * 64;
+  // Past the wait every earlier kernel of the forward has finished, so no
+  // reader of the routing flag or of the z count is left: clear both for the
+  // next forward.
+  auto tail_dep = [&](int kbeg, int kend) {
+    pdl_wait();
+    pdl_trigger();
+    if (KIND == KIND_TAIL && tid == 0) {
+      *p.route_ready = 0;
+      if (p.z_done) *p.z_done = 0;
+    }
+    if (KIND == KIND_TAIL && p.res_off) {
+      build_resident(p, res, tid, kbeg, kend);
+      named_sync(1, kConsumerThreads);
+    }
+  };
+  bool dep_done = !lazy;
+  if (lazy) {
+    if (p.res_off) {
+      build_resident(p, res, tid, klat, p.res_k);
+      named_sync(1, kConsumerThreads);
+    }
+  } else if (!late) {
+    tail_dep(0, p.res_k);
   }
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
   int n_pieces = 0, n_fin = 0;
@@ -1358,6 +1444,10 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
     const Hdr h = *reinterpret_cast<const Hdr*>(sb);
     if (tr && tid == 0 && n_pieces == 0 && (h.flags & HDR_FIRST)) tr[6] = global_ns();
     if (h.flags & HDR_END) break;
+    if (lazy && !dep_done && h.dep) {
+      tail_dep(0, klat);  // the first latent stage: y, and the combine, need the expert phases
+      dep_done = true;
+    }
     if (h.flags & HDR_FIRST) {
       zero_acc(acc);
       zero_acc(acc2);
@@ -1450,6 +1540,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       finalize<KIND, NT>(p, pend_h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
     }
   }
+  if (late) pdl_wait();  // this grid completes only after the front grid
   if (tr && tid == 0) {
     tr[2] = (unsigned long long)n_pieces;
     tr[3] = (unsigned long long)n_fin;

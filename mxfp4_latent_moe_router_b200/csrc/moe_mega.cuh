@@ -293,7 +293,7 @@ __device__ __forceinline__ bool mega_piece(const Params& p, MegaCons& cs, uint8_
       wait_count(p.done + 1, p.need_rb_sh, p.err, lane);
     }
     named_sync(1, kConsumerThreads);
-    build_resident(p, res, tid);
+    build_resident(p, res, tid, 0, p.res_k);
     named_sync(1, kConsumerThreads);
     cs.res_built = true;
   }

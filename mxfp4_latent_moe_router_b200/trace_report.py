@@ -8,8 +8,11 @@ module turns that array into one summary per kernel.
 
     MOE_TRACE=1 python -m mxfp4_latent_moe_router_b200.trace_report --workload b64
 
-The forward is timed on its own (no other work on the GPU), after three
-warm-up forwards, so the figures describe a single step, not a steady stream.
+By default the forward is timed on its own (no other work on the GPU), after
+three warm-up forwards, so the figures describe a single step, not a steady
+stream.  With --steady the traced forward is the last of a CUDA graph of ten
+back to back, so its first kernel overlaps the previous forward's last one as
+in the benchmark (times are still relative to its own first CTA start).
 """
 from __future__ import annotations
 
@@ -96,6 +99,8 @@ def format_summary(rows: list[dict]) -> str:
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--workload", default="b1")
+    ap.add_argument("--steady", action="store_true",
+                    help="trace the last of ten forwards replayed back to back from a CUDA graph")
     args = ap.parse_args(argv)
     if not os.environ.get("MOE_TRACE"):
         raise SystemExit("set MOE_TRACE=1: the plan keeps the timeline only then")
@@ -115,7 +120,19 @@ def main(argv=None) -> int:
         for _ in range(3):
             plan.forward(x, out)
         torch.cuda.synchronize()
-        plan.forward(x, out)
+        if args.steady:
+            s = torch.cuda.Stream()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for _ in range(10):
+                        plan.forward(x, out, stream=s)
+                g.replay()
+                g.replay()
+            s.synchronize()
+            del g
+        else:
+            plan.forward(x, out)
         torch.cuda.synchronize()
         info = plan.info()
         tr = moe.moe_debug_trace(plan.handle, info.num_sms)
