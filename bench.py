@@ -271,6 +271,10 @@ def _kernel_bytes(shape, distinct):
           "expert_down": distinct * per_expert_dn,
           "latent_tail": 2 * L * H + 2 * Is * H}
     kb["fused_block"] = sum(kb.values())  # one launch streams them all
+    # the side lane: the shared expert's gate/up rows and its down projection;
+    # the routed lane's front and tail then stream the rest
+    kb["shared_front"] = 2 * H * 2 * Is
+    kb["shared_tail"] = 2 * Is * H
     return kb
 
 
@@ -292,7 +296,7 @@ def measure_workload(name, args, rank, local, dist, headline):
         w_np, dw = _device_instance(shape, inst, torch)
         if inst == 0:
             host_w0 = w_np
-        p = moe.MoePlan(moe.config_from_shape(shape), device=local)
+        p = moe.MoePlan(moe.config_from_shape(shape, shared_sms=args.shared_sms), device=local)
         p.load(dw, stream)
         del dw
         plans.append(p)
@@ -399,6 +403,9 @@ def measure_workload(name, args, rank, local, dist, headline):
         cnt += c
     kern_us = {n: tot[n] * 1e3 / max(cnt, 1) for n in tot if tot[n] > 0}
     kern_bytes = _kernel_bytes(shape, mean_distinct)
+    if "shared_front" in kern_us:
+        kern_bytes["dense_front"] -= kern_bytes["shared_front"]
+        kern_bytes["latent_tail"] -= kern_bytes["shared_tail"]
     dom = max(kern_us, key=lambda n: kern_us[n])
     traffic = _measured_traffic(name)
     ach = kern_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9 if kern_us[dom] > 0 else 0.0
@@ -555,6 +562,9 @@ def main():
                     help="resident weight instances rotated per step (4 keeps every step out of L2)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-check", action="store_true")
+    ap.add_argument("--shared-sms", type=int, default=0,
+                    help="side lane for the shared expert at B <= 4: n > 0 = on with n CTAs per "
+                         "kernel; 0 (the measured best) or -1 = off")
     ap.add_argument("--only", dest="all_workloads", action="store_false",
                     help="measure only --workload (default at N=1: every workload, the "
                          "chosen one as the headline)")

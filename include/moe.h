@@ -76,6 +76,14 @@ typedef struct moe_config {
   int32_t score_fn;     /* MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID */
   int32_t renormalize;  /* 1: combine weights divided by their sum over the k chosen */
   float routed_scale;   /* factor applied to every combine weight (1.0 = none) */
+  int32_t shared_sms;   /* the shared expert as a side lane for forwards of at
+                           most 4 tokens: n > 0 = its gate/up rows and its down
+                           projection run as two kernels of n CTAs each on a
+                           side stream, sharing the SMs with the routed
+                           experts' chain; 0 (the measured best) or -1 = no
+                           side lane: its gate/up rows ride the front pass and
+                           its down projection leads the tail.  Ignored when
+                           shared_inter == 0. */
 } moe_config;
 
 /*
@@ -126,7 +134,8 @@ typedef struct moe_plan_info {
   int64_t workspace_bytes;  /* library-owned activations, routing metadata, partial sums */
   int64_t dense_weight_bytes;      /* bf16 bytes one forward streams regardless of routing */
   int64_t expert_weight_bytes;     /* MXFP4 bytes of one expert (gate/up + down, codes + scales) */
-  int32_t kernels_per_forward;     /* launches one moe_forward of max_tokens tokens makes */
+  int32_t kernels_per_forward;     /* launches one moe_forward of max_tokens tokens makes
+                                      (six with the side lane's two) */
 } moe_plan_info;
 
 /*
@@ -147,6 +156,15 @@ typedef struct moe_plan_info {
  *                           2 at one token tile)
  *   MOE_EXPERT_SMALL_MAX_B=n  largest B with 8-token virtual experts (default
  *                           128; above it, 32-token groups)
+ *   MOE_SIDE_LANE=0         no side lane, whatever shared_sms says
+ *   MOE_TAIL_SPLIT=0        the tail's shared-expert part is not scheduled first
+ *   MOE_Z_FLAG=0            expert gate/up waits for the whole front kernel
+ *   MOE_PREFETCH_MB=n       L2 prefetch of the chosen experts' tiles by the
+ *                           routing CTA once they are known, at most n MB
+ *                           (default 0 = off: one SM issues them too slowly)
+ *   MOE_DIRECT_ROUTE=0      the routing CTA waits for summed logits also at
+ *                           B <= 4 (default: it sums the router partials itself)
+ *   MOE_PROD_SLEEP, MOE_CONS_SLEEP  ns a ring warp sleeps between barrier polls
  *   MOE_FAIL_ALLOC_AFTER=n  fail this plan's (n+1)-th device allocation with
  *                           MOE_ERR_OOM (tests of the error path; everything
  *                           allocated before it is released)
@@ -222,10 +240,12 @@ MOE_API moe_status moe_get_plan_info(moe_plan p, moe_plan_info *info);
  * each of its kernels with CUDA events on the stream that kernel runs on and
  * waits for them before returning (so profiled forwards are synchronous and
  * must not be captured into a graph).  moe_get_profile writes the accumulated
- * milliseconds per kernel to ms[0..4] -- {dense front (router, latent, shared
- * gate/up, top-k), expert gate/up, expert down, latent tail, fused single
- * launch}; a forward of at most 8 tokens runs only the last, larger ones the
- * first four -- and the number of profiled forwards to *count, then clears
+ * milliseconds per kernel to ms[0..6] -- {dense front (router, latent
+ * [, shared gate/up], top-k), expert gate/up, expert down, latent tail, fused
+ * single launch, side-lane front (shared gate/up), side-lane tail (shared
+ * down)}; the fused launch (MOE_FUSED=1, at most 8 tokens) replaces the
+ * first four, the side lane (at most 4 tokens, shared_sms > 0) adds the
+ * last two -- and the number of profiled forwards to *count, then clears
  * both.
  */
 MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
@@ -233,7 +253,7 @@ MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
 /*
  * Per-CTA timeline of the most recent forward, for measurement only; exists
  * when the plan was created with the environment variable MOE_TRACE set
- * (else MOE_ERR_UNSUPPORTED).  host receives count = 5 * num_sms * 24 uint64:
+ * (else MOE_ERR_UNSUPPORTED).  host receives count = 7 * num_sms * 24 uint64:
  * for launch slot k (as in moe_get_profile) and CTA c, the 24 values at
  * (k * num_sms + c) * 24 are (ns from globaltimer, cycles from clock64):
  *   0 start ns, 1 end ns, 2 pieces, 3 finalizes, 4/5 top-k start/end ns (the
@@ -254,7 +274,9 @@ MOE_API moe_status moe_get_profile(moe_plan p, float *ms, int32_t *count);
 
 /* Launch geometry of one kernel kind, as moe_forward would choose it. */
 typedef struct moe_geometry {
-  int32_t kind;               /* 0 dense front, 1 expert gate/up, 2 expert down, 3 latent tail */
+  int32_t kind;               /* 0 dense front, 1 expert gate/up, 2 expert down, 3 latent tail,
+                                 4 side-lane front (shared gate/up), 5 side-lane tail
+                                 (shared down) */
   int32_t grid;               /* CTAs launched */
   int32_t ctas_per_sm;        /* 1, or 2 for the one-tile expert kernels */
   int32_t token_tiles;        /* 8-column token tiles the kernel is instantiated for */
@@ -271,7 +293,8 @@ typedef struct moe_geometry {
 
 /*
  * The geometry moe_forward(num_tokens) would use on a device with num_sms
- * SMs, for the 4 kinds (out[0..3]), with the default settings (environment
+ * SMs, for the 6 kinds (out[0..5]; the side lane's two have grid 0 when the
+ * forward has no side lane), with the default settings (environment
  * variables are not read).  Host only: needs no device and allocates no
  * device memory, so the planner can be checked anywhere.
  * Errors: INVALID_ARG (null, bad shape, num_sms < 2, num_tokens outside

@@ -32,7 +32,8 @@ ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forwar
 # streams the router, latent-projection and shared-expert gate/up rows and
 # runs top-k), then the single fused launch that MOE_FUSED=1 selects for
 # forwards of at most 8 tokens
-KERNEL_NAMES = ["dense_front", "expert_gate_up", "expert_down", "latent_tail", "fused_block"]
+KERNEL_NAMES = ["dense_front", "expert_gate_up", "expert_down", "latent_tail", "fused_block",
+                "shared_front", "shared_tail"]
 
 
 class MoeError(RuntimeError):
@@ -46,7 +47,8 @@ class moe_config(ctypes.Structure):
                 ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("expert_inter", ctypes.c_int32), ("shared_inter", ctypes.c_int32),
                 ("max_tokens", ctypes.c_int32), ("score_fn", ctypes.c_int32),
-                ("renormalize", ctypes.c_int32), ("routed_scale", ctypes.c_float)]
+                ("renormalize", ctypes.c_int32), ("routed_scale", ctypes.c_float),
+                ("shared_sms", ctypes.c_int32)]
 
 
 class moe_weights(ctypes.Structure):
@@ -208,7 +210,7 @@ def moe_route_noalloc(x, router_w, router_bias, num_tokens: int, hidden: int, nu
 
 
 def moe_debug_trace(plan: int, num_sms: int):
-    """Per-CTA timeline of the last forward: uint64 array [5 launch slots][num_sms][24]."""
+    """Per-CTA timeline of the last forward: uint64 array [7 launch slots][num_sms][24]."""
     import numpy as np
     a = np.zeros((len(KERNEL_NAMES), num_sms, 24), np.uint64)
     _check(load_library().moe_debug_trace(plan, a.ctypes.data, a.size), "moe_debug_trace")
@@ -218,7 +220,7 @@ def moe_debug_trace(plan: int, num_sms: int):
 def moe_debug_geometry(cfg: moe_config, num_sms: int, num_tokens: int) -> list:
     """Launch geometry of the four kernels for a forward of num_tokens tokens on
     num_sms SMs, with default settings (host only: no device needed)."""
-    out = (moe_geometry * 4)()
+    out = (moe_geometry * 6)()
     _check(load_library().moe_debug_geometry(ctypes.byref(cfg), num_sms, num_tokens, out),
            "moe_debug_geometry")
     return [{f[0]: getattr(g, f[0]) for f in moe_geometry._fields_} for g in out]
@@ -231,11 +233,11 @@ def moe_plan_destroy(plan: int) -> None:
 
 # ---- convenience wrapper ---------------------------------------------------
 
-def config_from_shape(shape, max_tokens: int | None = None) -> moe_config:
+def config_from_shape(shape, max_tokens: int | None = None, shared_sms: int = 0) -> moe_config:
     return moe_config(shape.hidden, shape.latent, shape.num_experts, shape.top_k,
                       shape.expert_inter, shape.shared_inter,
                       shape.tokens if max_tokens is None else max_tokens, shape.score_fn,
-                      shape.renormalize, float(shape.routed_scale))
+                      shape.renormalize, float(shape.routed_scale), shared_sms)
 
 
 def weights_to_device(w: dict, device: str = "cuda"):

@@ -54,6 +54,36 @@ struct Params {
   // land while the expert kernels finish stream them at once; the latent
   // pieces follow.  ppr_sh + ppr_lat == PPR pieces per row block.
   int tail_split, ppr_lat, ppr_sh;
+  // TAIL, one lane of two (the shared expert on a side stream): 0 every
+  // piece, 1 the latent pieces only (the routed lane), 2 the shared-expert
+  // pieces only (the side lane).  Both lanes share the row blocks' tickets and
+  // partial-sum slots, so whichever finishes a row block last writes it.
+  int tail_part;
+  // FRONT: the row blocks this launch streams, [rb_lo, rb_hi): everything
+  // (0, RB), or one lane -- router + latent rows (the routed lane, with the
+  // routing CTA) or the shared expert's gate/up rows (the side lane)
+  int rb_lo, rb_hi;
+  // TAIL: first k of the resident activation (its record holds k in
+  // [res_k0, res_k0 + res_k)); a lane keeps only its own part
+  int res_k0;
+  // host side: launch the instantiation compiled for two CTAs per SM (at most
+  // 112 registers a thread), so that a CTA of the other lane fits beside it
+  int half_sm;
+  // FRONT, routing CTA: once the experts are chosen it asks L2 for their
+  // packed gate/up and down tiles (the kernels that stream them start a few
+  // round trips later), for the chosen experts whose first virtual expert
+  // index is below pf_ves; 0 = none
+  const uint8_t* pf_egu;
+  const uint8_t* pf_edn;
+  long long pf_egu_bytes, pf_edn_bytes;  // per expert
+  int pf_ves;
+  // FRONT, few tokens: the router pieces write their partial sums here (no
+  // tickets, no finalisation) and the routing CTA sums them itself, polling
+  // on the data: every element starts as the 0xFFFFFFFF pattern, which no
+  // sum takes, and the routing CTA restores it after reading.  That is one
+  // round trip from the last router piece to the selection instead of four
+  // (ticket, partial sums, count, logits).  Null: the usual split-K finish.
+  float* rpart;
   // EGU: the latent row blocks' finalisations count up here (release); the
   // expert gate/up kernel reads z once it reaches RB_lat instead of waiting
   // for the whole front grid (whose last CTAs stream shared-expert rows)

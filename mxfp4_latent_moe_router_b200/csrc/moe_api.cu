@@ -25,10 +25,22 @@ constexpr int kScratchOff = 1024;
 constexpr int kScratchBytes = 20480;
 constexpr int kStageOff = kScratchOff + kScratchBytes;
 constexpr int kHdr = 128;
-// per-kind slots (scheduling state, profile, trace) plus one for the fused
-// single launch, which uses slot KIND_COUNT
-constexpr int kSlots = KIND_COUNT + 1;
+// per-kind slots (scheduling state, profile, trace), one for the fused
+// single launch, and two for the side lane's kernels (the shared expert's
+// gate/up rows and its down projection, on the side stream)
+constexpr int kSlots = KIND_COUNT + 3;
 constexpr int kFused = KIND_COUNT;
+constexpr int kSideFront = KIND_COUNT + 1;
+constexpr int kSideTail = KIND_COUNT + 2;
+// largest batch that runs the shared expert as a side lane (a second stream
+// whose CTAs share the SMs with the routed chain's): every kernel of either
+// lane then fits in half an SM's shared memory
+constexpr int kSideMaxTokens = 4;
+// largest batch whose routing CTA sums the router pieces' partials itself
+constexpr int kDirectRouteMaxTokens = 4;
+// kernels moe_debug_geometry describes: the routed chain's four, then the
+// side lane's two
+constexpr int kGeometryKinds = KIND_COUNT + 2;
 // largest batch the fused single launch takes (one 8-column token tile)
 constexpr int kFusedMaxTokens = 8;
 constexpr int kTailTg = 16;
@@ -96,6 +108,19 @@ struct moe_plan_s {
   int* route_ready = nullptr;
   float* partials[KIND_COUNT] = {};
   size_t partial_cap[KIND_COUNT] = {};  // floats
+  float* side_partials = nullptr;       // the side lane's front (shared gate/up rows)
+  float* rpart = nullptr;               // router pieces' partials, read by the routing CTA
+  size_t rpart_floats = 0;
+  size_t side_partial_cap = 0;
+  cudaStream_t side = nullptr;          // the side lane's stream
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_egu = nullptr;
+  bool side_env_off = false;            // environment MOE_SIDE_LANE=0
+  // L2 prefetch of the chosen experts' tiles by the routing CTA, at most this
+  // many bytes (environment MOE_PREFETCH_MB; 0 turns it off)
+  long long prefetch_bytes = 0;
+  // the routing CTA sums the router partials itself for few tokens
+  // (environment MOE_DIRECT_ROUTE=0 turns it off)
+  bool direct_route = true;
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* out_stage = nullptr;
@@ -133,6 +158,15 @@ struct moe_plan_s {
 // tokens per virtual expert for a forward of B tokens
 int expert_tg(const moe_plan_s* p, int B) {
   return B <= p->expert_small_max_b ? kExpertTgSmall : kExpertTgLarge;
+}
+
+// Whether a forward of B tokens runs the shared expert as a side lane.
+// (shared_sms 0 is the measured choice: no side lane -- at B = 1 it took
+// 95-100 us per step against 82-85 us with the shared expert's rows in the
+// front pass and its down projection leading the tail)
+bool side_lane(const moe_plan_s* p, int B) {
+  return p->cfg.shared_inter > 0 && p->cfg.shared_sms > 0 && !p->side_env_off &&
+         B <= kSideMaxTokens;
 }
 
 namespace {
@@ -225,6 +259,9 @@ struct FwdGeom {
   int nt_front, nt_e, nt_tail, tail_tg;
   int front_grid, front_workers, tail_grid, expert_grid;
   int expert_per_sm;  // CTAs of each expert kernel per SM (1 or 2)
+  bool side;          // the shared expert runs as a side lane
+  int side_grid;      // CTAs of each side-lane kernel
+  int budget;         // shared memory one CTA of the front and tail kernels may take
 };
 
 FwdGeom fwd_geom(const moe_plan_s* p, int B) {
@@ -246,7 +283,24 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
     if (h.nstages >= 3 && h.total <= (size_t)kHalfSmem) f.expert_per_sm = 2;
   }
   f.expert_grid = p->num_sms * f.expert_per_sm;
+  f.side = side_lane(p, B);
+  f.side_grid = f.side ? std::min(p->cfg.shared_sms, p->num_sms) : 0;
+  f.budget = f.side ? kHalfSmem : kBigSmem;
   return f;
+}
+
+// Row blocks of the routed lane's front (router + latent rows) and the side
+// lane's (the shared expert's gate/up rows).
+int rb_routed(const moe_plan_s* p) { return p->RB_router + p->RB_lat; }
+int rb_shared(const moe_plan_s* p) { return p->g[KIND_FRONT].RB - rb_routed(p); }
+
+// Front split-K factor: over every row block, or over one lane's.
+int front_ppr(const moe_plan_s* p, const FwdGeom& f, bool side_part) {
+  const KindGeom& g = p->g[KIND_FRONT];
+  if (!f.side) return best_ppr(g.RB, g.C, f.front_workers, p->split_cost * (1 + std::max(1, f.nt_front) / 4));
+  const int mats = side_part ? rb_shared(p) : rb_routed(p);
+  const int ctas = side_part ? f.side_grid : f.front_workers;
+  return best_ppr(mats, g.C, ctas, p->split_cost * (1 + std::max(1, f.nt_front) / 4));
 }
 
 Params base_params(const moe_plan_s* p, int B) {
@@ -305,13 +359,22 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   q.stage_off = s.stage_off;
   q.matrix_bytes = (long long)p->g[kind].weight_bytes;
   switch (kind) {
-    case KIND_FRONT:  // its routing CTA groups expert tokens by tg
+    case KIND_FRONT: {  // its routing CTA groups expert tokens by tg
       q.wt = p->w_front;
+      q.rb_lo = 0;
+      q.rb_hi = p->g[KIND_FRONT].RB;
+      q.pf_egu = p->w_egu;
+      q.pf_edn = p->w_edn;
+      q.pf_egu_bytes = (long long)p->g[KIND_EGU].weight_bytes;
+      q.pf_edn_bytes = (long long)p->g[KIND_EDN].weight_bytes;
+      const long long per = q.pf_egu_bytes + q.pf_edn_bytes;
+      q.pf_ves = per > 0 ? (int)std::min<long long>(p->ve_max, p->prefetch_bytes / per) : 0;
       q.tg = expert_tg(p, q.B);
       q.RB_router = p->RB_router;
       q.RB_lat = p->RB_lat;
       q.route_cta = 1;
       break;
+    }
     case KIND_EGU: q.wt = p->w_egu; q.tg = expert_tg(p, q.B); break;
     case KIND_EDN: q.wt = p->w_edn; q.tg = expert_tg(p, q.B); break;
     default: q.wt = p->w_tail; q.tg = p->tail_tg; break;
@@ -330,6 +393,9 @@ int ppr_for(const moe_plan_s* p, int mats, int C, int ctas, int nt) {
 
 // Router row blocks are the first pieces handed out and the routing waits
 // for all of them: they get pieces of at most ~C/12 chunks.
+// (Dealing them over every CTA instead -- each CTA's first piece a router
+// piece -- brought the logits no earlier at B = 1 and cost 30 us at B = 128,
+// where every router piece writes 64 KB of partial sums.)
 int router_ppr(int ppr, int C) { return std::max(1, std::min(C, std::max(ppr, 12))); }
 
 // The tail's pieces per row block with its shared part first: ppr pieces
@@ -339,17 +405,31 @@ int router_ppr(int ppr, int C) { return std::max(1, std::min(C, std::max(ppr, 12
 struct TailSplit {
   int ppr_lat, ppr_sh;
 };
-TailSplit tail_split_for(const moe_plan_s* p, int ppr) {
+// The split pays where the tail keeps its activation resident (at most 4
+// tokens: b1 92 -> 84 us per step); with staged activations it cost about
+// 10% of the tail (b64 109 -> 119 us), so larger batches keep one split.
+TailSplit tail_split_for(const moe_plan_s* p, int ppr, int B) {
   const int C = p->g[KIND_TAIL].C, C_lat = p->C_lat, C_sh = C - p->C_lat;
-  if (!p->tail_split || C_sh <= 0) return {ppr, 0};
+  if (!p->tail_split || C_sh <= 0 || B > kSideMaxTokens) return {ppr, 0};
   int lat = (int)std::lround((double)ppr * C_lat / C);
   lat = std::max(1, std::min(C_lat, lat));
   const int sh = std::max(1, std::min(C_sh, ppr - lat));
   return {lat, sh};
 }
-int tail_ppr(const moe_plan_s* p, int ppr) {
-  const TailSplit t = tail_split_for(p, ppr);
+int tail_ppr(const moe_plan_s* p, int ppr, int B) {
+  const TailSplit t = tail_split_for(p, ppr, B);
   return t.ppr_lat + t.ppr_sh;
+}
+
+// largest number of partial-sum floats the side lane's front can need
+size_t side_partial_floats(const moe_plan_s* p) {
+  size_t best = 0;
+  for (int B = 1; B <= p->cfg.max_tokens; ++B) {
+    const FwdGeom f = fwd_geom(p, B);
+    if (!f.side) continue;
+    best = std::max(best, (size_t)rb_shared(p) * front_ppr(p, f, true) * f.nt_front * 1024);
+  }
+  return best;
 }
 
 // largest number of partial-sum floats a kind can need for B <= maxB
@@ -362,12 +442,13 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     const KindGeom& g = p->g[kind];
     if (kind == KIND_FRONT) {
       nt = f.nt_front;
-      const int ppr = ppr_for(p, g.RB, g.C, f.front_workers, nt);
-      pieces = (size_t)p->RB_router * router_ppr(ppr, g.C) + (size_t)(g.RB - p->RB_router) * ppr;
+      const int ppr = front_ppr(p, f, false);
+      const int rb_hi = f.side ? rb_routed(p) : g.RB;
+      pieces = (size_t)p->RB_router * router_ppr(ppr, g.C) + (size_t)(rb_hi - p->RB_router) * ppr;
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      pieces = (size_t)passes * g.RB * tail_ppr(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, nt));
+      pieces = (size_t)passes * g.RB * tail_ppr(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, nt), B);
     } else {
       nt = f.nt_e;
       // the split depends on the routing: take the largest over every
@@ -403,6 +484,7 @@ moe_status check_cfg(const moe_config* c) {
   if (c->top_k > c->num_experts) return MOE_ERR_INVALID_ARG;
   if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
   if (!(c->routed_scale == c->routed_scale)) return MOE_ERR_INVALID_ARG;
+  if (c->shared_sms < -1) return MOE_ERR_INVALID_ARG;
   if (c->num_experts > 1024 || c->top_k > 16 || c->max_tokens > 128) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -451,6 +533,7 @@ void plan_shape(moe_plan_s* p) {
 constexpr size_t kControlBytes = 1024 + sizeof(Ctl) * kSlots;
 moe_status reset_control(moe_plan p) {
   CUDA_TRY(cudaMemset(p->nve, 0, kControlBytes));
+  CUDA_TRY(cudaMemset(p->rpart, 0xFF, sizeof(float) * p->rpart_floats));  // "not yet written"
   for (int k = 0; k < KIND_COUNT; ++k) CUDA_TRY(cudaMemset(p->counters[k], 0, sizeof(int) * p->counter_n[k]));
   CUDA_TRY(cudaDeviceSynchronize());
   return MOE_OK;
@@ -478,6 +561,9 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   if (const char* e = getenv("MOE_PROD_SLEEP")) p->prod_sleep = std::max(0, std::min(2000, atoi(e)));
   if (const char* e = getenv("MOE_TAIL_SPLIT")) p->tail_split = atoi(e) != 0;
   if (const char* e = getenv("MOE_Z_FLAG")) p->z_flag = atoi(e) != 0;
+  if (const char* e = getenv("MOE_SIDE_LANE")) p->side_env_off = atoi(e) == 0;
+  if (const char* e = getenv("MOE_PREFETCH_MB")) p->prefetch_bytes = std::max(0LL, (long long)atoi(e)) << 20;
+  if (const char* e = getenv("MOE_DIRECT_ROUTE")) p->direct_route = atoi(e) != 0;
   if (const char* e = getenv("MOE_CONS_SLEEP")) p->cons_sleep = std::max(0, std::min(2000, atoi(e)));
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
@@ -544,6 +630,19 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
     TRY(alloc(p, &v, sizeof(float) * std::max<size_t>(p->partial_cap[k], 4), false));
     p->partials[k] = (float*)v;
   }
+  // router pieces' partial sums for the routing CTA (few tokens: one token
+  // tile, at most one piece per chunk), every element "not yet written"
+  p->rpart_floats = (size_t)p->RB_router * fr.C * 8 * kRowsPerBlock;
+  TRY(alloc(p, &v, sizeof(float) * p->rpart_floats, false));
+  p->rpart = (float*)v;
+  CUDA_TRY(cudaMemset(v, 0xFF, sizeof(float) * p->rpart_floats));
+  p->side_partial_cap = side_partial_floats(p);
+  TRY(alloc(p, &v, sizeof(float) * std::max<size_t>(p->side_partial_cap, 4), false));
+  p->side_partials = (float*)v;
+  CUDA_TRY(cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking));
+  CUDA_TRY(cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming));
+  CUDA_TRY(cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming));
+  CUDA_TRY(cudaEventCreateWithFlags(&p->ev_egu, cudaEventDisableTiming));
   if (getenv("MOE_TRACE")) {
     // rows for up to two CTAs per SM in every slot
     TRY(alloc(p, &v, sizeof(unsigned long long) * kSlots * 2 * p->num_sms * 24, false));
@@ -576,6 +675,10 @@ void destroy_impl(moe_plan p) {
   for (int k = 0; k < kSlots; ++k)
     for (int j = 0; j < 2; ++j)
       if (p->ev_prof[k][j]) cudaEventDestroy(p->ev_prof[k][j]);
+  if (p->ev_fork) cudaEventDestroy(p->ev_fork);
+  if (p->ev_join) cudaEventDestroy(p->ev_join);
+  if (p->ev_egu) cudaEventDestroy(p->ev_egu);
+  if (p->side) cudaStreamDestroy(p->side);
   cudaGetLastError();
   delete p;
 }
@@ -645,6 +748,64 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
   return MOE_OK;
 }
 
+// Front launch of one forward: every row block (part 0), the routed lane's
+// router + latent rows with the routing CTA (part 1), or the side lane's
+// shared-expert gate/up rows (part 2).
+struct FrontLaunch {
+  SmemGeom sm;
+  int grid, ppr, ppr_r, rb_lo, rb_hi, route_cta;
+};
+FrontLaunch front_launch(const moe_plan_s* p, const FwdGeom& f, int B, int part) {
+  FrontLaunch l;
+  const int tail_tg_eff = std::min(B, p->tail_tg);
+  l.sm = smem_geom(p, KIND_FRONT, f.nt_front, tail_tg_eff, B * p->cfg.top_k, 0, f.budget);
+  const KindGeom& g = p->g[KIND_FRONT];
+  l.ppr = front_ppr(p, f, part == 2);
+  l.ppr_r = router_ppr(l.ppr, g.C);
+  l.rb_lo = part == 2 ? rb_routed(p) : 0;
+  l.rb_hi = part == 1 ? rb_routed(p) : g.RB;
+  l.route_cta = part == 2 ? 0 : 1;
+  l.grid = part == 2 ? f.side_grid : f.front_grid;
+  return l;
+}
+
+// Tail launch: every piece (part 0, shared part first), the latent pieces
+// (part 1, the routed lane) or the shared-expert pieces (part 2, the side
+// lane).  A lane keeps only its own part of the resident activation.
+struct TailLaunch {
+  SmemGeom sm;
+  int grid, ppr, ppr_lat, ppr_sh, split, res_bytes, res_k0, res_k;
+};
+TailLaunch tail_launch(const moe_plan_s* p, const FwdGeom& f, int B, int part) {
+  TailLaunch l;
+  const int tail_tg_eff = std::min(B, p->tail_tg);
+  const KindGeom& g = p->g[KIND_TAIL];
+  const int klat = p->C_lat * kDenseChunkK, kall = g.C * kDenseChunkK;
+  l.res_k0 = part == 2 ? klat : 0;
+  l.res_k = part == 1 ? klat : (part == 2 ? kall - klat : kall);
+  l.res_bytes = (B * resident_stride(l.res_k) <= kResidentMax) ? B * resident_stride(l.res_k) : 0;
+  l.sm = smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * p->cfg.top_k, l.res_bytes, f.budget);
+  const int passes = (B + p->tail_tg - 1) / p->tail_tg;
+  const int grid = part == 2 ? f.side_grid : f.tail_grid;
+  // one split for both lanes: they share every row block's partial-sum slots
+  // and its ticket count
+  const TailSplit ts = tail_split_for(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, f.nt_tail), B);
+  l.ppr_lat = ts.ppr_lat;
+  l.ppr_sh = ts.ppr_sh;
+  l.ppr = ts.ppr_lat + ts.ppr_sh;
+  l.split = ts.ppr_sh > 0;
+  l.grid = grid;
+  return l;
+}
+
+moe_status launch_timed(moe_plan p, int slot, int kind, int nt, const Params& q, int grid, size_t smem,
+                        cudaStream_t s) {
+  if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[slot][0], s));
+  CUDA_TRY((cudaError_t)launch_kind(kind, nt, q, grid, smem, s, p->use_pdl));
+  if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[slot][1], s));
+  return MOE_OK;
+}
+
 moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStream_t s) {
   const moe_config& c = p->cfg;
   const FwdGeom f = fwd_geom(p, B);
@@ -654,17 +815,50 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
   base.out = (uint16_t*)out;
   if (p->use_fused && B <= kFusedMaxTokens) return enqueue_fused(p, base, f, B, s);
 
-  // One stream, each kernel a programmatic dependent of the one before:
-  //   front (router, latent, shared gate/up) -> expert gate/up -> expert down -> tail.
+  // Routed chain on `s`, each kernel a programmatic dependent of the one
+  // before: front (router, latent [, shared gate/up]) -> expert gate/up ->
+  // expert down -> tail.  With the side lane, the shared expert's gate/up
+  // rows and its down projection run as two kernels of their own on the
+  // plan's side stream (forked from and joined back to `s`), their CTAs
+  // sharing the SMs with the routed chain's: the shared expert overlaps the
+  // routing and the routed experts ("Hyper Optimizing Kimi K3 in vLLM",
+  // section 从算子之间找时间), and it streams while the routed chain waits at
+  // its kernel boundaries.  The two lanes meet in the tail's row blocks.
+  if (f.side) {
+    CUDA_TRY(cudaEventRecord(p->ev_fork, s));
+    CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_fork, 0));
+    {
+      Params q = base;
+      const FrontLaunch l = front_launch(p, f, B, 2);
+      set_kind(q, p, KIND_FRONT, l.sm);
+      q.ctl = p->ctl + kSideFront;
+      q.trace = p->trace ? p->trace + (size_t)kSideFront * 2 * p->num_sms * 24 : nullptr;
+      q.partials = p->side_partials;
+      q.PPR = l.ppr;
+      q.PPR_r = l.ppr_r;
+      q.rb_lo = l.rb_lo;
+      q.rb_hi = l.rb_hi;
+      q.route_cta = 0;
+      q.half_sm = 1;
+      TRY(launch_timed(p, kSideFront, KIND_FRONT, f.nt_front, q, l.grid, l.sm.total, p->side));
+    }
+  }
   {
     Params q = base;
-    const SmemGeom sm = smem_geom(p, KIND_FRONT, f.nt_front, tail_tg_eff, B * c.top_k);
-    set_kind(q, p, KIND_FRONT, sm);
-    q.PPR = ppr_for(p, q.RB, q.C, f.front_workers, f.nt_front);
-    q.PPR_r = router_ppr(q.PPR, q.C);
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_FRONT, f.nt_front, q, f.front_grid, sm.total, s, p->use_pdl));
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_FRONT][1], s));
+    const FrontLaunch l = front_launch(p, f, B, f.side ? 1 : 0);
+    set_kind(q, p, KIND_FRONT, l.sm);
+    q.PPR = l.ppr;
+    q.PPR_r = l.ppr_r;
+    q.rb_lo = l.rb_lo;
+    q.rb_hi = l.rb_hi;
+    q.half_sm = f.side ? 1 : 0;
+    if (B <= kDirectRouteMaxTokens && f.nt_front == 1 && p->direct_route) {
+      // at most 16 router pieces a row block: the routing CTA's poll keeps
+      // every load of a round in flight
+      q.rpart = p->rpart;
+      q.PPR_r = std::min(q.C, 16);
+    }
+    TRY(launch_timed(p, KIND_FRONT, KIND_FRONT, f.nt_front, q, l.grid, l.sm.total, s));
   }
   {
     Params q = base;
@@ -673,9 +867,35 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     set_kind(q, p, KIND_EGU, sm);
     q.piece_ctas = f.expert_grid;
     q.split_cost = split_cost_for(p, f.nt_e);
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EGU][1], s));
+    TRY(launch_timed(p, KIND_EGU, KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s));
+  }
+  if (f.side) {
+    // The side lane's down projection starts after expert gate/up: until
+    // then the SMs that the front kernels free go to the routed chain, whose
+    // latency is the step's critical path.
+    CUDA_TRY(cudaEventRecord(p->ev_egu, s));
+    CUDA_TRY(cudaStreamWaitEvent(p->side, p->ev_egu, 0));
+    {
+      Params q = base;
+      const TailLaunch l = tail_launch(p, f, B, 2);
+      set_kind(q, p, KIND_TAIL, l.sm);
+      q.ctl = p->ctl + kSideTail;
+      q.trace = p->trace ? p->trace + (size_t)kSideTail * 2 * p->num_sms * 24 : nullptr;
+      if (l.res_bytes) {
+        q.res_off = kStageOff + l.sm.table_bytes;
+        q.res_stride = resident_stride(l.res_k);
+        q.res_k = l.res_k;
+        q.res_k0 = l.res_k0;
+      }
+      q.PPR = l.ppr;
+      q.ppr_lat = l.ppr_lat;
+      q.ppr_sh = l.ppr_sh;
+      q.tail_split = l.split;
+      q.tail_part = 2;
+      q.half_sm = 1;
+      TRY(launch_timed(p, kSideTail, KIND_TAIL, f.nt_tail, q, l.grid, l.sm.total, p->side));
+    }
+    CUDA_TRY(cudaEventRecord(p->ev_join, p->side));
   }
   {
     Params q = base;
@@ -684,36 +904,31 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     set_kind(q, p, KIND_EDN, sm);
     q.piece_ctas = f.expert_grid;
     q.split_cost = split_cost_for(p, f.nt_e);
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s, p->use_pdl));
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_EDN][1], s));
+    TRY(launch_timed(p, KIND_EDN, KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s));
   }
   {
     Params q = base;
-    const int res_k = p->g[KIND_TAIL].C * kDenseChunkK;
-    const int res_bytes =
-        (B * resident_stride(res_k) <= kResidentMax) ? B * resident_stride(res_k) : 0;
-    const SmemGeom sm =
-        smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * c.top_k, res_bytes);
-    set_kind(q, p, KIND_TAIL, sm);
-    if (res_bytes) {
-      q.res_off = kStageOff + sm.table_bytes;
-      q.res_stride = resident_stride(res_k);
-      q.res_k = res_k;
+    const TailLaunch l = tail_launch(p, f, B, f.side ? 1 : 0);
+    set_kind(q, p, KIND_TAIL, l.sm);
+    if (l.res_bytes) {
+      q.res_off = kStageOff + l.sm.table_bytes;
+      q.res_stride = resident_stride(l.res_k);
+      q.res_k = l.res_k;
+      q.res_k0 = l.res_k0;
     }
-    const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-    const TailSplit ts = tail_split_for(p, ppr_for(p, q.RB * passes, q.C, f.tail_grid, f.nt_tail));
-    q.PPR = ts.ppr_lat + ts.ppr_sh;
-    q.tail_split = ts.ppr_sh > 0;
-    q.ppr_lat = ts.ppr_lat;
-    q.ppr_sh = ts.ppr_sh;
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][0], s));
-    CUDA_TRY((cudaError_t)launch_kind(KIND_TAIL, f.nt_tail, q, f.tail_grid, sm.total, s, p->use_pdl));
-    if (p->profiling) CUDA_TRY(cudaEventRecord(p->ev_prof[KIND_TAIL][1], s));
+    q.PPR = l.ppr;
+    q.tail_split = l.split;
+    q.ppr_lat = l.ppr_lat;
+    q.ppr_sh = l.ppr_sh;
+    q.tail_part = f.side ? 1 : 0;
+    q.half_sm = f.side ? 1 : 0;
+    TRY(launch_timed(p, KIND_TAIL, KIND_TAIL, f.nt_tail, q, f.tail_grid, l.sm.total, s));
   }
+  if (f.side) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));
   p->last_B = B;
   if (p->profiling) {
-    for (int k = 0; k < KIND_COUNT; ++k) {
+    for (int k = 0; k < kSlots; ++k) {
+      if (k == kFused || ((k == kSideFront || k == kSideTail) && !f.side)) continue;
       CUDA_TRY(cudaEventSynchronize(p->ev_prof[k][1]));
       float ms = 0.f;
       CUDA_TRY(cudaEventElapsedTime(&ms, p->ev_prof[k][0], p->ev_prof[k][1]));
@@ -1002,7 +1217,9 @@ moe_status moe_get_plan_info(moe_plan p, moe_plan_info* info) {
       6LL * c.hidden * c.shared_inter;
   info->expert_weight_bytes =
       (3LL * c.expert_inter * c.latent) / 2 + (3LL * c.expert_inter * c.latent) / 32;
-  info->kernels_per_forward = (p->use_fused && p->cfg.max_tokens <= kFusedMaxTokens) ? 1 : KIND_COUNT;
+  info->kernels_per_forward = (p->use_fused && p->cfg.max_tokens <= kFusedMaxTokens)
+                                 ? 1
+                                 : KIND_COUNT + (side_lane(p, p->cfg.max_tokens) ? 2 : 0);
   return MOE_OK;
 }
 
@@ -1054,26 +1271,33 @@ moe_status moe_debug_geometry(const moe_config* cfg, int32_t num_sms, int32_t nu
   const int B = num_tokens, K = c.top_k;
   const FwdGeom f = fwd_geom(p, B);
   const int tail_tg_eff = std::min(B, p->tail_tg);
-  for (int k = 0; k < KIND_COUNT; ++k) {
+  // out[0..3]: the routed chain's kernels; out[4], out[5]: the side lane's
+  // front and tail (grid 0 when this forward has no side lane)
+  for (int k = 0; k < kGeometryKinds; ++k) {
     moe_geometry& o = out[k];
     std::memset(&o, 0, sizeof(o));
     o.kind = k;
-    o.partial_floats_capacity = (int64_t)partial_floats(p, k);
-    const KindGeom& g = p->g[k];
+    const int kk = k == 4 ? KIND_FRONT : k == 5 ? KIND_TAIL : k;
+    o.partial_floats_capacity = (int64_t)(k == 4 ? p->side_partial_cap = side_partial_floats(p)
+                                                 : partial_floats(p, kk));
+    const KindGeom& g = p->g[kk];
     SmemGeom sm;
-    if (k == KIND_FRONT) {
-      sm = smem_geom(p, KIND_FRONT, f.nt_front, tail_tg_eff, B * K);
-      const int ppr = ppr_for(p, g.RB, g.C, f.front_workers, f.nt_front);
-      const int pieces = p->RB_router * router_ppr(ppr, g.C) + (g.RB - p->RB_router) * ppr;
-      o.grid = f.front_grid;
-      o.ctas_per_sm = 1;
+    if (k >= 4 && !f.side) continue;
+    if (kk == KIND_FRONT) {
+      const FrontLaunch l = front_launch(p, f, B, k == 4 ? 2 : (f.side ? 1 : 0));
+      sm = l.sm;
+      const int pieces = (l.rb_lo == 0 ? p->RB_router * l.ppr_r : 0) +
+                         (l.rb_hi - (l.rb_lo == 0 ? p->RB_router : l.rb_lo)) * l.ppr;
+      o.grid = l.grid;
+      o.ctas_per_sm = 1;  // (with the side lane: one CTA of either lane per half SM)
       o.token_tiles = f.nt_front;
       o.max_piece_tokens = B;
-      o.pieces_per_row_block = ppr;
+      o.pieces_per_row_block = l.ppr;
       o.partial_floats_needed = (int64_t)pieces * f.nt_front * 1024;
-      o.route_logit_floats = sm.nstages * sm.stage_bytes / 4 - ((c.num_experts + 31) & ~31);
-    } else if (k == KIND_EGU || k == KIND_EDN) {
-      sm = smem_geom(p, k, f.nt_e, tail_tg_eff, B * K, 0, f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
+      if (l.route_cta)
+        o.route_logit_floats = sm.nstages * sm.stage_bytes / 4 - ((c.num_experts + 31) & ~31);
+    } else if (kk == KIND_EGU || kk == KIND_EDN) {
+      sm = smem_geom(p, kk, f.nt_e, tail_tg_eff, B * K, 0, f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
       o.grid = f.expert_grid;
       o.ctas_per_sm = f.expert_per_sm;
       o.token_tiles = f.nt_e;
@@ -1084,19 +1308,16 @@ moe_status moe_debug_geometry(const moe_config* cfg, int32_t num_sms, int32_t nu
         most = std::max(most, (int64_t)V * g.RB * ppr_for(p, V * g.RB, g.C, f.expert_grid, f.nt_e));
       o.partial_floats_needed = most * f.nt_e * 1024;
     } else {
-      const int res_k = g.C * kDenseChunkK;
-      const int res_bytes =
-          (B * resident_stride(res_k) <= kResidentMax) ? B * resident_stride(res_k) : 0;
-      sm = smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * K, res_bytes);
+      const TailLaunch l = tail_launch(p, f, B, k == 5 ? 2 : (f.side ? 1 : 0));
+      sm = l.sm;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      const int ppr = tail_ppr(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, f.nt_tail));
-      o.grid = f.tail_grid;
+      o.grid = l.grid;
       o.ctas_per_sm = 1;
       o.token_tiles = f.nt_tail;
       o.max_piece_tokens = tail_tg_eff;
-      o.pieces_per_row_block = ppr;
-      o.partial_floats_needed = (int64_t)passes * g.RB * ppr * f.nt_tail * 1024;
-      o.resident_tail_bytes = res_bytes;
+      o.pieces_per_row_block = l.ppr;
+      o.partial_floats_needed = (int64_t)passes * g.RB * l.ppr * f.nt_tail * 1024;
+      o.resident_tail_bytes = l.res_bytes;
     }
     o.stages = sm.nstages;
     o.stage_bytes = sm.stage_bytes;

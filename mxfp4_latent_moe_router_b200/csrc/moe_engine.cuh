@@ -106,11 +106,15 @@ __device__ __forceinline__ Space make_space(const Params& p, int V = 0) {
   } else if (KIND == KIND_TAIL) {
     const int passes = (p.B + p.tg - 1) / p.tg;
     s.ppr = p.PPR;
-    s.total = passes * p.RB * p.PPR;  // (split or not: ppr_sh + ppr_lat == PPR)
+    const int per = p.tail_part == 1 ? p.ppr_lat : p.tail_part == 2 ? p.ppr_sh : p.PPR;
+    s.total = passes * p.RB * per;  // (split or not: ppr_sh + ppr_lat == PPR)
   } else {
     // FRONT: the router row blocks come first, in pieces of their own size
+    // (when this launch holds them), then the rest of [rb_lo, rb_hi)
     s.ppr = p.PPR;
-    s.total = p.RB_router * p.PPR_r + (p.RB - p.RB_router) * p.PPR;
+    const bool router = p.rb_lo == 0;
+    const int rb0 = router ? p.RB_router : p.rb_lo;
+    s.total = (router ? p.RB_router * p.PPR_r : 0) + (p.rb_hi - rb0) * p.PPR;
   }
   return s;
 }
@@ -146,11 +150,13 @@ __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, i
   h.piece = piece;
   h.expert = 0;
   h.dep = 1;
-  if (KIND == KIND_TAIL && p.tail_split) {
+  if (KIND == KIND_TAIL && (p.tail_split || p.tail_part)) {
     // shared-expert pieces of every (pass, row block) first, then the latent
     // ones; a row block's partial slots stay contiguous (latent j, then
-    // shared ppr_lat + j) so the finalising sum keeps one fixed order
-    const int n_sh = sp.total / p.PPR * p.ppr_sh;
+    // shared ppr_lat + j) so the finalising sum keeps one fixed order.  A
+    // lane (tail_part 1 or 2) holds only one of the two kinds, and waits for
+    // its own predecessor before reading any activation.
+    const int n_sh = p.tail_part == 1 ? 0 : p.tail_part == 2 ? sp.total : sp.total / p.PPR * p.ppr_sh;
     int q, pp, cb, cn, slot0;
     if (piece < n_sh) {
       q = piece / p.ppr_sh;
@@ -167,6 +173,7 @@ __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, i
       slot0 = 0;
     }
     const int pieces_here = h.dep ? p.ppr_lat : p.ppr_sh;
+    if (p.tail_part) h.dep = 1;
     h.v = q / p.RB;
     h.rb = q % p.RB;
     h.ppr = p.PPR;
@@ -178,7 +185,7 @@ __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, i
     h.ntok = min(p.tg, p.B - h.tok0);
     return;
   }
-  const int nr = KIND == KIND_FRONT ? p.RB_router * p.PPR_r : 0;
+  const int nr = (KIND == KIND_FRONT && p.rb_lo == 0) ? p.RB_router * p.PPR_r : 0;
   if (piece < nr) {  // router row blocks (smaller pieces, so the logits are summed early)
     h.v = 0;
     h.rb = piece / p.PPR_r;
@@ -186,8 +193,9 @@ __device__ __forceinline__ void piece_header(const Params& p, const Space& sp, i
     h.p0 = h.rb * p.PPR_r;
   } else {
     const int q = piece - nr;
-    const int rb0 = KIND == KIND_FRONT ? p.RB_router : 0;
-    const int per_v = (p.RB - rb0) * sp.ppr;
+    const int rb0 = KIND == KIND_FRONT ? (p.rb_lo == 0 ? p.RB_router : p.rb_lo) : 0;
+    const int rb1 = KIND == KIND_FRONT ? p.rb_hi : p.RB;
+    const int per_v = (rb1 - rb0) * sp.ppr;
     const int v = q / per_v;
     const int rem = q - v * per_v;
     h.v = v;
@@ -414,7 +422,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   // The tail with its shared part first: those pieces need no dependency, so
   // CTAs take pieces (and keep a grab in flight) from the start; the first
   // latent piece they hold waits for it.
-  const bool free_start = KIND == KIND_TAIL && p.tail_split;
+  const bool free_start = KIND == KIND_TAIL && p.tail_split && !p.tail_part;
   if (KIND == KIND_EGU && p.z_done) pdl_trigger();
   // routing tables in shared memory: the per-stage lookups then cost no
   // global round trip (they are visible to the consumers through the first
@@ -710,6 +718,7 @@ __device__ __forceinline__ void mma_mx(const Params& p, const Hdr& h, const uint
 // k < C_lat*64 is the combine c = sum_j w_j y_j (zero past L); the rest is h_s.
 // Only the groups of eight k in [kbeg, kend) are formed (multiples of 8): the
 // h_s part can be built before the routed experts finish, the combine after.
+// The record holds k in [res_k0, res_k0 + res_k) (one lane's part, or all).
 __device__ __forceinline__ void build_resident(const Params& p, uint8_t* res, int tid, int kbeg,
                                                int kend) {
   const int K = p.topk, KR = p.res_k, klat = p.C_lat * 64;
@@ -771,8 +780,9 @@ __device__ __forceinline__ void build_resident(const Params& p, uint8_t* res, in
       lo[u] = pack_bf16x2(v[2 * u] - bf16_lo_to_float(hi[u]), v[2 * u + 1] - bf16_hi_to_float(hi[u]));
     }
     uint8_t* rec = res + (size_t)b * p.res_stride;
-    *reinterpret_cast<uint4*>(rec + k0 * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(rec + KR * 2 + k0 * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    const int kr = k0 - p.res_k0;
+    *reinterpret_cast<uint4*>(rec + kr * 2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(rec + KR * 2 + kr * 2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -781,7 +791,7 @@ __device__ __forceinline__ void mma_tail_resident(const Params& p, const Hdr& h,
                                                   const uint8_t* res, float (&acc)[NT][4],
                                                   float (&acc2)[NT][4], int warp, int lane) {
   const int g = lane >> 2, tig = lane & 3;
-  const int kbase = h.chunk * kDenseChunkK;
+  const int kbase = h.chunk * kDenseChunkK - p.res_k0;
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
     if (b < h.nb) {
@@ -938,7 +948,7 @@ __device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int wa
 
 __device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
                                           float* lg_s, int lg_cap, int* wtot, int tid, int warp,
-                                          int lane);
+                                          int lane, const float* lg_sm = nullptr);
 
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
@@ -1085,9 +1095,11 @@ __device__ __forceinline__ void stage_floats(const float* src, int n, float* dst
 }
 
 // lg_s: shared memory for lg_cap floats of logits (at least E).
+// lg_sm: the logits [B][E] already in shared memory (few tokens, summed by
+// the routing CTA itself), else they are read from p.logits.
 __device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
                                           float* lg_s, int lg_cap, int* wtot, int tid, int warp,
-                                          int lane) {
+                                          int lane, const float* lg_sm) {
   const int E = p.E, K = p.topk, B = p.B;
   const int tg = p.tg > 0 ? p.tg : 1;
   int* cnt = reinterpret_cast<int*>(scratch);  // [E] slots per expert
@@ -1147,8 +1159,12 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
       const int e0 = (int)((long long)q * E / P), e1 = (int)((long long)(q + 1) * E / P);
       TopkCand c;
       float smax, ssum;
-      warp_topk_slice_any(p.logits + (long long)b * E, bias, e0, e1, K, p.score_fn, lane, c, smax,
-                          ssum);
+      if (lg_sm)
+        warp_topk_slice_any<true>(lg_sm + (long long)b * E, bias, e0, e1, K, p.score_fn, lane, c,
+                                  smax, ssum);
+      else
+        warp_topk_slice_any(p.logits + (long long)b * E, bias, e0, e1, K, p.score_fn, lane, c,
+                            smax, ssum);
       if (lane < K) cand[(b * P + q) * K + lane] = c;
       if (lane == 0) part[b * P + q] = make_float2(smax, ssum);
     }
@@ -1220,6 +1236,25 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
     bg += gsz[i];
   }
   if (tid == kConsumerThreads - 1) *p.nve = bg < p.ve_max ? bg : p.ve_max;
+  // the chosen experts' weights into L2, gate/up before down, in the order
+  // the expert kernels take them (virtual expert index), 64 KB a request
+  if (p.pf_ves > 0) {
+    for (int pass = 0; pass < 2; ++pass) {
+      const uint8_t* base = pass == 0 ? p.pf_egu : p.pf_edn;
+      const long long per = pass == 0 ? p.pf_egu_bytes : p.pf_edn_bytes;
+      int v = bg - sg;  // this thread's first virtual expert index
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = 4 * tid + i;
+        if (e < E && gsz[i] > 0 && v < p.pf_ves) {
+          const uint8_t* src = base + (long long)e * per;
+          for (long long o = 0; o < per; o += 65536)
+            prefetch_l2(src + o, (uint32_t)min(65536LL, per - o));
+        }
+        v += gsz[i];
+      }
+    }
+  }
   named_sync(1, kConsumerThreads);
   if (tr) tr[18] = global_ns();
   for (int s = tid; s < B * K; s += kConsumerThreads) {
@@ -1237,8 +1272,63 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
 // every router row block has been summed, select the experts, build the
 // per-expert token lists and publish them; the other CTAs keep streaming the
 // latent and shared-expert rows meanwhile.
+// Few tokens (p.rpart): the router logits are the sums of the router pieces'
+// partials, read straight from where the pieces wrote them, polling on the
+// data (see Params::rpart).  pstride: floats between two pieces' partials.
+// Writes the logits to lgs [B][E] (shared memory) and to p.logits; false if
+// they never all arrived (the wait is bounded).
+__device__ __forceinline__ bool route_poll_logits(const Params& p, float* lgs, int pstride, int tid) {
+  constexpr int kMaxPieces = 16;  // router pieces per row block in this mode (host: at most 16)
+  constexpr int kOut = 2;         // outputs a thread sums per round: 32 loads in flight
+  const int E = p.E, B = p.B, ppr = p.PPR_r, n = B * E;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 0; it < (1u << 20); ++it) {
+    bool missing = false;
+    for (int o0 = tid; o0 < n; o0 += kOut * kConsumerThreads) {
+      float v[kOut][kMaxPieces];
+      // every load of the round first (one round trip), then the sums, each
+      // in piece order (the same sum every run)
+#pragma unroll
+      for (int u = 0; u < kOut; ++u) {
+        const int o = o0 + u * kConsumerThreads;
+        const int b = o / E, e = o - b * E;
+        const float* src =
+            p.rpart + (long long)(e >> 7) * ppr * pstride + b * kRowsPerBlock + (e & 127);
+#pragma unroll
+        for (int j = 0; j < kMaxPieces; ++j)
+          v[u][j] = (o < n && j < ppr) ? __ldcg(src + (long long)j * pstride) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kOut; ++u) {
+        const int o = o0 + u * kConsumerThreads;
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxPieces; ++j) {
+          missing |= __float_as_uint(v[u][j]) == 0xFFFFFFFFu;
+          acc += v[u][j];
+        }
+        if (o < n) lgs[o] = acc;
+      }
+    }
+    if (!named_sync_or(1, kConsumerThreads, missing)) {
+      // every piece's partials arrived: publish the logits, restore the marks
+      for (int o = tid; o < n; o += kConsumerThreads) {
+        p.logits[o] = lgs[o];
+        const int b = o / E, e = o - b * E;
+        float* dst = p.rpart + (long long)(e >> 7) * ppr * pstride + b * kRowsPerBlock + (e & 127);
+        for (int j = 0; j < ppr; ++j) dst[(long long)j * pstride] = __uint_as_float(0xFFFFFFFFu);
+      }
+      return true;
+    }
+    __nanosleep(64);
+    if ((it & 15) == 15 && global_ns() - t0 > 1000000000ull) break;
+  }
+  if (tid == 0) atomicOr(p.err, 1 << ERR_WAIT_DEP);
+  return false;
+}
+
 __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, float* bias_s,
-                                          int* sm_flag, int tid, int warp, int lane) {
+                                          int* sm_flag, int tid, int warp, int lane, int pstride) {
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
   // the selection bias is static: stage it in shared memory before the
   // logits exist, so the selection waits on one round trip, not two
@@ -1248,6 +1338,24 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
     bias = bias_s;
   }
   named_sync(1, kConsumerThreads);
+  // the rest of the idle ring holds staged logits
+  const int bias_floats = (p.E + 31) & ~31;
+  const int ring_floats = p.nstages * p.stage_bytes / 4;
+  float* lgs = bias_s + bias_floats;
+  if (p.rpart) {
+    // the logits straight from the router pieces' partial sums
+    const bool ok = route_poll_logits(p, lgs, pstride, tid);
+    named_sync(1, kConsumerThreads);
+    if (!ok) return;
+    if (tr && tid == 0) tr[4] = global_ns();
+    route_tokens(p, bias, scratch, lgs + p.B * p.E, ring_floats - bias_floats - p.B * p.E,
+                 sm_flag + 16, tid, warp, lane, lgs);  // ends with a barrier
+    if (tid == 0) {
+      if (tr) tr[5] = global_ns();
+      st_release(p.route_ready, 1);
+    }
+    return;
+  }
   if (tid == 0) {
     bool ok = false;
     for (uint32_t i = 0; i < (1u << 22); ++i) {
@@ -1263,9 +1371,6 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
   if (!sm_flag[0]) return;
   if (tr && tid == 0) tr[4] = global_ns();
-  // the rest of the idle ring holds staged logits
-  const int bias_floats = (p.E + 31) & ~31;
-  const int ring_floats = p.nstages * p.stage_bytes / 4;
   route_tokens(p, bias, scratch, bias_s + bias_floats, ring_floats - bias_floats, sm_flag + 16,
                tid, warp, lane);  // ends with a barrier
   if (tid == 0) {
@@ -1405,7 +1510,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   //   - the expert gate/up kernel with a z count reads nothing of the front
   //     kernel but what its producer copies after that count; it waits for
   //     the front grid only before exiting.
-  const bool lazy = KIND == KIND_TAIL && p.tail_split;
+  const bool lazy = KIND == KIND_TAIL && p.tail_split && !p.tail_part;
   const bool late = KIND == KIND_EGU && p.z_done;
   uint8_t* res = stage_base - p.stage_off + p.res_off;  // shared-memory base + offset
   const int klat = p.C_lat * 64;
@@ -1415,7 +1520,9 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   auto tail_dep = [&](int kbeg, int kend) {
     pdl_wait();
     pdl_trigger();
-    if (KIND == KIND_TAIL && tid == 0) {
+    // (the side lane's tail waits only for the shared expert's gate/up, so
+    // it leaves them alone)
+    if (KIND == KIND_TAIL && tid == 0 && p.tail_part != 2) {
       *p.route_ready = 0;
       if (p.z_done) *p.z_done = 0;
     }
@@ -1431,7 +1538,8 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       named_sync(1, kConsumerThreads);
     }
   } else if (!late) {
-    tail_dep(0, p.res_k);
+    // everything the record holds: both parts, or one lane's
+    tail_dep(p.res_k0, p.res_k0 + p.res_k);
   }
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
   int n_pieces = 0, n_fin = 0;
@@ -1480,6 +1588,17 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[t][q] += acc2[t][q];
 
+    if (KIND == KIND_FRONT && p.rpart && h.rb < p.RB_router) {
+      // router piece, few tokens: its partial sums go where the routing CTA
+      // polls for them; no ticket, no finalisation
+      Params q = p;
+      q.partials = p.rpart;
+      write_partial<NT>(q, h.piece, h.ntok, acc, warp, lane);
+      const long long t_c = clock64();
+      c_end += t_c - t_a;
+      t_a = t_c;
+      continue;
+    }
     if (h.ppr == 1) {
       ++n_fin;
       epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
@@ -1552,8 +1671,11 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
 
 // ---------------------------------------------------------------------------
 
-template <int KIND, int NT>
-__global__ void __launch_bounds__(kThreads, (KIND == KIND_EGU || KIND == KIND_EDN) && NT == 1 ? 2 : 1)
+// MINB: CTAs per SM the instantiation is compiled for.  Two for the expert
+// kernels at one token tile, and for the one-tile front and tail variants the
+// side lane uses (a CTA of each lane on one SM); one otherwise.
+template <int KIND, int NT, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
     moe_kernel(const __grid_constant__ Params p) {
   // shared memory: [0,128) full barriers, [128,256) empty barriers,
   // [256,512) flags, [scratch_off, ...) scratch, [table_off, ...) routing
@@ -1587,7 +1709,8 @@ __global__ void __launch_bounds__(kThreads, (KIND == KIND_EGU || KIND == KIND_ED
     pdl_wait();
     pdl_trigger();
     if (warp < kConsumerWarps)
-      route_cta(p, scratch, reinterpret_cast<float*>(stages), sm_flag, threadIdx.x, warp, lane);
+      route_cta(p, scratch, reinterpret_cast<float*>(stages), sm_flag, threadIdx.x, warp, lane,
+                NT * 8 * kRowsPerBlock);
   } else if (warp == kConsumerWarps) {
     producer<KIND>(p, ctl, stages, tables, full, empty, lane);
   } else {
@@ -1609,8 +1732,13 @@ __global__ void __launch_bounds__(kThreads, (KIND == KIND_EGU || KIND == KIND_ED
 // host-side launch of one instantiation
 
 template <int KIND, int NT>
+constexpr int default_minb() {
+  return (KIND == KIND_EGU || KIND == KIND_EDN) && NT == 1 ? 2 : 1;
+}
+
+template <int KIND, int NT, int MINB = default_minb<KIND, NT>()>
 static int launch_one(const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
-  auto kfn = moe_kernel<KIND, NT>;
+  auto kfn = moe_kernel<KIND, NT, MINB>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -1624,17 +1752,22 @@ static int launch_one(const Params& p, int grid, size_t smem, cudaStream_t s, bo
   return (int)cudaLaunchKernelEx(&cfg, kfn, p);
 }
 
-template <int KIND, int NT>
+template <int KIND, int NT, int MINB = default_minb<KIND, NT>()>
 static int set_attr(size_t bytes) {
-  return (int)cudaFuncSetAttribute(moe_kernel<KIND, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)bytes);
+  return (int)cudaFuncSetAttribute(moe_kernel<KIND, NT, MINB>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 // Token tiles (NT) each kind is built for: dense kinds up to 16 (128 tokens),
-// expert kinds up to 4 (groups of 32), the tail up to 2 (groups of 16).
+// expert kinds up to 4 (groups of 32), the tail up to 2 (groups of 16); the
+// front and tail also at one tile for two CTAs per SM (p.half_sm).
 template <int KIND>
 static int launch_kind_nt(int nt, const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
   constexpr bool kDense = (KIND == KIND_FRONT);
+  constexpr bool kHalf = (KIND == KIND_FRONT || KIND == KIND_TAIL);
+  if constexpr (kHalf) {
+    if (p.half_sm) return nt == 1 ? launch_one<KIND, 1, 2>(p, grid, smem, s, pdl) : (int)cudaErrorInvalidValue;
+  }
   switch (nt) {
     case 1: return launch_one<KIND, 1>(p, grid, smem, s, pdl);
     case 2: return launch_one<KIND, 2>(p, grid, smem, s, pdl);
@@ -1657,6 +1790,7 @@ static int set_attr_kind(size_t bytes) {
   int e = set_attr<KIND, 1>(bytes) | set_attr<KIND, 2>(bytes);
   if constexpr (KIND != KIND_TAIL) e |= set_attr<KIND, 4>(bytes);
   if constexpr (KIND == KIND_FRONT) e |= set_attr<KIND, 8>(bytes) | set_attr<KIND, 16>(bytes);
+  if constexpr (KIND == KIND_FRONT || KIND == KIND_TAIL) e |= set_attr<KIND, 1, 2>(bytes);
   return e;
 }
 

@@ -510,7 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_mega_kernel(const __grid_cons
     pdl_wait();
     pdl_trigger();
     if (warp < kConsumerWarps)
-      route_cta(pf, scratch, reinterpret_cast<float*>(stages), sm_flag, threadIdx.x, warp, lane);
+      route_cta(pf, scratch, reinterpret_cast<float*>(stages), sm_flag, threadIdx.x, warp, lane,
+                8 * kRowsPerBlock);
   } else if (warp == kConsumerWarps) {
     mega_producer(mp, stages, tables, full, empty, lane);
   } else {

@@ -69,6 +69,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       : "memory");
 }
 
+// ---- L2 prefetch of a global range (16-byte aligned, a multiple of 16 bytes)
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---- 16-byte asynchronous copies (global -> shared, past L1) -------------------
 // Many small rows: every producer lane copies its share.  The mbarrier then
 // tracks them: cp_async_mbar_arrive raises the barrier's pending count at once
@@ -117,6 +122,17 @@ __device__ __forceinline__ unsigned smid() {
 // ---- named barrier among the consumer warps ---------------------------------
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// the same barrier, returning whether any participating thread passed true
+__device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, %2, %3, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ---- loads that bypass L1 (data written by other CTAs of this grid) ----------

@@ -66,8 +66,11 @@ def summarize(trace: np.ndarray, names, clock_ghz: float = 1.965) -> list[dict]:
         if len(route):
             c = rows[route[0]]
             pub = rows[:, LOGITS_PUBLISHED]
+            st = lambda i: float(us(c[i])) if c[i] > 0 else None  # noqa: E731
             s["routing_us"] = {
                 "logits_published_last": float(us(pub[pub > 0].max())) if (pub > 0).any() else None,
+                "cleared": st(ROUTE_CLEARED), "staged_or_slices": st(ROUTE_STAGED),
+                "first_token_or_merge": st(ROUTE_FIRST_TOKEN), "first_group": st(ROUTE_FIRST_GROUP),
                 "start": float(us(c[ROUTE_START])),
                 "selected": float(us(c[ROUTE_SELECTED])),
                 "tables_built": float(us(c[ROUTE_SCANNED])),
@@ -90,9 +93,12 @@ def format_summary(rows: list[dict]) -> str:
                         s["producer_us"]["wait"], s["producer_us"]["issue"]))
         if "routing_us" in s:
             r = s["routing_us"]
-            lines.append("    routing: logits %s, start %.1f, selected %.1f, tables %.1f, published %.1f"
-                         % ("%.1f" % r["logits_published_last"] if r["logits_published_last"] is not None
-                            else "-", r["start"], r["selected"], r["tables_built"], r["published"]))
+            f = lambda v: "-" if v is None else "%.1f" % v  # noqa: E731
+            lines.append("    routing: logits %s, start %.1f, cleared %s, slices/staged %s, merge/first token %s, "
+                         "first group %s, selected %.1f, tables %.1f, published %.1f"
+                         % (f(r["logits_published_last"]), r["start"], f(r["cleared"]),
+                            f(r["staged_or_slices"]), f(r["first_token_or_merge"]), f(r["first_group"]),
+                            r["selected"], r["tables_built"], r["published"]))
     return "\n".join(lines)
 
 

@@ -19,10 +19,11 @@ pytestmark = pytest.mark.gpu
 
 
 class GpuBlock:
-    def __init__(self, shape, w, max_tokens):
+    def __init__(self, shape, w, max_tokens, shared_sms=0):
         self.shape = shape
         self.w = w
-        self.plan = moe.MoePlan(moe.config_from_shape(shape, max_tokens=max_tokens))
+        self.plan = moe.MoePlan(moe.config_from_shape(shape, max_tokens=max_tokens,
+                                                      shared_sms=shared_sms))
         self.dev_w = moe.weights_to_device(w)
         self.plan.load(self.dev_w)
         torch.cuda.synchronize()
@@ -294,3 +295,65 @@ def test_batched_full_size_as_benchmarked(name):
         blk.plan.close()
         del blk
         torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# the shared expert as a side lane (B <= 4): on, off, bounded
+
+
+@pytest.mark.parametrize("shared_sms", [0, -1, 24, 148])
+@pytest.mark.parametrize("B", [1, 3, 4])
+def test_side_lane_settings_agree_with_the_oracle(tiny, shared_sms, B):
+    shape, w = tiny
+    plan = moe.MoePlan(moe.config_from_shape(shape, max_tokens=4, shared_sms=shared_sms))
+    try:
+        plan.load(moe.weights_to_device(w))
+        x = synth.make_x(shape, tokens=B, step=60 + B)
+        xt = torch.from_numpy(x.view(np.int16)).cuda()
+        out = torch.empty_like(xt)
+        plan.forward(xt, out)
+        torch.cuda.synchronize()
+        assert plan.sync_status() == 0
+        ref = oracle.forward(shape, w, x)
+        ids, wts = plan.routing(B)
+        check_routing(shape, w, x, ids, wts, plan.fetch(moe.MOE_DBG_LOGITS, B), ref)
+        assert_close(plan.fetch(moe.MOE_DBG_HS, B), ref["h_s"], "h_s")
+        assert_close(bf16_to_f32(out.cpu().numpy().view(np.uint16)), ref["out"], "out")
+        side = shared_sms > 0
+        assert plan.info().kernels_per_forward == (6 if side else 4)
+    finally:
+        plan.close()
+
+
+def test_side_lane_graph_replay_and_back_to_back(tiny):
+    """The side stream's fork and join captured into a CUDA graph; forwards
+    back to back on one stream keep their own inputs."""
+    shape, w = tiny
+    blk = GpuBlock(shape, w, max_tokens=4, shared_sms=148)
+    xa = synth.make_x(shape, tokens=3, step=70)
+    xb = synth.make_x(shape, tokens=3, step=71)
+    ta = torch.from_numpy(xa.view(np.int16)).cuda()
+    tb = torch.from_numpy(xb.view(np.int16)).cuda()
+    oa, ob, og = torch.empty_like(ta), torch.empty_like(tb), torch.empty_like(ta)
+    for _ in range(3):
+        blk.plan.forward(ta, oa)
+        blk.plan.forward(tb, ob)
+    torch.cuda.synchronize()
+    for x, o in ((xa, oa), (xb, ob)):
+        ref = oracle.forward(shape, w, x, intermediates=False)
+        assert_close(bf16_to_f32(o.cpu().numpy().view(np.uint16)), ref["out"], "out")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        blk.plan.forward(ta, og, stream=s)
+        s.synchronize()
+        og.zero_()
+        with torch.cuda.graph(g, stream=s):
+            blk.plan.forward(tb, ob, stream=s)
+            blk.plan.forward(ta, og, stream=s)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(og, oa)
+    assert blk.plan.sync_status() == 0
