@@ -84,6 +84,15 @@ struct Params {
   // round trip from the last router piece to the selection instead of four
   // (ticket, partial sums, count, logits).  Null: the usual split-K finish.
   float* rpart;
+  // TAIL with staged activations (more than the resident size): the tail's
+  // CTAs first form every token's activation once -- the combine c = sum_j
+  // w_j y_j for the latent chunks, h_s for the shared ones -- as records of
+  // 64 bf16 hi then 64 bf16 lo values, t_rec[chunk][B][256 bytes], and count
+  // themselves done in t_ready (release); the producers stream activation
+  // rows from those records once the count reaches the grid.  Null: the
+  // combine is formed per stage (the fused single launch).
+  uint8_t* t_rec;
+  int* t_ready;
   // EGU: the latent row blocks' finalisations count up here (release); the
   // expert gate/up kernel reads z once it reaches RB_lat instead of waiting
   // for the whole front grid (whose last CTAs stream shared-expert rows)
@@ -91,7 +100,7 @@ struct Params {
   int RB_router;      // FRONT: leading row blocks holding router rows
   int RB_lat;         // FRONT: row blocks of the latent projection (after the router's);
                       // the shared expert's gate/up row blocks follow
-  int route_cta;      // FRONT: 1 when the grid's last CTA is the routing CTA (no pieces)
+  int route_cta;      // FRONT: routing CTAs, the grid's last ones (no pieces); 0: none
   int tg;             // tokens per group (EGU/EDN/TAIL)
   int KL;             // K extent of the chunked dimension (for ragged last chunk)
   int KS;             // TAIL: K extent of the shared part (I_s)
@@ -129,6 +138,7 @@ struct Params {
   unsigned long long* trace;
   int* counters;   // finalize tickets per (virtual matrix, row block)
   int* router_done;
+  int* route_cnt;  // FRONT, several routing CTAs: tickets of those done selecting
   // 1 once this forward's routing tables are published (release by the
   // routing CTA); the expert kernels stream their experts' tiles as soon as
   // it is set, before their own dependency resolves.  Cleared by the tail,

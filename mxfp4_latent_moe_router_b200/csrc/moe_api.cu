@@ -43,7 +43,10 @@ constexpr int kDirectRouteMaxTokens = 4;
 constexpr int kGeometryKinds = KIND_COUNT + 2;
 // largest batch the fused single launch takes (one 8-column token tile)
 constexpr int kFusedMaxTokens = 8;
-constexpr int kTailTg = 16;
+// tokens a tail pass takes: 64 (eight token tiles) with formed records; the
+// fused single launch stages the k slots' y rows per token and takes at most
+// 8 tokens
+constexpr int kTailTg = 64;
 // Tokens per virtual expert (an expert's slots are cut into groups of at most
 // this many).  Groups of 8 keep the expert kernels at one token tile, where
 // two CTAs share an SM.  That wins even for 128 Zipf-skewed tokens (675 vs
@@ -110,6 +113,9 @@ struct moe_plan_s {
   size_t partial_cap[KIND_COUNT] = {};  // floats
   float* side_partials = nullptr;       // the side lane's front (shared gate/up rows)
   float* rpart = nullptr;               // router pieces' partials, read by the routing CTA
+  uint8_t* t_rec = nullptr;             // the tail's formed activation records
+  int* t_ready = nullptr;
+  int* route_cnt = nullptr;
   size_t rpart_floats = 0;
   size_t side_partial_cap = 0;
   cudaStream_t side = nullptr;          // the side lane's stream
@@ -217,7 +223,7 @@ constexpr int kResidentMax = 72 * 1024;
 int resident_stride(int res_k) { return res_k * 4 + 64; }
 
 SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int slots,
-                   int res_bytes = 0, int budget = kBigSmem) {
+                   int res_bytes = 0, int budget = kBigSmem, bool formed = false) {
   const int topk = p->cfg.top_k, ve_max = p->ve_max;
   SmemGeom s;
   // routing tables (virtual experts + expert-sorted slots) for the expert kernels
@@ -235,7 +241,9 @@ SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int s
     s.act_stride = 576;
     act = 8 * nt * s.act_stride;
   } else {
-    act = res_bytes ? 0 : tail_tg_eff * std::max(1, topk) * 256;
+    // resident: none; formed records: 256 bytes a token; else the k slots'
+    // y rows a token (the fused single launch)
+    act = res_bytes ? 0 : formed ? tail_tg_eff * 256 : tail_tg_eff * std::max(1, topk) * 256;
   }
   const int tile = (kind == KIND_EGU || kind == KIND_EDN) ? kMxTileBytes : kDenseTileBytes;
   s.act_off = kHdr + tile;
@@ -259,6 +267,7 @@ struct FwdGeom {
   int nt_front, nt_e, nt_tail, tail_tg;
   int front_grid, front_workers, tail_grid, expert_grid;
   int expert_per_sm;  // CTAs of each expert kernel per SM (1 or 2)
+  int route_ctas;     // the front's routing CTAs (its last ones)
   bool side;          // the shared expert runs as a side lane
   int side_grid;      // CTAs of each side-lane kernel
   int budget;         // shared memory one CTA of the front and tail kernels may take
@@ -273,8 +282,11 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   // every kernel takes every SM (one CTA each; the one-tile expert kernels
   // two, when half the shared memory still holds a ring of 3 stages); the
   // front kernel's last CTA is the routing CTA and streams nothing
+  // one routing CTA selects up to 16 tokens (two a warp); more tokens share
+  // the selection over more CTAs, the last of which builds the tables
+  f.route_ctas = std::max(1, std::min(8, (B + 15) / 16));
   f.front_grid = p->num_sms;
-  f.front_workers = p->num_sms - 1;
+  f.front_workers = p->num_sms - f.route_ctas;
   f.tail_grid = p->num_sms;
   f.expert_per_sm = 1;
   if (f.nt_e == 1 && p->expert_per_sm_max >= 2) {
@@ -334,6 +346,8 @@ Params base_params(const moe_plan_s* p, int B) {
   q.route_ready = p->route_ready;
   q.err = p->err;
   q.z_done = p->z_flag ? p->z_done : nullptr;
+  q.t_ready = p->t_ready;
+  q.route_cnt = p->route_cnt;
   q.RB_lat = p->RB_lat;
   q.prod_sleep = p->prod_sleep;
   q.cons_sleep = p->cons_sleep;
@@ -520,7 +534,7 @@ void plan_shape(moe_plan_s* p) {
   tl.C = p->C_lat + ceil_div(Is, kDenseChunkK);
   tl.KL = L;
   tl.weight_bytes = (size_t)tl.RB * tl.C * kDenseTileBytes;
-  p->tail_tg = std::max(1, std::min(kTailTg, 128 / c.top_k));
+  p->tail_tg = kTailTg;
 
   const int maxB = c.max_tokens, K = c.top_k;
   const int slots = maxB * K;
@@ -618,6 +632,8 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->done = p->nve + 8;
   p->route_ready = p->nve + 3;
   p->z_done = p->nve + 5;  // (nve + 4: a flag nothing sets, for the expiring-wait test)
+  p->t_ready = p->nve + 6;
+  p->route_cnt = p->nve + 7;
   p->ctl = reinterpret_cast<Ctl*>((uint8_t*)v + 1024);
   CUDA_TRY(cudaMemset(v, 0, kControlBytes));
   const int cnt_n[KIND_COUNT] = {fr.RB, p->ve_max * eg.RB, p->ve_max * ed.RB, maxB * tl.RB};
@@ -636,6 +652,9 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   TRY(alloc(p, &v, sizeof(float) * p->rpart_floats, false));
   p->rpart = (float*)v;
   CUDA_TRY(cudaMemset(v, 0xFF, sizeof(float) * p->rpart_floats));
+  // the tail's formed activation records, [C chunks][max_tokens][256 bytes]
+  TRY(alloc(p, &v, (size_t)tl.C * maxB * 256, false));
+  p->t_rec = (uint8_t*)v;
   p->side_partial_cap = side_partial_floats(p);
   TRY(alloc(p, &v, sizeof(float) * std::max<size_t>(p->side_partial_cap, 4), false));
   p->side_partials = (float*)v;
@@ -764,7 +783,7 @@ FrontLaunch front_launch(const moe_plan_s* p, const FwdGeom& f, int B, int part)
   l.ppr_r = router_ppr(l.ppr, g.C);
   l.rb_lo = part == 2 ? rb_routed(p) : 0;
   l.rb_hi = part == 1 ? rb_routed(p) : g.RB;
-  l.route_cta = part == 2 ? 0 : 1;
+  l.route_cta = part == 2 ? 0 : f.route_ctas;
   l.grid = part == 2 ? f.side_grid : f.front_grid;
   return l;
 }
@@ -775,6 +794,7 @@ FrontLaunch front_launch(const moe_plan_s* p, const FwdGeom& f, int B, int part)
 struct TailLaunch {
   SmemGeom sm;
   int grid, ppr, ppr_lat, ppr_sh, split, res_bytes, res_k0, res_k;
+  bool formed;  // staged activations from formed records (not resident)
 };
 TailLaunch tail_launch(const moe_plan_s* p, const FwdGeom& f, int B, int part) {
   TailLaunch l;
@@ -784,7 +804,9 @@ TailLaunch tail_launch(const moe_plan_s* p, const FwdGeom& f, int B, int part) {
   l.res_k0 = part == 2 ? klat : 0;
   l.res_k = part == 1 ? klat : (part == 2 ? kall - klat : kall);
   l.res_bytes = (B * resident_stride(l.res_k) <= kResidentMax) ? B * resident_stride(l.res_k) : 0;
-  l.sm = smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * p->cfg.top_k, l.res_bytes, f.budget);
+  l.formed = l.res_bytes == 0;
+  l.sm = smem_geom(p, KIND_TAIL, f.nt_tail, tail_tg_eff, B * p->cfg.top_k, l.res_bytes, f.budget,
+                   l.formed);
   const int passes = (B + p->tail_tg - 1) / p->tail_tg;
   const int grid = part == 2 ? f.side_grid : f.tail_grid;
   // one split for both lanes: they share every row block's partial-sum slots
@@ -851,6 +873,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     q.PPR_r = l.ppr_r;
     q.rb_lo = l.rb_lo;
     q.rb_hi = l.rb_hi;
+    q.route_cta = l.route_cta;
     q.half_sm = f.side ? 1 : 0;
     if (B <= kDirectRouteMaxTokens && f.nt_front == 1 && p->direct_route) {
       // at most 16 router pieces a row block: the routing CTA's poll keeps
@@ -922,6 +945,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     q.ppr_sh = l.ppr_sh;
     q.tail_part = f.side ? 1 : 0;
     q.half_sm = f.side ? 1 : 0;
+    if (l.formed) q.t_rec = p->t_rec;
     TRY(launch_timed(p, KIND_TAIL, KIND_TAIL, f.nt_tail, q, f.tail_grid, l.sm.total, s));
   }
   if (f.side) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));

@@ -232,7 +232,7 @@ __device__ __forceinline__ void chunk_header(const Params& p, int c, int c_first
   else if (KIND == KIND_EGU || KIND == KIND_EDN)
     ab = h.ntok * kActRecBytes;
   else
-    ab = p.res_off ? 0 : ((c < p.C_lat) ? h.ntok * p.topk * 256 : h.ntok * 256);
+    ab = p.res_off ? 0 : p.t_rec ? h.ntok * 256 : ((c < p.C_lat) ? h.ntok * p.topk * 256 : h.ntok * 256);
   h.act_bytes = ab;
 }
 
@@ -350,7 +350,9 @@ __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t
                p.h_mx + ((long long)h.chunk * p.ld_slots + h.tok0 + r) * kActRecBytes, kActRecBytes,
                bar);
   } else {
-    if (lane == 0 && !p.res_off) {
+    if (lane == 0 && !p.res_off && p.t_rec) {
+      bulk_g2s(act, p.t_rec + ((long long)h.chunk * p.B + h.tok0) * 256, h.act_bytes, bar);
+    } else if (lane == 0 && !p.res_off) {
       if (h.chunk < p.C_lat)
         bulk_g2s(act, p.y + ((long long)h.chunk * p.ld_slots + (long long)h.tok0 * p.topk) * 64,
                  h.act_bytes, bar);
@@ -398,6 +400,13 @@ __device__ __forceinline__ bool wait_count(const int* counter, int target, int* 
 //                     predecessor).
 template <int KIND>
 __device__ __forceinline__ bool producer_dep_wait(const Params& p, int lane) {
+  if (KIND == KIND_TAIL && p.t_rec) {
+    // the records the grid's consumers form after the expert kernels
+    pdl_trigger();
+    const bool ok = wait_count(p.t_ready, (int)gridDim.x, p.err, lane);
+    fence_proxy_async_global();  // the records are read by bulk copies
+    return ok;
+  }
   if (KIND == KIND_EGU && p.z_done) {
     const bool ok = wait_count(p.z_done, p.RB_lat, p.err, lane);
     fence_proxy_async_global();  // the z records are read by bulk copies
@@ -815,6 +824,103 @@ __device__ __forceinline__ void mma_tail_resident(const Params& p, const Hdr& h,
   }
 }
 
+// TAIL with formed records: token b's row in the stage is 64 bf16 hi values
+// then 64 bf16 lo values (256 bytes); two MMAs per k16 step.
+template <int NT>
+__device__ __forceinline__ void mma_tail_formed(const Hdr& h, const uint8_t* tile, const uint8_t* act,
+                                                float (&acc)[NT][4], float (&acc2)[NT][4], int warp,
+                                                int lane) {
+  const int g = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    if (b < h.nb) {
+      const uint4 a0 = lds128(tile + ((warp * 2 + b) * 2 + 0) * 512 + lane * 16);
+      const uint4 a1 = lds128(tile + ((warp * 2 + b) * 2 + 1) * 512 + lane * 16);
+      const uint32_t A0[4] = {a0.x, a0.y, a0.z, a0.w};
+      const uint32_t A1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        if (8 * t >= h.ntok) break;  // (uniform over the CTA)
+        const int tok = 8 * t + g < h.ntok ? 8 * t + g : 0;
+        const uint8_t* rec = act + tok * 256 + (32 * b + 8 * tig) * 2;
+        const uint4 bh = lds128(rec), bl = lds128(rec + 128);
+        mma_bf16(acc[t], A0, bh.x, bh.y);
+        mma_bf16(acc2[t], A1, bh.z, bh.w);
+        mma_bf16(acc[t], A0, bl.x, bl.y);
+        mma_bf16(acc2[t], A1, bl.z, bl.w);
+      }
+    }
+  }
+}
+
+// TAIL, staged activations: form the records (see Params::t_rec) for every
+// (chunk, token) -- this CTA's share of the grid-wide work, 8 values an item.
+__device__ __forceinline__ void form_tail_records(const Params& p, int tid) {
+  const int K = p.topk, klat = p.C_lat * 64;
+  const long long items = (long long)p.C * p.B * 8;
+  for (long long it = (long long)blockIdx.x * kConsumerThreads + tid; it < items;
+       it += (long long)gridDim.x * kConsumerThreads) {
+    const int c = (int)(it / (p.B * 8)), rem = (int)(it % (p.B * 8));
+    const int b = rem >> 3, q = rem & 7;
+    const int k0 = c * 64 + q * 8;  // K index of the chunk space ([L chunks ; I_s chunks])
+    float v[8];
+    if (c < p.C_lat) {
+      float4 ya[16], yb[16];
+      float wj[16];
+      const float* ybase = p.y + ((long long)c * p.ld_slots + (long long)b * K) * 64 + q * 8;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j < K) {
+          wj[j] = __ldcg(p.wts + b * K + j);
+          ya[j] = __ldcg(reinterpret_cast<const float4*>(ybase + j * 64));
+          yb[j] = __ldcg(reinterpret_cast<const float4*>(ybase + j * 64 + 4));
+        } else {
+          wj[j] = 0.f;
+          ya[j] = yb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v[0] = fmaf(wj[j], ya[j].x, v[0]);
+        v[1] = fmaf(wj[j], ya[j].y, v[1]);
+        v[2] = fmaf(wj[j], ya[j].z, v[2]);
+        v[3] = fmaf(wj[j], ya[j].w, v[3]);
+        v[4] = fmaf(wj[j], yb[j].x, v[4]);
+        v[5] = fmaf(wj[j], yb[j].y, v[5]);
+        v[6] = fmaf(wj[j], yb[j].z, v[6]);
+        v[7] = fmaf(wj[j], yb[j].w, v[7]);
+      }
+      if (k0 >= p.L) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = 0.f;
+      }
+    } else {
+      const int ks = k0 - klat;
+      if (ks < p.KS) {
+        const float* hb = p.h_s + ((long long)(ks >> 6) * p.B + b) * 64 + (ks & 63);
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(hb));
+        const float4 d = __ldcg(reinterpret_cast<const float4*>(hb + 4));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = 0.f;
+      }
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      hi[u] = pack_bf16x2(v[2 * u], v[2 * u + 1]);
+      lo[u] = pack_bf16x2(v[2 * u] - bf16_lo_to_float(hi[u]), v[2 * u + 1] - bf16_hi_to_float(hi[u]));
+    }
+    uint8_t* rec = p.t_rec + ((long long)c * p.B + b) * 256 + q * 16;
+    *reinterpret_cast<uint4*>(rec) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(rec + 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
 // TAIL: build the activation tile (combine of y, or h_s) as bf16 hi + lo in a
 // transform buffer, then bf16 MMAs against W_out / W_sd.
 template <int NT>
@@ -946,9 +1052,10 @@ __device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int wa
   named_sync(1, kConsumerThreads);
 }
 
-__device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
+__device__ __forceinline__ bool route_tokens(const Params& p, const float* bias, uint8_t* scratch,
                                           float* lg_s, int lg_cap, int* wtot, int tid, int warp,
-                                          int lane, const float* lg_sm = nullptr);
+                                          int lane, const float* lg_sm = nullptr, int b_lo = 0,
+                                          int b_hi = -1);
 
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&acc)[NT][4], uint8_t* scratch,
@@ -1097,10 +1204,15 @@ __device__ __forceinline__ void stage_floats(const float* src, int n, float* dst
 // lg_s: shared memory for lg_cap floats of logits (at least E).
 // lg_sm: the logits [B][E] already in shared memory (few tokens, summed by
 // the routing CTA itself), else they are read from p.logits.
-__device__ __forceinline__ void route_tokens(const Params& p, const float* bias, uint8_t* scratch,
+// [b_lo, b_hi): the tokens this CTA selects for (b_hi < 0: all).  With
+// several routing CTAs (p.route_cta > 1) each selects its share; the last to
+// finish (a ticket) gathers every token's choice and builds the tables, and
+// only it returns true (the caller then publishes them).
+__device__ __forceinline__ bool route_tokens(const Params& p, const float* bias, uint8_t* scratch,
                                           float* lg_s, int lg_cap, int* wtot, int tid, int warp,
-                                          int lane, const float* lg_sm) {
+                                          int lane, const float* lg_sm, int b_lo, int b_hi) {
   const int E = p.E, K = p.topk, B = p.B;
+  if (b_hi < 0) b_hi = B;
   const int tg = p.tg > 0 ? p.tg : 1;
   int* cnt = reinterpret_cast<int*>(scratch);  // [E] slots per expert
   int* fill = cnt + E;                          // [E] placement cursor
@@ -1120,14 +1232,14 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
   const int P = B >= kConsumerWarps ? 1 : kConsumerWarps / B;  // B * P <= 8 warps
   if (P == 1) {
     const bool staged = lg_cap >= E;  // (the ring always holds a token's logits)
-    const int chunk = staged ? min(B, lg_cap / E) : B;
-    for (int b0 = 0; b0 < B; b0 += chunk) {
-      const int nb = min(chunk, B - b0);
+    const int chunk = staged ? min(b_hi - b_lo, lg_cap / E) : b_hi - b_lo;
+    for (int b0 = b_lo; b0 < b_hi; b0 += chunk) {
+      const int nb = min(chunk, b_hi - b0);
       if (staged) {
         stage_floats(p.logits + (long long)b0 * E, nb * E, lg_s, tid);
         named_sync(1, kConsumerThreads);
       }
-      if (tr && b0 == 0) tr[21] = global_ns();
+      if (tr && b0 == b_lo) tr[21] = global_ns();
       for (int bl = warp; bl < nb; bl += kConsumerWarps) {
         const int b = b0 + bl;
         int sel_id;
@@ -1144,9 +1256,9 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
           ids_s[b * K + lane] = sel_id;
           atomicAdd(&cnt[sel_id], 1);
         }
-        if (tr && b0 == 0 && bl == 0) tr[22] = global_ns();
+        if (tr && b0 == b_lo && bl == 0) tr[22] = global_ns();
       }
-      if (tr && b0 == 0) tr[20] = global_ns();
+      if (tr && b0 == b_lo) tr[20] = global_ns();
       named_sync(1, kConsumerThreads);  // every warp is done with lg_s
     }
   } else {
@@ -1187,6 +1299,26 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
   }
   named_sync(1, kConsumerThreads);
   if (tr) tr[17] = global_ns();
+  if (p.route_cta > 1) {
+    // every CTA's ids precede its ticket (barrier cumulativity); the last
+    // one gathers all of them
+    int* flag = wtot + 16;
+    if (tid == 0) flag[0] = atom_add_acqrel(p.route_cnt, 1) == p.route_cta - 1;
+    named_sync(1, kConsumerThreads);
+    if (!flag[0]) return false;
+    for (int i = tid; i < E; i += kConsumerThreads) cnt[i] = 0;
+    named_sync(1, kConsumerThreads);
+    for (int sl = tid; sl < B * K; sl += kConsumerThreads) {
+      const int e = ld_cg(p.ids + sl);
+      ids_s[sl] = e;
+      atomicAdd(&cnt[e], 1);
+    }
+    if (tid == 0) {
+      *p.route_cnt = 0;    // every routing CTA has taken its ticket
+      *p.router_done = 0;  // ... so each has seen the router rows complete
+    }
+    named_sync(1, kConsumerThreads);
+  }
   // block-wide exclusive scan of (slots, token groups) per expert; thread t
   // owns experts 4t .. 4t+3 (E <= 1024)
   int c[4], gsz[4], sc = 0, sg = 0;
@@ -1263,6 +1395,7 @@ __device__ __forceinline__ void route_tokens(const Params& p, const float* bias,
     p.slots_sorted[pos] = s;
   }
   named_sync(1, kConsumerThreads);
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -1330,6 +1463,9 @@ __device__ __forceinline__ bool route_poll_logits(const Params& p, float* lgs, i
 __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, float* bias_s,
                                           int* sm_flag, int tid, int warp, int lane, int pstride) {
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
+  // the previous forward's tail is complete (this CTA waited for it): its
+  // record count starts again from zero
+  if (p.t_ready && tid == 0 && blockIdx.x == gridDim.x - 1) *p.t_ready = 0;
   // the selection bias is static: stage it in shared memory before the
   // logits exist, so the selection waits on one round trip, not two
   const float* bias = nullptr;
@@ -1371,11 +1507,16 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
   if (!sm_flag[0]) return;
   if (tr && tid == 0) tr[4] = global_ns();
-  route_tokens(p, bias, scratch, bias_s + bias_floats, ring_floats - bias_floats, sm_flag + 16,
-               tid, warp, lane);  // ends with a barrier
-  if (tid == 0) {
+  // this routing CTA's share of the tokens
+  const int R = p.route_cta;
+  const int r = (int)blockIdx.x - ((int)gridDim.x - R);
+  const int per = (p.B + R - 1) / R;
+  const int b_lo = min(p.B, r * per), b_hi = min(p.B, b_lo + per);
+  const bool last = route_tokens(p, bias, scratch, bias_s + bias_floats, ring_floats - bias_floats,
+                                 sm_flag + 16, tid, warp, lane, nullptr, b_lo, b_hi);
+  if (last && tid == 0) {
     if (tr) tr[5] = global_ns();
-    *p.router_done = 0;
+    if (R == 1) *p.router_done = 0;
     // every thread's table writes precede this release (barrier cumulativity)
     st_release(p.route_ready, 1);
   }
@@ -1530,6 +1671,11 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       build_resident(p, res, tid, kbeg, kend);
       named_sync(1, kConsumerThreads);
     }
+    if (KIND == KIND_TAIL && p.t_rec) {
+      form_tail_records(p, tid);
+      named_sync(1, kConsumerThreads);  // every thread's records precede the release
+      if (tid == 0) red_release_add(p.t_ready, 1);
+    }
   };
   bool dep_done = !lazy;
   if (lazy) {
@@ -1568,6 +1714,8 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       mma_mx<NT>(p, h, tile, act, acc, warp, lane);
     } else if (p.res_off) {
       mma_tail_resident<NT>(p, h, tile, res, acc, acc2, warp, lane);
+    } else if (p.t_rec) {
+      mma_tail_formed<NT>(h, tile, act, acc, acc2, warp, lane);
     } else {
       uint8_t* tbuf = scratch + 4096 + (nbuf & 1) * (16 * 320);
       ++nbuf;
@@ -1704,7 +1852,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     fence_mbar_init();
   }
   __syncthreads();
-  if (KIND == KIND_FRONT && p.route_cta && blockIdx.x == gridDim.x - 1) {
+  if (KIND == KIND_FRONT && p.route_cta && (int)blockIdx.x >= (int)gridDim.x - p.route_cta) {
     // it writes the routing tables the previous forward's tail reads
     pdl_wait();
     pdl_trigger();
@@ -1758,8 +1906,8 @@ static int set_attr(size_t bytes) {
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-// Token tiles (NT) each kind is built for: dense kinds up to 16 (128 tokens),
-// expert kinds up to 4 (groups of 32), the tail up to 2 (groups of 16); the
+// Token tiles (NT) each kind is built for: the front up to 16 (128 tokens),
+// expert kinds up to 4 (groups of 32), the tail up to 8 (passes of 64); the
 // front and tail also at one tile for two CTAs per SM (p.half_sm).
 template <int KIND>
 static int launch_kind_nt(int nt, const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
@@ -1771,11 +1919,9 @@ static int launch_kind_nt(int nt, const Params& p, int grid, size_t smem, cudaSt
   switch (nt) {
     case 1: return launch_one<KIND, 1>(p, grid, smem, s, pdl);
     case 2: return launch_one<KIND, 2>(p, grid, smem, s, pdl);
-    case 4:
-      if constexpr (KIND != KIND_TAIL) return launch_one<KIND, 4>(p, grid, smem, s, pdl);
-      break;
+    case 4: return launch_one<KIND, 4>(p, grid, smem, s, pdl);
     case 8:
-      if constexpr (kDense) return launch_one<KIND, 8>(p, grid, smem, s, pdl);
+      if constexpr (kDense || KIND == KIND_TAIL) return launch_one<KIND, 8>(p, grid, smem, s, pdl);
       break;
     case 16:
       if constexpr (kDense) return launch_one<KIND, 16>(p, grid, smem, s, pdl);
@@ -1787,9 +1933,9 @@ static int launch_kind_nt(int nt, const Params& p, int grid, size_t smem, cudaSt
 
 template <int KIND>
 static int set_attr_kind(size_t bytes) {
-  int e = set_attr<KIND, 1>(bytes) | set_attr<KIND, 2>(bytes);
-  if constexpr (KIND != KIND_TAIL) e |= set_attr<KIND, 4>(bytes);
-  if constexpr (KIND == KIND_FRONT) e |= set_attr<KIND, 8>(bytes) | set_attr<KIND, 16>(bytes);
+  int e = set_attr<KIND, 1>(bytes) | set_attr<KIND, 2>(bytes) | set_attr<KIND, 4>(bytes);
+  if constexpr (KIND == KIND_FRONT || KIND == KIND_TAIL) e |= set_attr<KIND, 8>(bytes);
+  if constexpr (KIND == KIND_FRONT) e |= set_attr<KIND, 16>(bytes);
   if constexpr (KIND == KIND_FRONT || KIND == KIND_TAIL) e |= set_attr<KIND, 1, 2>(bytes);
   return e;
 }

@@ -21,7 +21,7 @@ RESIDENT_MAX = 72 * KB
 SIDE_MAX_TOKENS = 4           # largest batch with the shared expert as a side lane
 INVALID_ARG, UNSUPPORTED = 1, 2  # moe_status codes
 # token-tile instantiations the library compiles, per kind
-TILES = {0: {1, 2, 4, 8, 16}, 1: {1, 2, 4}, 2: {1, 2, 4}, 3: {1, 2}, 4: {1}, 5: {1}}
+TILES = {0: {1, 2, 4, 8, 16}, 1: {1, 2, 4}, 2: {1, 2, 4}, 3: {1, 2, 4, 8}, 4: {1}, 5: {1}}
 
 
 def _cfg(shape, max_tokens=128):
