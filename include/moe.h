@@ -152,10 +152,19 @@ typedef struct moe_plan_info {
  *   MOE_NO_PDL=1            no programmatic dependent launch between kernels
  *   MOE_MAX_STAGES=n        ring depth cap, 2..8 (default 5)
  *   MOE_SPLIT_COST=n        split-K piece-end price in stages (default 2)
+ *   MOE_UMMA=0              expert kernels on the warp-level MMA (e2m1 decoded
+ *                           to f16, f16 activations with a power-of-two scale
+ *                           per 32) instead of the 5th-generation tensor cores
+ *                           (block-scaled e2m1 x e2m1 MMA, activations as four
+ *                           e2m1 terms); fixes the packed weight order, so it
+ *                           holds for the plan's life.  MOE_UMMA=0 also allows
+ *                           MOE_FUSED, which keeps the warp-level MMA
  *   MOE_EXPERT_CTAS_PER_SM=1  one CTA per SM for the expert kernels (default
- *                           2 at one token tile)
- *   MOE_EXPERT_SMALL_MAX_B=n  largest B with 8-token virtual experts (default
+ *                           2 at one token tile, and at two on the tensor cores)
+ *   MOE_EXPERT_SMALL_MAX_B=n  largest B with 8-token virtual experts (16-token
+ *                           ones on the tensor cores above B = 64; default
  *                           128; above it, 32-token groups)
+ *   MOE_EXPERT_TG=8|16|32   tokens per virtual expert for every B
  *   MOE_SIDE_LANE=0         no side lane, whatever shared_sms says
  *   MOE_TAIL_SPLIT=0        the tail's shared-expert part is not scheduled first
  *   MOE_Z_FLAG=0            expert gate/up waits for the whole front kernel
@@ -207,7 +216,8 @@ MOE_API moe_status moe_last_routing(moe_plan p, int32_t *ids_host, float *w_host
 /* Intermediates of the most recent forward, decoded to float32 (synchronises). */
 enum {
   MOE_DBG_LOGITS = 0, /* [B][E] router logits */
-  MOE_DBG_Z = 1,      /* [B][L] latent activations as stored for the experts */
+  MOE_DBG_Z = 1,      /* [B][L] latent activations as stored for the experts (f16 with a
+                         power-of-two scale per 32, or the sum of four e2m1 terms) */
   MOE_DBG_H = 2,      /* [B][k][I] expert SwiGLU outputs as stored for the down projection */
   MOE_DBG_Y = 3,      /* [B][k][L] expert outputs (before the weighted combine) */
   MOE_DBG_HS = 4      /* [B][I_s] shared-expert SwiGLU output */
@@ -266,7 +276,9 @@ MOE_API moe_status moe_set_profiling(moe_plan p, int32_t enable);
  *   19 ns the router logits of a row block were published, 21..22 routing
  *   CTA: slice selection end, merge end (8 or more tokens: logits staged,
  *   first token selected; 20: the first warp's tokens of the first staged
- *   group selected).
+ *   group selected); in the expert kernels' slots 20/21 producer cycles
+ *   setting stages up (header, weight tile) / copying activations, 22/23 the
+ *   tensor-core MMA warp's cycles waiting for stages / issuing.
  * Synchronises the device.
  */
 MOE_API moe_status moe_debug_trace(moe_plan p, uint64_t *host, int64_t count);

@@ -19,7 +19,7 @@ OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["moe_kernels.cu", "moe_k_front.cu", "moe_k_egu.cu", "moe_k_edn.cu",
            "moe_k_tail.cu", "moe_k_mega.cu", "moe_pack.cu", "moe_api.cu", "moe_static.cu"]
-HEADERS = ["ptx.cuh", "layout.cuh", "engine.cuh", "topk.cuh", "moe_engine.cuh", "moe_mega.cuh"]
+HEADERS = ["ptx.cuh", "layout.cuh", "engine.cuh", "topk.cuh", "umma.cuh", "moe_engine.cuh", "moe_mega.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",

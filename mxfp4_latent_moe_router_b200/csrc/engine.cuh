@@ -93,6 +93,13 @@ struct Params {
   // combine is formed per stage (the fused single launch).
   uint8_t* t_rec;
   int* t_ready;
+  // EGU/EDN on the 5th-generation tensor cores (block-scaled tcgen05 MMA,
+  // e2m1 weights x e4m3 activation terms): the packed tiles and the z / h
+  // records take the layouts of layout.cuh; FRONT and EGU write their
+  // records in that form.  0: the warp-level MMA; else nonzero, and at an
+  // expert kernel's launch the token tiles of its stages (its NT)
+  int umma;
+  int act_rec;  // bytes of one activation record (kActRecBytes or kActRecBytesU)
   // EGU: the latent row blocks' finalisations count up here (release); the
   // expert gate/up kernel reads z once it reaches RB_lat instead of waiting
   // for the whole front grid (whose last CTAs stream shared-expert rows)
@@ -179,6 +186,6 @@ int set_smem_limits(size_t bytes);
 int launch_pack_dense(const void* src, int K, int N, int layout, int RB, int C, int rows_valid,
                       uint8_t* dst, void* stream, const void* src2, int K2, int C_first);
 int launch_pack_mx(const uint8_t* codes, const uint8_t* scales, int E, int rows, int K,
-                   int layout, int RB, int C, uint8_t* dst, int* err, void* stream);
+                   int layout, int RB, int C, uint8_t* dst, int* err, void* stream, int umma);
 
 }  // namespace moe

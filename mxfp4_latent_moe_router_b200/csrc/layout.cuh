@@ -44,6 +44,38 @@ constexpr int kMxTileBytes = kMxCodeBytes + kMxScaleBytes;    // 17408
 // scales that undo it.  544 bytes, 16-byte multiple.
 constexpr int kActRecBytes = kMxChunkK * 2 + 8 * 4;
 
+// Tensor-core (tcgen05, kind::mxf4) layouts of the MXFP4 expert kernels,
+// selected per plan.  A weight tile keeps its 17408 bytes, reordered for the
+// block-scaled MMA's K-major "core matrices" (8 rows x 16 bytes, see
+// umma.cuh): the codes as 1024 slots of 16 bytes, slot (kb * 16 + rg) * 8 + r
+// holding row rg * 8 + r, K elements 32 kb .. 32 kb + 31 of the chunk (element
+// 2t in the low nibble of byte t), so that row groups lie 128 bytes apart and
+// K blocks 2048; then the e8m0 scales as two 512-byte units (K blocks 0-3,
+// 4-7), byte (m % 32) * 16 + (m / 32) * 4 + kb % 4.
+//
+// An activation record (per row, 256-wide chunk) holds the value as a sum of
+// kUTerms e2m1 terms, each with its own e8m0 scale per 32-block:
+//   value = sum_t e2m1(q_t) * 2^(s_t - 127),
+// term t's codes packed as 8 K blocks of 16 bytes (128 bytes), then the
+// terms' 8 scale bytes each.  Term 1 takes the block maximum to at most 4
+// times its scale, each later term a scale 2^-3 of the previous one, and
+// each carries what the earlier terms left: the residual after 4 terms is at
+// most 2^-11 of the block maximum.
+constexpr int kUTerms = 4;
+constexpr int kUTermBytes = kMxChunkK / 2;                      // 128
+constexpr int kActRecBytesU = kUTerms * kUTermBytes + kUTerms * 8;  // 544
+
+// A tensor-core ring stage: [header 128][A: packed codes 16 KB][A scales
+// 1 KB][B: kUTerms * 8 NT token-term rows of 128 bytes][B scales 1 KB]
+constexpr int kUHdrBytes = 128;
+constexpr int kUAOff = kUHdrBytes;
+constexpr int kUSfaOff = kUAOff + kMxCodeBytes;
+constexpr int kUBOff = kUSfaOff + kMxScaleBytes;
+__host__ __device__ constexpr int umma_rows(int nt) { return kUTerms * 8 * nt; }
+__host__ __device__ constexpr int umma_stage_bytes(int nt) {
+  return ((kUBOff + umma_rows(nt) * kUTermBytes + 1024) + 127) / 128 * 128;
+}
+
 // fragment map: lane (g,t), k16 step s, register q (0..3), half e (0..1) ->
 // (row within the 16-row warp tile, physical k within the 32-block)
 __host__ __device__ constexpr int frag_row(int g, int q) { return (q & 1) ? g + 8 : g; }

@@ -55,7 +55,7 @@ constexpr int kTailTg = 64;
 // at about the same time, so most re-reads can hit L2.  Groups of 32 (four
 // tiles, one CTA per SM) remain for batches above the environment variable
 // MOE_EXPERT_SMALL_MAX_B.
-constexpr int kExpertTgSmall = 8, kExpertTgLarge = 32;
+constexpr int kExpertTgSmall = 8, kExpertTgLarge = 32, kExpertTgUmmaLarge = 16;
 constexpr int kBigSmem = 227 * 1024;
 // two CTAs of the one-tile expert kernels share an SM (228 KB, 1 KB reserved
 // per CTA): twice the warps to hide the MXFP4 loop's latencies
@@ -127,6 +127,12 @@ struct moe_plan_s {
   // the routing CTA sums the router partials itself for few tokens
   // (environment MOE_DIRECT_ROUTE=0 turns it off)
   bool direct_route = true;
+  // expert kernels on the 5th-generation tensor cores (block-scaled MMA of
+  // e2m1 weights and e4m3 activation terms; environment MOE_UMMA=0 keeps
+  // the warp-level MMA): decides the expert tiles' packed order and the
+  // activation records' form, so it is fixed when the plan is made
+  bool umma = true;
+  int act_rec = kActRecBytesU;
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* out_stage = nullptr;
@@ -139,6 +145,7 @@ struct moe_plan_s {
   int max_stages = 5;  // ring depth cap (environment MOE_MAX_STAGES)
   int expert_per_sm_max = 2;     // environment MOE_EXPERT_CTAS_PER_SM
   int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
+  int expert_tg_fixed = 0;       // environment MOE_EXPERT_TG (8, 16 or 32; 0: by batch size)
   bool use_pdl = true;
   int fail_alloc_after = -1;     // environment MOE_FAIL_ALLOC_AFTER (tests only)
   int prod_sleep = 200, cons_sleep = 32;  // environment MOE_PROD_SLEEP / MOE_CONS_SLEEP (ns)
@@ -163,6 +170,12 @@ struct moe_plan_s {
 
 // tokens per virtual expert for a forward of B tokens
 int expert_tg(const moe_plan_s* p, int B) {
+  if (p->expert_tg_fixed) return p->expert_tg_fixed;
+  // the tensor-core kernels take 16-token groups above 64 tokens: two token
+  // tiles cost their MMAs little, and a popular expert's weights are read
+  // half as often (128 Zipf-skewed tokens: 578 vs 603 us per step; at 64
+  // near-uniform tokens, where few experts see more than 8, 536 vs 515)
+  if (p->umma && B > 64 && B <= p->expert_small_max_b) return kExpertTgUmmaLarge;
   return B <= p->expert_small_max_b ? kExpertTgSmall : kExpertTgLarge;
 }
 
@@ -237,6 +250,11 @@ SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int s
   if (kind == KIND_FRONT) {
     s.act_stride = 192;
     act = 8 * nt * s.act_stride;
+  } else if ((kind == KIND_EGU || kind == KIND_EDN) && p->umma) {
+    // tensor-core stage: unpacked codes, scales, the token-term rows
+    s.act_stride = 0;
+    s.act_off = kUBOff;
+    s.stage_bytes = umma_stage_bytes(nt);
   } else if (kind == KIND_EGU || kind == KIND_EDN) {
     s.act_stride = 576;
     act = 8 * nt * s.act_stride;
@@ -246,8 +264,10 @@ SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int s
     act = res_bytes ? 0 : formed ? tail_tg_eff * 256 : tail_tg_eff * std::max(1, topk) * 256;
   }
   const int tile = (kind == KIND_EGU || kind == KIND_EDN) ? kMxTileBytes : kDenseTileBytes;
-  s.act_off = kHdr + tile;
-  s.stage_bytes = ((kHdr + tile + act) + 127) / 128 * 128;
+  if (!((kind == KIND_EGU || kind == KIND_EDN) && p->umma)) {
+    s.act_off = kHdr + tile;
+    s.stage_bytes = ((kHdr + tile + act) + 127) / 128 * 128;
+  }
   // one CTA per SM (the whole shared memory for the ring): a running kernel
   // and the next one, launched early by programmatic dependent launch, never
   // share an SM; with the half budget, two CTAs of one expert kernel do
@@ -289,9 +309,11 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
   f.front_workers = p->num_sms - f.route_ctas;
   f.tail_grid = p->num_sms;
   f.expert_per_sm = 1;
-  if (f.nt_e == 1 && p->expert_per_sm_max >= 2) {
+  // (the tensor-core kernels: up to two token tiles, each CTA then holding
+  // half the SM's tensor memory)
+  if (f.nt_e <= (p->umma ? 2 : 1) && p->expert_per_sm_max >= 2) {
     const int slots = B * p->cfg.top_k;
-    const SmemGeom h = smem_geom(p, KIND_EGU, 1, 1, slots, 0, kHalfSmem);
+    const SmemGeom h = smem_geom(p, KIND_EGU, f.nt_e, 1, slots, 0, kHalfSmem);
     if (h.nstages >= 3 && h.total <= (size_t)kHalfSmem) f.expert_per_sm = 2;
   }
   f.expert_grid = p->num_sms * f.expert_per_sm;
@@ -354,6 +376,8 @@ Params base_params(const moe_plan_s* p, int B) {
   q.C_lat = p->C_lat;
   q.KS = c.shared_inter;
   q.scratch_off = kScratchOff;
+  q.umma = p->umma ? 1 : 0;
+  q.act_rec = p->act_rec;
   return q;
 }
 
@@ -541,6 +565,32 @@ void plan_shape(moe_plan_s* p) {
   p->ve_max = std::min(E, slots) + ceil_div(slots, kExpertTgSmall) + 1;  // any group size
 }
 
+// Tuning knobs and switches from the environment, read when a plan is made
+// (and by moe_debug_geometry, which reports what such a plan would launch).
+void read_env(moe_plan_s* p) {
+  if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
+  if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_EXPERT_TG")) {
+    const int v = atoi(e);
+    p->expert_tg_fixed = (v == 8 || v == 16 || v == 32) ? v : 0;
+  }
+  if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
+  if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
+  if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
+  if (const char* e = getenv("MOE_FAIL_ALLOC_AFTER")) p->fail_alloc_after = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_PROD_SLEEP")) p->prod_sleep = std::max(0, std::min(2000, atoi(e)));
+  if (const char* e = getenv("MOE_TAIL_SPLIT")) p->tail_split = atoi(e) != 0;
+  if (const char* e = getenv("MOE_Z_FLAG")) p->z_flag = atoi(e) != 0;
+  if (const char* e = getenv("MOE_SIDE_LANE")) p->side_env_off = atoi(e) == 0;
+  if (const char* e = getenv("MOE_PREFETCH_MB")) p->prefetch_bytes = std::max(0LL, (long long)atoi(e)) << 20;
+  if (const char* e = getenv("MOE_DIRECT_ROUTE")) p->direct_route = atoi(e) != 0;
+  if (const char* e = getenv("MOE_CONS_SLEEP")) p->cons_sleep = std::max(0, std::min(2000, atoi(e)));
+  if (const char* e = getenv("MOE_UMMA")) p->umma = atoi(e) != 0;
+  p->act_rec = p->umma ? kActRecBytesU : kActRecBytes;
+  if (p->umma) p->use_fused = false;  // the single launch keeps the warp-level MMA
+}
+
 // The control block (routing count, router-row count, error word, routing
 // flag, phase counts, per-kind piece cursors) and every kind's split-K
 // tickets back to zero, as a fresh plan has them.  Synchronous.
@@ -565,20 +615,7 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   CUDA_TRY(cudaGetDeviceProperties(&prop, device));
   if (prop.major != 10) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
   p->num_sms = prop.multiProcessorCount;
-  if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
-  if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
-  if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
-  if (const char* e = getenv("MOE_NO_PDL")) p->use_pdl = atoi(e) == 0;
-  if (const char* e = getenv("MOE_FUSED")) p->use_fused = atoi(e) != 0;
-  if (const char* e = getenv("MOE_MAX_STAGES")) p->max_stages = std::max(2, std::min(8, atoi(e)));
-  if (const char* e = getenv("MOE_FAIL_ALLOC_AFTER")) p->fail_alloc_after = std::max(0, atoi(e));
-  if (const char* e = getenv("MOE_PROD_SLEEP")) p->prod_sleep = std::max(0, std::min(2000, atoi(e)));
-  if (const char* e = getenv("MOE_TAIL_SPLIT")) p->tail_split = atoi(e) != 0;
-  if (const char* e = getenv("MOE_Z_FLAG")) p->z_flag = atoi(e) != 0;
-  if (const char* e = getenv("MOE_SIDE_LANE")) p->side_env_off = atoi(e) == 0;
-  if (const char* e = getenv("MOE_PREFETCH_MB")) p->prefetch_bytes = std::max(0LL, (long long)atoi(e)) << 20;
-  if (const char* e = getenv("MOE_DIRECT_ROUTE")) p->direct_route = atoi(e) != 0;
-  if (const char* e = getenv("MOE_CONS_SLEEP")) p->cons_sleep = std::max(0, std::min(2000, atoi(e)));
+  read_env(p);
   if (set_smem_limits(kBigSmem) != 0) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -608,12 +645,15 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
 
   TRY(alloc(p, &v, sizeof(float) * maxB * E, false));
   p->logits = (float*)v;
-  TRY(alloc(p, &v, (size_t)maxB * ceil_div(L, kMxChunkK) * kActRecBytes, false));
+  // (zeroed: the entries past L and I are never written and must read as 0)
+  TRY(alloc(p, &v, (size_t)maxB * ceil_div(L, kMxChunkK) * p->act_rec, false));
   p->z_mx = (uint8_t*)v;
+  CUDA_TRY(cudaMemset(v, 0, (size_t)maxB * ceil_div(L, kMxChunkK) * p->act_rec));
   TRY(alloc(p, &v, sizeof(float) * (size_t)ceil_div(std::max(Is, 1), 64) * maxB * 64, false));
   p->h_s = (float*)v;
-  TRY(alloc(p, &v, (size_t)ceil_div(I, kMxChunkK) * slots * kActRecBytes, false));
+  TRY(alloc(p, &v, (size_t)ceil_div(I, kMxChunkK) * slots * p->act_rec, false));
   p->h_mx = (uint8_t*)v;
+  CUDA_TRY(cudaMemset(v, 0, (size_t)ceil_div(I, kMxChunkK) * slots * p->act_rec));
   TRY(alloc(p, &v, sizeof(float) * (size_t)ceil_div(L, 64) * slots * 64, false));
   p->y = (float*)v;
   TRY(alloc(p, &v, sizeof(int) * slots, false));
@@ -888,6 +928,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     const SmemGeom sm = smem_geom(p, KIND_EGU, f.nt_e, tail_tg_eff, B * c.top_k, 0,
                                   f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
     set_kind(q, p, KIND_EGU, sm);
+    q.half_sm = f.expert_per_sm == 2 ? 1 : 0;
     q.piece_ctas = f.expert_grid;
     q.split_cost = split_cost_for(p, f.nt_e);
     TRY(launch_timed(p, KIND_EGU, KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s));
@@ -925,6 +966,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     const SmemGeom sm = smem_geom(p, KIND_EDN, f.nt_e, tail_tg_eff, B * c.top_k, 0,
                                   f.expert_per_sm == 2 ? kHalfSmem : kBigSmem);
     set_kind(q, p, KIND_EDN, sm);
+    q.half_sm = f.expert_per_sm == 2 ? 1 : 0;
     q.piece_ctas = f.expert_grid;
     q.split_cost = split_cost_for(p, f.nt_e);
     TRY(launch_timed(p, KIND_EDN, KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s));
@@ -1062,10 +1104,10 @@ moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
                                           Is > 0 ? w->sh_down : w->w_out, Is, p->C_lat));
   const KindGeom& eg = p->g[KIND_EGU];
   CUDA_TRY((cudaError_t)launch_pack_mx(w->gu_codes, w->gu_scales, E, 2 * I, L, 1, eg.RB, eg.C,
-                                       p->w_egu, p->err, s));
+                                       p->w_egu, p->err, s, p->umma ? 1 : 0));
   const KindGeom& ed = p->g[KIND_EDN];
   CUDA_TRY((cudaError_t)launch_pack_mx(w->dn_codes, w->dn_scales, E, L, I, 0, ed.RB, ed.C,
-                                       p->w_edn, p->err, s));
+                                       p->w_edn, p->err, s, p->umma ? 1 : 0));
   if (use_bias) {
     CUDA_TRY(cudaMemcpyAsync(p->bias, w->router_bias, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
   } else {
@@ -1151,6 +1193,33 @@ moe_status moe_last_routing(moe_plan p, int32_t* ids_host, float* w_host, int32_
   return MOE_OK;
 }
 
+// e2m1 code -> float: sign, 2 exponent bits (bias 1), 1 mantissa bit;
+// exponent 0 is subnormal (0 or 0.5)
+float e2m1_value(int code) {
+  const int e = (code >> 1) & 3, m = code & 1;
+  const float v = e == 0 ? 0.5f * m : std::ldexp(1.0f + 0.5f * m, e - 1);
+  return (code & 8) ? -v : v;
+}
+
+// element i (0..255) of one activation record, in either form (layout.cuh)
+float record_value(const moe_plan_s* p, const uint8_t* rec, int i) {
+  if (p->umma) {
+    float v = 0.f;
+    for (int t = 0; t < kUTerms; ++t) {
+      const uint8_t sb = rec[kUTerms * kUTermBytes + t * 8 + i / 32];
+      if (sb == 0xFF) return NAN;
+      const int code = (rec[t * kUTermBytes + i / 2] >> (4 * (i & 1))) & 15;
+      v += e2m1_value(code) * std::ldexp(1.0f, (int)sb - 127);
+    }
+    return v;
+  }
+  uint16_t hv;
+  float sc;
+  std::memcpy(&hv, rec + i * 2, 2);
+  std::memcpy(&sc, rec + 512 + 4 * (i / 32), 4);
+  return half_to_float(hv) * sc;
+}
+
 moe_status moe_debug_fetch(moe_plan p, int32_t what, int32_t num_tokens, float* host,
                            int64_t count) {
   if (!p || !host) return MOE_ERR_INVALID_ARG;
@@ -1170,23 +1239,19 @@ moe_status moe_debug_fetch(moe_plan p, int32_t what, int32_t num_tokens, float* 
     case MOE_DBG_Z: {
       if (count != (int64_t)B * L) return MOE_ERR_INVALID_ARG;
       const int cz = ceil_div(L, kMxChunkK);
-      std::vector<uint8_t> raw((size_t)B * cz * kActRecBytes);
+      std::vector<uint8_t> raw((size_t)B * cz * p->act_rec);
       CUDA_TRY(cudaMemcpy(raw.data(), p->z_mx, raw.size(), cudaMemcpyDeviceToHost));
       for (int b = 0; b < B; ++b)
         for (int l = 0; l < L; ++l) {
-          const uint8_t* rec = raw.data() + ((size_t)b * cz + l / kMxChunkK) * kActRecBytes;
-          uint16_t hv;
-          float sc;
-          std::memcpy(&hv, rec + (l % kMxChunkK) * 2, 2);
-          std::memcpy(&sc, rec + 512 + 4 * ((l % kMxChunkK) / 32), 4);
-          host[(size_t)b * L + l] = half_to_float(hv) * sc;
+          const uint8_t* rec = raw.data() + ((size_t)b * cz + l / kMxChunkK) * p->act_rec;
+          host[(size_t)b * L + l] = record_value(p, rec, l % kMxChunkK);
         }
       return MOE_OK;
     }
     case MOE_DBG_H: {
       if (count != (int64_t)slots * I) return MOE_ERR_INVALID_ARG;
       const int ci = ceil_div(I, kMxChunkK);
-      std::vector<uint8_t> raw((size_t)ci * slots * kActRecBytes);
+      std::vector<uint8_t> raw((size_t)ci * slots * p->act_rec);
       std::vector<int> sorted(slots);
       CUDA_TRY(cudaMemcpy(raw.data(), p->h_mx, raw.size(), cudaMemcpyDeviceToHost));
       CUDA_TRY(cudaMemcpy(sorted.data(), p->slots_sorted, sizeof(int) * slots, cudaMemcpyDeviceToHost));
@@ -1194,12 +1259,8 @@ moe_status moe_debug_fetch(moe_plan p, int32_t what, int32_t num_tokens, float* 
         const int slot = sorted[pos];
         if (slot < 0 || slot >= slots) return MOE_ERR_RANGE;
         for (int i = 0; i < I; ++i) {
-          const uint8_t* rec = raw.data() + ((size_t)(i / kMxChunkK) * slots + pos) * kActRecBytes;
-          uint16_t hv;
-          float sc;
-          std::memcpy(&hv, rec + (i % kMxChunkK) * 2, 2);
-          std::memcpy(&sc, rec + 512 + 4 * ((i % kMxChunkK) / 32), 4);
-          host[(size_t)slot * I + i] = half_to_float(hv) * sc;
+          const uint8_t* rec = raw.data() + ((size_t)(i / kMxChunkK) * slots + pos) * p->act_rec;
+          host[(size_t)slot * I + i] = record_value(p, rec, i % kMxChunkK);
         }
       }
       return MOE_OK;
@@ -1290,6 +1351,7 @@ moe_status moe_debug_geometry(const moe_config* cfg, int32_t num_sms, int32_t nu
   if (!p) return MOE_ERR_OOM;
   p->cfg = *cfg;
   p->num_sms = num_sms;
+  read_env(p);
   plan_shape(p);
   const moe_config& c = p->cfg;
   const int B = num_tokens, K = c.top_k;

@@ -48,10 +48,12 @@
 #include "layout.cuh"
 #include "ptx.cuh"
 #include "topk.cuh"
+#include "umma.cuh"
 
 namespace moe {
 
 constexpr int kHdrBytes = 128;
+static_assert(kHdrBytes == kUHdrBytes, "tensor-core stages share the header size");
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMaxStages = 8;
 constexpr int kTraceStride = 24;  // u64 per CTA in the optional trace
@@ -230,7 +232,7 @@ __device__ __forceinline__ void chunk_header(const Params& p, int c, int c_first
   if (KIND == KIND_FRONT)
     ab = h.ntok * h.nb * 64;
   else if (KIND == KIND_EGU || KIND == KIND_EDN)
-    ab = h.ntok * kActRecBytes;
+    ab = h.ntok * p.act_rec;
   else
     ab = p.res_off ? 0 : p.t_rec ? h.ntok * 256 : ((c < p.C_lat) ? h.ntok * p.topk * 256 : h.ntok * 256);
   h.act_bytes = ab;
@@ -252,7 +254,8 @@ __device__ __forceinline__ const uint8_t* weight_src(const Params& p, const Hdr&
 // copies have landed and lane 0 has arrived.
 constexpr int kBulkRowsMax = 8;
 template <int KIND>
-__device__ __forceinline__ bool rows_async(const Hdr& h) {
+__device__ __forceinline__ bool rows_async(const Params& p, const Hdr& h) {
+  if ((KIND == KIND_EGU || KIND == KIND_EDN) && p.umma) return true;  // scattered into the MMA's B layout
   return (KIND == KIND_FRONT || KIND == KIND_EGU || KIND == KIND_EDN) && h.ntok > kBulkRowsMax;
 }
 
@@ -261,14 +264,25 @@ template <int KIND>
 __device__ __forceinline__ void stage_begin(const Params& p, const Hdr& h, uint8_t* sb, uint64_t* bar) {
   constexpr int kTile = KindTraits<KIND>::kTileBytes;
   *reinterpret_cast<Hdr*>(sb) = h;
-  // a slot whose activations once came in 16-byte copies may now take a bulk
-  // copy: order the two proxies' writes
-  if ((KIND == KIND_FRONT || KIND == KIND_EGU || KIND == KIND_EDN) && p.B > kBulkRowsMax)
+  // A slot's activation rows come in 16-byte copies for stages of more than
+  // kBulkRowsMax rows and in bulk copies otherwise.  Only the warp-level
+  // expert kernels with token groups above that size can mix the two in one
+  // launch: there a slot's earlier copies are ordered before the next bulk
+  // copy into it.  (The front kernel's stages all hold the same B rows; the
+  // tensor-core stages fill each region one way.)
+  if ((KIND == KIND_EGU || KIND == KIND_EDN) && !p.umma && p.tg > kBulkRowsMax)
     fence_proxy_async_smem();
-  if (rows_async<KIND>(h))
+  if (rows_async<KIND>(p, h))
     mbar_expect_tx(bar, kTile);  // lane 0 arrives once the rows are issued
   else
     mbar_arrive_expect_tx(bar, kTile + h.act_bytes);
+  if (KindTraits<KIND>::kMx && p.umma) {
+    // the packed codes as the A operand, the scales behind them
+    const uint8_t* src = weight_src<KIND>(p, h);
+    bulk_g2s(sb + kUAOff, src, kMxCodeBytes, bar);
+    bulk_g2s(sb + kUSfaOff, src + kMxCodeBytes, kMxScaleBytes, bar);
+    return;
+  }
   bulk_g2s(sb + kHdrBytes, weight_src<KIND>(p, h), kTile, bar);
 }
 
@@ -311,23 +325,62 @@ __device__ __forceinline__ void copy_records_async(uint8_t* act, int stride, int
   rows_async_done(bar, lane);
 }
 
+// Tensor-core stage: every token's kUTerms term rows into the B operand's
+// core-matrix layout (row n = term * 8 NT + token; K block kb of row n at
+// (kb * ng + n / 8) * 128 + (n % 8) * 16, ng = rows / 8) and their scales into
+// the two 512-byte units; 16- and 4-byte copies spread over the producer
+// lanes.  nt: the kernel's token tiles.
+template <int KIND>
+__device__ __forceinline__ void copy_records_umma(const Params& p, const Hdr& h, uint8_t* sb,
+                                                  uint64_t* bar, int lane, const int* slot_tab,
+                                                  int nt) {
+  const int rows = umma_rows(nt), ng = rows / 8, per_tok = 8 * nt;
+  uint8_t* B = sb + kUBOff;
+  uint8_t* sfb = B + rows * kUTermBytes;
+  const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
+  constexpr int kPerTerm = kMxChunkK / 32 + 2;  // 8 K blocks of 16 bytes, 2 scale words
+  constexpr int kPerTok = kUTerms * kPerTerm;
+  const int items = h.ntok * kPerTok;
+  for (int it = lane; it < items; it += 32) {
+    const int tok = it / kPerTok, rem = it - tok * kPerTok;
+    const int t = rem / kPerTerm, q = rem - t * kPerTerm;
+    const uint8_t* rec;
+    if (KIND == KIND_EGU)
+      rec = p.z_mx + ((long long)(slot_tab[h.tok0 + tok] / p.topk) * cz + h.chunk) * p.act_rec;
+    else
+      rec = p.h_mx + ((long long)h.chunk * p.ld_slots + h.tok0 + tok) * p.act_rec;
+    const int n = t * per_tok + tok;
+    if (q < kPerTerm - 2) {
+      cp_async16(B + (q * ng + (n >> 3)) * 128 + (n & 7) * 16, rec + t * kUTermBytes + q * 16);
+    } else {
+      const int u = q - (kPerTerm - 2);
+      cp_async4(sfb + u * 512 + (n & 31) * 16 + (n >> 5) * 4, rec + kUTerms * kUTermBytes + t * 8 + u * 4);
+    }
+  }
+  rows_async_done(bar, lane);
+}
+
 // Issue this stage's activation copies (all 32 producer lanes).
 template <int KIND>
 __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t* act, uint64_t* bar,
                                           int lane, const int* slot_tab) {
-  if (rows_async<KIND>(h)) {
+  if ((KIND == KIND_EGU || KIND == KIND_EDN) && p.umma) {
+    copy_records_umma<KIND>(p, h, act - p.act_off, bar, lane, slot_tab, p.umma);  // (umma = NT)
+    return;
+  }
+  if (rows_async<KIND>(p, h)) {
     if (KIND == KIND_FRONT) {
       const uint8_t* x = reinterpret_cast<const uint8_t*>(p.x + h.chunk * kDenseChunkK);
       copy_x_rows_async(act, p.act_stride, h.ntok, h.nb == 2 ? 3 : 2, x, (long long)p.H * 2, bar, lane);
     } else if (KIND == KIND_EGU) {
       // lane r: token row of slot r (a virtual expert holds at most 32 slots)
       const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
-      const uint8_t* mine = p.z_mx + (long long)h.chunk * kActRecBytes;
-      if (lane < h.ntok) mine += (long long)(slot_tab[h.tok0 + lane] / p.topk) * cz * kActRecBytes;
+      const uint8_t* mine = p.z_mx + (long long)h.chunk * p.act_rec;
+      if (lane < h.ntok) mine += (long long)(slot_tab[h.tok0 + lane] / p.topk) * cz * p.act_rec;
       copy_records_async(act, p.act_stride, h.ntok, mine, true, bar, lane);
     } else {
       copy_records_async(act, p.act_stride, h.ntok,
-                         p.h_mx + ((long long)h.chunk * p.ld_slots + h.tok0) * kActRecBytes, false,
+                         p.h_mx + ((long long)h.chunk * p.ld_slots + h.tok0) * p.act_rec, false,
                          bar, lane);
     }
     return;
@@ -480,7 +533,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   // start where the first pieces need none): CTAs that land early (while the
   // previous kernel's last CTAs still run) would otherwise take several
   // pieces each before the late ones can start, and finish last.
-  long long pw = 0, pi = 0, nst = 0;
+  long long pw = 0, pi = 0, nst = 0, pb = 0, pa = 0;
   int grabbed = 0;
   bool in_flight = false;
   const int workers = (int)gridDim.x - (KIND == KIND_FRONT ? p.route_cta : 0);
@@ -507,8 +560,11 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       chunk_header<KIND>(p, c, c_first, c_last, h);
       if (lane == 0) stage_begin<KIND>(p, h, sb, &full[stage]);
       __syncwarp();
+      const long long tb = clock64();
+      pb += tb - tw1;
       if (waited || !h.dep) {
         issue_act<KIND>(p, h, sb + p.act_off, &full[stage], lane, slot_tab);
+        pa += clock64() - tb;
       } else {
         if (prefetched == 0) pend_first = stage;
         ++prefetched;
@@ -533,6 +589,10 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
     tr[11] = (unsigned long long)pw;
     tr[12] = (unsigned long long)pi;
     tr[13] = (unsigned long long)nst;
+    if (KIND == KIND_EGU || KIND == KIND_EDN) {  // (slots the routing uses in the front kernel)
+      tr[20] = (unsigned long long)pb;
+      tr[21] = (unsigned long long)pa;
+    }
   }
   // end marker
   if (!mbar_wait_bounded(&empty[stage], ephase, p.err, ERR_WAIT_EMPTY, p.prod_sleep)) return;
@@ -1052,6 +1112,106 @@ __device__ __forceinline__ void store_f16mx(const float (&val)[NT][2][2], int wa
   named_sync(1, kConsumerThreads);
 }
 
+// The tensor-core record (layout.cuh): per 32-block of a token, kUTerms e2m1
+// terms.  The block maximum a sets term 1's exponent e1, the least with
+// a <= 4 * 2^e1; term t + 1 takes 2^(e1 - 3 t).  Every element's term code is
+// its remaining value over the term's scale rounded to e2m1, and that code's
+// value comes off the remainder (which stays within 4 times the next scale).
+//
+// The tile's values go through shared memory, two token tiles at a time
+// ([token][row], row stride padded to 4 mod 32 floats: conflict-free on both
+// sides); then four adjacent threads take one (token, 32-row block), eight
+// rows each, and store each term's eight codes as one word.
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// SWIGLU: the tile has 64 rows, row 8 warp + g of token column col holding
+// silu(acc[t][c]) * acc[t][2 + c] (the expert gate/up kernel); otherwise 128
+// rows, rows 16 warp + g and + 8 holding acc[t][c] and acc[t][2 + c].  Token
+// column col's record is rec0 + col * col_stride; the tile's row r sits at
+// position pos0 + r of the record (pos0 a multiple of 32), and rows from
+// nrows on lie beyond K (not stored).
+template <int NT, bool SWIGLU>
+__device__ __forceinline__ void store_e2m1_terms(const float (&acc)[NT][4], int warp, int lane, int tid,
+                                                 int ntok, float* sv, uint8_t* rec0,
+                                                 long long col_stride, int pos0, int nrows) {
+  constexpr int kRows = SWIGLU ? 64 : 128;
+  constexpr int kLd = kRows + 4;
+  constexpr int kChunk = NT < 2 ? NT : 2;  // token tiles staged at a time
+  constexpr int kBlocks = kRows / 32;
+  const int g = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int t0 = 0; t0 < NT; t0 += kChunk) {
+    // this chunk's values into shared memory
+#pragma unroll
+    for (int tt = 0; tt < kChunk; ++tt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int tok = 8 * tt + 2 * tig + c;
+        const int t = t0 + tt;
+        if (SWIGLU) {
+          sv[tok * kLd + 8 * warp + g] = silu(acc[t][c]) * acc[t][2 + c];
+        } else {
+          sv[tok * kLd + 16 * warp + g] = acc[t][c];
+          sv[tok * kLd + 16 * warp + g + 8] = acc[t][2 + c];
+        }
+      }
+    named_sync(1, kConsumerThreads);
+    // four threads a (token, block): quarter q holds rows 8 q .. 8 q + 7
+    const int q = tid & 3, grp = tid >> 2;
+    const int blk = grp % kBlocks, tokl = grp / kBlocks;
+    const bool active = tokl < 8 * kChunk;
+    const int tok = 8 * t0 + (active ? tokl : 0);
+    const int r0 = 32 * blk + 8 * q;
+    float v[8];
+    float a = 0.f;
+    {
+      const float4* src = reinterpret_cast<const float4*>(sv + (active ? tokl : 0) * kLd + r0);
+      const float4 x0 = src[0], x1 = src[1];
+      v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+      v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (r0 + i >= nrows) v[i] = 0.f;
+        a = fmaxf(a, fabsf(v[i]));
+      }
+    }
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    // e1: the least e with a <= 4 * 2^e (kept where every term's scale and
+    // its inverse are normal floats); a NaN or infinite maximum makes every
+    // scale NaN
+    const bool nan = (__float_as_uint(a) & 0x7F800000u) == 0x7F800000u;
+    int e1 = -118;
+    if (a > 0.f && !nan) {
+      const uint32_t bits = __float_as_uint(a * 0.25f);
+      e1 = (int)((bits >> 23) & 0xFF) - 127 + ((bits & 0x7FFFFFu) ? 1 : 0);
+      e1 = e1 < -118 ? -118 : (e1 > 126 ? 126 : e1);
+    }
+    const bool store = active && tok < ntok && 32 * blk < nrows;
+    uint8_t* r = rec0 + (long long)tok * col_stride;
+    const int pos = pos0 + r0;
+#pragma unroll
+    for (int term = 0; term < kUTerms; ++term) {
+      const int e = e1 - 3 * term;
+      const float inv = pow2f(-e), sc = pow2f(e);
+      uint32_t w = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t code = f32_to_e2m1(v[i] * inv);
+        v[i] -= e2m1_to_f32(code) * sc;
+        w |= code << (4 * i);
+      }
+      if (store) *reinterpret_cast<uint32_t*>(r + term * kUTermBytes + (pos >> 1)) = w;
+    }
+    if (store && q == 0) {
+#pragma unroll
+      for (int term = 0; term < kUTerms; ++term)
+        r[kUTerms * kUTermBytes + term * 8 + (pos >> 5)] = nan ? (uint8_t)0xFF : (uint8_t)(e1 - 3 * term + 127);
+    }
+    named_sync(1, kConsumerThreads);  // (the staging is reused)
+  }
+}
+
 __device__ __forceinline__ bool route_tokens(const Params& p, const float* bias, uint8_t* scratch,
                                           float* lg_s, int lg_cap, int* wtot, int tid, int warp,
                                           int lane, const float* lg_sm = nullptr, int b_lo = 0,
@@ -1080,20 +1240,27 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
     // latent rows -> z records
     const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
     const int l0 = (h.rb - p.RB_router) * kRowsPerBlock + 16 * warp + g;
-    const int idx[2] = {l0, l0 + 8};
-    float val[NT][2][2];
-    uint8_t* rec[NT][2];
+    if (p.umma) {
+      const int lb = (h.rb - p.RB_router) * kRowsPerBlock;  // the tile's first latent row
+      store_e2m1_terms<NT, false>(acc, warp, lane, tid, p.B, reinterpret_cast<float*>(scratch),
+                                  p.z_mx + (long long)(lb >> 8) * p.act_rec, (long long)cz * p.act_rec,
+                                  lb & (kMxChunkK - 1), p.L - lb);  // ends with a barrier
+    } else {
+      const int idx[2] = {l0, l0 + 8};
+      float val[NT][2][2];
+      uint8_t* rec[NT][2];
 #pragma unroll
-    for (int t = 0; t < NT; ++t)
+      for (int t = 0; t < NT; ++t)
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        val[t][c][0] = acc[t][c];
-        val[t][c][1] = acc[t][2 + c];
-        const int col = 8 * t + 2 * tig + c;
-        rec[t][c] = p.z_mx + ((long long)(col < p.B ? col : 0) * cz + (l0 >> 8)) * kActRecBytes;
-      }
-    store_f16mx<NT, 2>(val, warp, lane, 2, p.B, reinterpret_cast<float*>(scratch), rec, idx,
-                       l0 < p.L, l0 + 8 < p.L);  // ends with a barrier
+        for (int c = 0; c < 2; ++c) {
+          val[t][c][0] = acc[t][c];
+          val[t][c][1] = acc[t][2 + c];
+          const int col = 8 * t + 2 * tig + c;
+          rec[t][c] = p.z_mx + ((long long)(col < p.B ? col : 0) * cz + (l0 >> 8)) * p.act_rec;
+        }
+      store_f16mx<NT, 2>(val, warp, lane, 2, p.B, reinterpret_cast<float*>(scratch), rec, idx,
+                         l0 < p.L, l0 + 8 < p.L);  // ends with a barrier
+    }
     if (p.done && tid == 0) red_release_add(p.done + 0, 1);
     // every thread's records precede the release (barrier cumulativity)
     if (p.z_done && tid == 0) red_release_add(p.z_done, 1);
@@ -1114,21 +1281,28 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
     }
   } else if (KIND == KIND_EGU) {
     const int i = 64 * h.rb + 8 * warp + g;
-    const int idx[2] = {i, i};
-    float val[NT][2][2];
-    uint8_t* rec[NT][2];
+    if (p.umma) {
+      const int ib = 64 * h.rb;  // the tile's first h row
+      store_e2m1_terms<NT, true>(acc, warp, lane, tid, h.ntok, reinterpret_cast<float*>(scratch),
+                                 p.h_mx + ((long long)(ib >> 8) * p.ld_slots + h.tok0) * p.act_rec,
+                                 (long long)p.act_rec, ib & (kMxChunkK - 1), p.I - ib);  // ends with a barrier
+    } else {
+      const int idx[2] = {i, i};
+      float val[NT][2][2];
+      uint8_t* rec[NT][2];
 #pragma unroll
-    for (int t = 0; t < NT; ++t)
+      for (int t = 0; t < NT; ++t)
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        val[t][c][0] = silu(acc[t][c]) * acc[t][2 + c];
-        val[t][c][1] = 0.f;
-        const int col = 8 * t + 2 * tig + c;
-        const int pos = h.tok0 + (col < h.ntok ? col : 0);
-        rec[t][c] = p.h_mx + ((long long)(i >> 8) * p.ld_slots + pos) * kActRecBytes;
-      }
-    store_f16mx<NT, 1>(val, warp, lane, 4, h.ntok, reinterpret_cast<float*>(scratch), rec, idx,
-                       i < p.I, false);  // ends with a barrier
+        for (int c = 0; c < 2; ++c) {
+          val[t][c][0] = silu(acc[t][c]) * acc[t][2 + c];
+          val[t][c][1] = 0.f;
+          const int col = 8 * t + 2 * tig + c;
+          const int pos = h.tok0 + (col < h.ntok ? col : 0);
+          rec[t][c] = p.h_mx + ((long long)(i >> 8) * p.ld_slots + pos) * p.act_rec;
+        }
+      store_f16mx<NT, 1>(val, warp, lane, 4, h.ntok, reinterpret_cast<float*>(scratch), rec, idx,
+                         i < p.I, false);  // ends with a barrier
+    }
     if (p.done && tid == 0) red_release_add(p.done + 2, 1);
   } else if (KIND == KIND_EDN) {
 #pragma unroll
@@ -1621,7 +1795,158 @@ __device__ __forceinline__ void finalize(const Params& p, const Hdr& h, float (&
   epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
 }
 
-template <int KIND, int NT>
+// ---------------------------------------------------------------------------
+// expert kernels on the 5th-generation tensor cores (p.umma = token tiles)
+//
+// Warp roles: the producer streams stages as for the warp-level MMA; one MMA
+// warp (its lane 0) issues each stage's four K = 64 block-scaled MMAs
+// (e2m1 weights x the activation's e2m1 terms) and releases the stage when
+// they complete; the eight consumer warps take each finished piece's sums
+// out of tensor memory and run the split-K and epilogue logic.  Two
+// accumulator buffers let the MMAs of the next piece run meanwhile.
+//
+// Tensor memory of a CTA: accumulator buffer b at columns N b, 128 rows x
+// (N = kUTerms x 8 NT token terms); then per ring slot s 16 columns of
+// scales at 2 N + 16 s: the weights' at +0, the activations' at +8, each two
+// 4-column units (K blocks 0-3, 4-7).  A slot's scales are rewritten only
+// after the MMAs that read them have completed (they release the slot).
+// Up to two token tiles the CTA takes 256 columns (two CTAs can share an
+// SM), at four 512.
+template <int NT>
+__host__ __device__ constexpr uint32_t tmem_dcols() { return (uint32_t)umma_rows(NT); }
+template <int NT>
+__host__ __device__ constexpr uint32_t tmem_sf() { return 2 * tmem_dcols<NT>(); }
+template <int NT>
+__host__ __device__ constexpr uint32_t tmem_cols() { return NT <= 2 ? 256u : 512u; }
+static_assert(tmem_sf<1>() + 16 * kMaxStages <= tmem_cols<1>(), "scale columns of every ring slot");
+static_assert(tmem_sf<2>() + 16 * kMaxStages <= tmem_cols<2>(), "scale columns of every ring slot");
+static_assert(tmem_sf<4>() + 16 * kMaxStages <= tmem_cols<4>(), "scale columns of every ring slot");
+// shared-memory handover: tensor-memory base at flag word kUTmemWord,
+// accumulator-full barriers (MMA completion + the header's release) at words
+// kUDfullWord + 2 b, accumulator-free barriers at kUDfreeWord + 2 b, the MMA
+// warp's drain barrier at kUDrainWord; the finished pieces' headers at the
+// end of the scratch area
+constexpr int kUTmemWord = 48, kUDfullWord = 50, kUDfreeWord = 54, kUDrainWord = 58;
+constexpr int kUPqOff = 19456;
+static_assert(2 * sizeof(Hdr) <= 1024, "two piece headers behind the consumers' scratch");
+constexpr int kThreadsU = kThreads + 32;  // + the MMA warp
+constexpr int kMmaWarp = kConsumerWarps + 1;
+
+template <int NT>
+__device__ void mma_issuer(const Params& p, uint8_t* stage_base, uint64_t* full, uint64_t* empty,
+                           uint64_t* dfull, uint64_t* dfree, uint64_t* drain, Hdr* pq, uint32_t tmem) {
+  constexpr int kRows = umma_rows(NT), kNg = kRows / 8;
+  int stage = 0, buf = 0;
+  uint32_t phase = 0, uses[2] = {0u, 0u};
+  long long mw = 0, mi = 0, t0 = clock64();
+  while (true) {
+    if (!mbar_wait_bounded(&full[stage], phase, p.err, ERR_WAIT_FULL, p.cons_sleep)) break;
+    const long long t1 = clock64();
+    mw += t1 - t0;
+    const uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
+    const Hdr h = *reinterpret_cast<const Hdr*>(sb);
+    const bool first = (h.flags & HDR_FIRST) != 0;
+    // a piece's first stage overwrites its accumulator buffer (and the end
+    // mark its header): the consumers must have read the piece before last
+    // out of it
+    if ((first || (h.flags & HDR_END)) &&
+        !mbar_wait_bounded(&dfree[buf], (uses[buf] & 1u) ^ 1u, p.err, ERR_WAIT_FULL, p.cons_sleep))
+      break;
+    if (h.flags & HDR_END) {
+      pq[buf] = h;
+      mbar_arrive(&dfull[buf]);
+      mbar_arrive(&dfull[buf]);
+      break;
+    }
+    fence_proxy_async_smem();  // the activation rows came in by cp.async
+    umma::fence_after_sync();
+    const uint8_t* A = sb + kUAOff;
+    const uint8_t* B = sb + kUBOff;
+    const uint32_t sfa_t = tmem + tmem_sf<NT>() + 16u * (uint32_t)stage, sfb_t = sfa_t + 8;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      umma::cp_scales(sfa_t + 4 * u, umma::smem_desc(sb + kUSfaOff + 512 * u, 128, 128));
+      umma::cp_scales(sfb_t + 4 * u, umma::smem_desc(B + kRows * kUTermBytes + 512 * u, 128, 128));
+    }
+    const uint32_t d = tmem + (uint32_t)buf * tmem_dcols<NT>();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint64_t ad = umma::smem_desc(A + j * 4096, 2048, 128);
+      const uint64_t bd = umma::smem_desc(B + j * 2 * kNg * 128, kNg * 128, 128);
+      umma::mma_mxf4(d, ad, bd, umma::idesc_mxf4(128, kRows, 2 * (j & 1), 2 * (j & 1)),
+                     sfa_t + 4 * (j >> 1), sfb_t + 4 * (j >> 1), !(first && j == 0));
+    }
+    umma::commit(&empty[stage]);  // the slot is free once these MMAs have read it
+    if (h.flags & HDR_LAST) {
+      pq[buf] = h;
+      umma::commit(&dfull[buf]);  // the sums are complete ...
+      mbar_arrive(&dfull[buf]);   // ... and the header is written
+      ++uses[buf];
+      buf ^= 1;
+    }
+    if (++stage == p.nstages) {
+      stage = 0;
+      phase ^= 1;
+    }
+    t0 = clock64();
+    mi += t0 - t1;
+  }
+  if (p.trace) {
+    unsigned long long* tr = p.trace + (size_t)blockIdx.x * kTraceStride;
+    tr[22] = (unsigned long long)mw;
+    tr[23] = (unsigned long long)mi;
+  }
+  // MMAs cut short by an error may still run: drain them before the tensor
+  // memory is given back
+  umma::commit(drain);
+  mbar_wait_bounded(drain, 0, p.err, ERR_WAIT_FULL, p.cons_sleep);
+}
+
+// A finished piece's sums out of tensor memory into the MMA-fragment
+// registers the epilogues take: warps 0-3 read their 32 rows (lane quarter
+// = warp), add the kUTerms terms of each token and stage the sums in shared
+// memory (128 rows x 8 NT tokens); the buffer is then released to the MMA
+// warp and every warp picks its fragment.
+template <int NT>
+__device__ __forceinline__ void umma_read_acc(uint32_t d, float* stage_s, float (&acc)[NT][4], int warp,
+                                             int lane, int tid, uint64_t* dfree_bar) {
+  umma::fence_after_sync();
+  constexpr int kTok = 8 * NT, kLd = kTok + 1;  // (row stride padded: no bank conflicts)
+  if (warp < 4) {
+    const int row = 32 * warp + lane;
+    const uint32_t lane_addr = d + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+    for (int c = 0; c < NT; ++c) {
+      float sum[8], t[8];
+      umma::ld_32x32b_x8(lane_addr + 8 * c, sum);
+      umma::wait_ld();
+#pragma unroll
+      for (int term = 1; term < kUTerms; ++term) {
+        umma::ld_32x32b_x8(lane_addr + term * kTok + 8 * c, t);
+        umma::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum[i] += t[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) stage_s[row * kLd + 8 * c + i] = sum[i];
+    }
+  }
+  umma::fence_before_sync();
+  named_sync(1, kConsumerThreads);
+  if (tid == 0) mbar_arrive(dfree_bar);
+  const int g = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = 8 * t + 2 * tig + (q & 1);
+      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+      acc[t][q] = stage_s[row * kLd + col];
+    }
+  named_sync(1, kConsumerThreads);
+}
+
+template <int KIND, int NT, bool UM>
 __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, uint64_t* empty,
                          uint8_t* scratch, int* sm_flag, const int* slot_tab, int warp, int lane) {
   const int tid = warp * 32 + lane;
@@ -1637,7 +1962,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   // issues the atomic after the piece's partials are written and reads its
   // result only at the next piece end, so nobody waits on the round trip.
   bool pend = false;
-  Hdr pend_h;
+  Hdr pend_h{};
   int ticket = 0;
   int* tflag = sm_flag + 4;  // two alternating slots
   int tslot = 0;
@@ -1690,47 +2015,15 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
   int n_pieces = 0, n_fin = 0;
   long long c_wait = 0, c_comp = 0, c_end = 0, t_a = clock64();
-  while (true) {
-    if (!mbar_wait_bounded(&full[stage], phase, p.err, ERR_WAIT_FULL, p.cons_sleep)) break;
-    long long t_b = clock64();
-    c_wait += t_b - t_a;
-    uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
-    const Hdr h = *reinterpret_cast<const Hdr*>(sb);
-    if (tr && tid == 0 && n_pieces == 0 && (h.flags & HDR_FIRST)) tr[6] = global_ns();
-    if (h.flags & HDR_END) break;
-    if (lazy && !dep_done && h.dep) {
-      tail_dep(0, klat);  // the first latent stage: y, and the combine, need the expert phases
-      dep_done = true;
-    }
-    if (h.flags & HDR_FIRST) {
-      zero_acc(acc);
-      zero_acc(acc2);
-    }
-    const uint8_t* tile = sb + kHdrBytes;
-    const uint8_t* act = sb + p.act_off;
-    if (KIND == KIND_FRONT) {
-      mma_dense_x<NT>(p, h, tile, act, acc, acc2, warp, lane);
-    } else if (KIND == KIND_EGU || KIND == KIND_EDN) {
-      mma_mx<NT>(p, h, tile, act, acc, warp, lane);
-    } else if (p.res_off) {
-      mma_tail_resident<NT>(p, h, tile, res, acc, acc2, warp, lane);
-    } else if (p.t_rec) {
-      mma_tail_formed<NT>(h, tile, act, acc, acc2, warp, lane);
-    } else {
-      uint8_t* tbuf = scratch + 4096 + (nbuf & 1) * (16 * 320);
-      ++nbuf;
-      mma_tail<NT>(p, h, tile, act, tbuf, acc, acc2, warp, lane, tid);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
-    if (++stage == p.nstages) {
-      stage = 0;
-      phase ^= 1;
-    }
-    t_a = clock64();
-    c_comp += t_a - t_b;
-    if (!(h.flags & HDR_LAST)) continue;
-    ++n_pieces;
+  // tensor-core expert kernels: tensor memory base, the handover barriers
+  // and the finished pieces' headers
+  const uint32_t tmem = UM ? *reinterpret_cast<volatile uint32_t*>(sm_flag + kUTmemWord) : 0u;
+  uint64_t* dfull = reinterpret_cast<uint64_t*>(sm_flag + kUDfullWord);
+  uint64_t* dfree = reinterpret_cast<uint64_t*>(sm_flag + kUDfreeWord);
+  const Hdr* pq = reinterpret_cast<const Hdr*>(scratch + kUPqOff);
+  // a piece's sums are in acc (+ acc2): split-K partials, tickets,
+  // finalisation, epilogue
+  auto piece_done = [&](const Hdr& h) {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
@@ -1745,12 +2038,12 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       const long long t_c = clock64();
       c_end += t_c - t_a;
       t_a = t_c;
-      continue;
+      return;
     }
     if (h.ppr == 1) {
       ++n_fin;
       epilogue<KIND, NT>(p, h, acc, scratch, sm_flag, slot_tab, tid, warp, lane);
-      continue;
+      return;
     }
     write_partial<NT>(p, h.piece, h.ntok, acc, warp, lane);
     if ((KIND == KIND_FRONT) && h.rb < p.RB_router) {
@@ -1779,7 +2072,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       const long long t_c = clock64();
       c_end += t_c - t_a;
       t_a = t_c;
-      continue;
+      return;
     }
     if (tid == 0 && pend) tflag[tslot] = (ticket == pend_h.ppr - 1);
     named_sync(1, kConsumerThreads);  // every warp's partials precede thread 0's release
@@ -1798,6 +2091,73 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
     const long long t_c = clock64();
     c_end += t_c - t_a;
     t_a = t_c;
+  };
+  if constexpr (UM) {
+    // tensor-core expert kernels: the MMA warp hands over each finished
+    // piece (its header in pq, its sums in accumulator buffer buf)
+    int buf = 0;
+    uint32_t uses[2] = {0u, 0u};
+    while (true) {
+      if (!mbar_wait_bounded(&dfull[buf], uses[buf] & 1u, p.err, ERR_WAIT_FULL, p.cons_sleep)) break;
+      long long t_b = clock64();
+      c_wait += t_b - t_a;
+      const Hdr h = pq[buf];
+      if (h.flags & HDR_END) break;
+      if (tr && tid == 0 && n_pieces == 0) tr[6] = global_ns();
+      zero_acc(acc2);
+      umma_read_acc<NT>(tmem + (uint32_t)buf * tmem_dcols<NT>(), reinterpret_cast<float*>(scratch), acc, warp,
+                        lane, tid, &dfree[buf]);
+      ++uses[buf];
+      buf ^= 1;
+      t_a = clock64();
+      c_comp += t_a - t_b;
+      ++n_pieces;
+      piece_done(h);
+    }
+  } else {
+    while (true) {
+      if (!mbar_wait_bounded(&full[stage], phase, p.err, ERR_WAIT_FULL, p.cons_sleep)) break;
+      long long t_b = clock64();
+      c_wait += t_b - t_a;
+      uint8_t* sb = stage_base + (size_t)stage * p.stage_bytes;
+      const Hdr h = *reinterpret_cast<const Hdr*>(sb);
+      if (tr && tid == 0 && n_pieces == 0 && (h.flags & HDR_FIRST)) tr[6] = global_ns();
+      if (h.flags & HDR_END) break;
+      if (lazy && !dep_done && h.dep) {
+        tail_dep(0, klat);  // the first latent stage: y, and the combine, need the expert phases
+        dep_done = true;
+      }
+      if (h.flags & HDR_FIRST) {
+        zero_acc(acc);
+        zero_acc(acc2);
+      }
+      const uint8_t* tile = sb + kHdrBytes;
+      const uint8_t* act = sb + p.act_off;
+      if (KIND == KIND_FRONT) {
+        mma_dense_x<NT>(p, h, tile, act, acc, acc2, warp, lane);
+      } else if (KIND == KIND_EGU || KIND == KIND_EDN) {
+        mma_mx<NT>(p, h, tile, act, acc, warp, lane);
+      } else if (p.res_off) {
+        mma_tail_resident<NT>(p, h, tile, res, acc, acc2, warp, lane);
+      } else if (p.t_rec) {
+        mma_tail_formed<NT>(h, tile, act, acc, acc2, warp, lane);
+      } else {
+        uint8_t* tbuf = scratch + 4096 + (nbuf & 1) * (16 * 320);
+        ++nbuf;
+        mma_tail<NT>(p, h, tile, act, tbuf, acc, acc2, warp, lane, tid);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == p.nstages) {
+        stage = 0;
+        phase ^= 1;
+      }
+      t_a = clock64();
+      c_comp += t_a - t_b;
+      if (!(h.flags & HDR_LAST)) continue;
+      ++n_pieces;
+      piece_done(h);
+    }
   }
   if (pend) {
     if (tid == 0) tflag[tslot] = (ticket == pend_h.ppr - 1);
@@ -1822,8 +2182,10 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
 // MINB: CTAs per SM the instantiation is compiled for.  Two for the expert
 // kernels at one token tile, and for the one-tile front and tail variants the
 // side lane uses (a CTA of each lane on one SM); one otherwise.
-template <int KIND, int NT, int MINB>
-__global__ void __launch_bounds__(kThreads, MINB)
+// UM: the expert kernels' tensor-core instantiation (its own kernel, so that
+// neither variant's registers are sized for the other's code).
+template <int KIND, int NT, int MINB, bool UM>
+__global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
     moe_kernel(const __grid_constant__ Params p) {
   // shared memory: [0,128) full barriers, [128,256) empty barriers,
   // [256,512) flags, [scratch_off, ...) scratch, [table_off, ...) routing
@@ -1844,14 +2206,35 @@ __global__ void __launch_bounds__(kThreads, MINB)
     for (int i = 2; i < kTraceStride; ++i) tr[i] = 0;
     tr[14] = smid();
   }
+  // tensor-core expert kernels: a stage is released by the commit of its
+  // MMAs (one arrival); an accumulator buffer is full once its MMAs have
+  // completed and the MMA warp has written the piece's header (two
+  // arrivals), free once the consumers have read it (one); tensor memory for
+  // the accumulators and the scales
+  static_assert(!UM || KIND == KIND_EGU || KIND == KIND_EDN, "tensor-core path: expert kernels only");
+  constexpr bool um = UM;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm_flag + kUTmemWord);
+  uint64_t* dfull = reinterpret_cast<uint64_t*>(sm_flag + kUDfullWord);
+  uint64_t* dfree = reinterpret_cast<uint64_t*>(sm_flag + kUDfreeWord);
+  uint64_t* drain = reinterpret_cast<uint64_t*>(sm_flag + kUDrainWord);
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.nstages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], um ? 1 : kConsumerWarps);
+    }
+    if (um) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&dfull[b], 2);
+        mbar_init(&dfree[b], 1);
+      }
+      mbar_init(drain, 1);
     }
     fence_mbar_init();
   }
+  if (um && warp == 0) umma::tmem_alloc(tmem_slot, tmem_cols<NT>());
+  if (um) umma::fence_before_sync();
   __syncthreads();
+  if (um) umma::fence_after_sync();
   if (KIND == KIND_FRONT && p.route_cta && (int)blockIdx.x >= (int)gridDim.x - p.route_cta) {
     // it writes the routing tables the previous forward's tail reads
     pdl_wait();
@@ -1861,10 +2244,19 @@ __global__ void __launch_bounds__(kThreads, MINB)
                 NT * 8 * kRowsPerBlock);
   } else if (warp == kConsumerWarps) {
     producer<KIND>(p, ctl, stages, tables, full, empty, lane);
+  } else if (UM && warp == kMmaWarp) {
+    if (lane == 0)
+      mma_issuer<NT>(p, stages, full, empty, dfull, dfree, drain,
+                     reinterpret_cast<Hdr*>(scratch + kUPqOff), *tmem_slot);
   } else {
-    consumer<KIND, NT>(p, stages, full, empty, scratch, sm_flag, slot_tab, warp, lane);
+    consumer<KIND, NT, UM>(p, stages, full, empty, scratch, sm_flag, slot_tab, warp, lane);
   }
+  if (um) umma::fence_before_sync();
   __syncthreads();
+  if (um && warp == 0) {
+    umma::fence_after_sync();
+    umma::tmem_dealloc(*tmem_slot, tmem_cols<NT>());
+  }
   if (p.trace && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 1] = global_ns();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -1884,12 +2276,12 @@ constexpr int default_minb() {
   return (KIND == KIND_EGU || KIND == KIND_EDN) && NT == 1 ? 2 : 1;
 }
 
-template <int KIND, int NT, int MINB = default_minb<KIND, NT>()>
+template <int KIND, int NT, int MINB = default_minb<KIND, NT>(), bool UM = false>
 static int launch_one(const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
-  auto kfn = moe_kernel<KIND, NT, MINB>;
+  auto kfn = moe_kernel<KIND, NT, MINB, UM>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(UM ? kThreadsU : kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1900,9 +2292,9 @@ static int launch_one(const Params& p, int grid, size_t smem, cudaStream_t s, bo
   return (int)cudaLaunchKernelEx(&cfg, kfn, p);
 }
 
-template <int KIND, int NT, int MINB = default_minb<KIND, NT>()>
+template <int KIND, int NT, int MINB = default_minb<KIND, NT>(), bool UM = false>
 static int set_attr(size_t bytes) {
-  return (int)cudaFuncSetAttribute(moe_kernel<KIND, NT, MINB>,
+  return (int)cudaFuncSetAttribute(moe_kernel<KIND, NT, MINB, UM>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
@@ -1910,8 +2302,24 @@ static int set_attr(size_t bytes) {
 // expert kinds up to 4 (groups of 32), the tail up to 8 (passes of 64); the
 // front and tail also at one tile for two CTAs per SM (p.half_sm).
 template <int KIND>
-static int launch_kind_nt(int nt, const Params& p, int grid, size_t smem, cudaStream_t s, bool pdl) {
+static int launch_kind_nt(int nt, const Params& p0, int grid, size_t smem, cudaStream_t s, bool pdl) {
   constexpr bool kDense = (KIND == KIND_FRONT);
+  // the tensor-core expert stages are laid out for the instantiation's tiles
+  Params p = p0;
+  if constexpr (KIND == KIND_EGU || KIND == KIND_EDN) {
+    if (p.umma) {
+      // half_sm: two CTAs an SM (up to two token tiles)
+      p.umma = nt;
+      switch (nt) {
+        case 1: return p.half_sm ? launch_one<KIND, 1, 2, true>(p, grid, smem, s, pdl)
+                                 : launch_one<KIND, 1, 1, true>(p, grid, smem, s, pdl);
+        case 2: return p.half_sm ? launch_one<KIND, 2, 2, true>(p, grid, smem, s, pdl)
+                                 : launch_one<KIND, 2, 1, true>(p, grid, smem, s, pdl);
+        case 4: return p.half_sm ? (int)cudaErrorInvalidValue : launch_one<KIND, 4, 1, true>(p, grid, smem, s, pdl);
+        default: return (int)cudaErrorInvalidValue;
+      }
+    }
+  }
   constexpr bool kHalf = (KIND == KIND_FRONT || KIND == KIND_TAIL);
   if constexpr (kHalf) {
     if (p.half_sm) return nt == 1 ? launch_one<KIND, 1, 2>(p, grid, smem, s, pdl) : (int)cudaErrorInvalidValue;
@@ -1937,6 +2345,10 @@ static int set_attr_kind(size_t bytes) {
   if constexpr (KIND == KIND_FRONT || KIND == KIND_TAIL) e |= set_attr<KIND, 8>(bytes);
   if constexpr (KIND == KIND_FRONT) e |= set_attr<KIND, 16>(bytes);
   if constexpr (KIND == KIND_FRONT || KIND == KIND_TAIL) e |= set_attr<KIND, 1, 2>(bytes);
+  if constexpr (KIND == KIND_EGU || KIND == KIND_EDN)
+    e |= set_attr<KIND, 1, 1, true>(bytes) | set_attr<KIND, 2, 1, true>(bytes) |
+         set_attr<KIND, 4, 1, true>(bytes) | set_attr<KIND, 1, 2, true>(bytes) |
+         set_attr<KIND, 2, 2, true>(bytes);
   return e;
 }
 

@@ -80,9 +80,59 @@ __device__ __forceinline__ int mx_src_row(int layout, int rb, int row_in_block, 
   return row;
 }
 
+// The tensor-core tile order (layout.cuh): unit v < 1024 is code slot v (16
+// bytes: 32 K elements of one row), unit 1024 + i the scale bytes 16 i ..
+// 16 i + 15.
+__device__ __forceinline__ void pack_mx_umma_unit(const uint8_t* ce, const uint8_t* se, int layout,
+                                                  int rb, int c, int rows, int rows_half, int K,
+                                                  int v, uint8_t* tdst, int* err) {
+  const int kb_total = K / 32;
+  uint8_t out[16];
+  if (v < 1024) {
+    const int r = v & 7, rg = (v >> 3) & 15, kb = v >> 7;
+    bool valid;
+    const int sr = mx_src_row(layout, rb, rg * 8 + r, rows_half, rows, valid);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int k = c * kMxChunkK + kb * 32 + 2 * j;
+      out[j] = (valid && k < K) ? ce[(long long)sr * (K / 2) + k / 2] : 0;
+    }
+    uint4 o;
+    o.x = out[0] | (out[1] << 8) | (out[2] << 16) | ((uint32_t)out[3] << 24);
+    o.y = out[4] | (out[5] << 8) | (out[6] << 16) | ((uint32_t)out[7] << 24);
+    o.z = out[8] | (out[9] << 8) | (out[10] << 16) | ((uint32_t)out[11] << 24);
+    o.w = out[12] | (out[13] << 8) | (out[14] << 16) | ((uint32_t)out[15] << 24);
+    *reinterpret_cast<uint4*>(tdst + v * 16) = o;
+    return;
+  }
+  const int o0 = (v - 1024) * 16;  // byte offset in the two 512-byte units
+  const int unit = o0 >> 9, m0 = (o0 & 511) >> 4;
+  int bad = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int m = m0 + 32 * (j >> 2), kb = 4 * unit + (j & 3);
+    const int blk = c * 8 + kb;
+    bool valid;
+    const int sr = mx_src_row(layout, rb, m, rows_half, rows, valid);
+    uint8_t sv = 127;
+    if (valid && blk < kb_total) {
+      sv = se[(long long)sr * kb_total + blk];
+      if (sv == 0xFF) bad = 1;
+    }
+    out[j] = sv;
+  }
+  if (bad) atomicOr(err, 1 << ERR_NAN_SCALE);
+  uint4 o;
+  o.x = out[0] | (out[1] << 8) | (out[2] << 16) | ((uint32_t)out[3] << 24);
+  o.y = out[4] | (out[5] << 8) | (out[6] << 16) | ((uint32_t)out[7] << 24);
+  o.z = out[8] | (out[9] << 8) | (out[10] << 16) | ((uint32_t)out[11] << 24);
+  o.w = out[12] | (out[13] << 8) | (out[14] << 16) | ((uint32_t)out[15] << 24);
+  *reinterpret_cast<uint4*>(tdst + kMxCodeBytes + o0) = o;
+}
+
 __global__ void pack_mx_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                                int E, int rows, int K, int layout, int RB, int C,
-                               uint8_t* __restrict__ dst, int* err) {
+                               uint8_t* __restrict__ dst, int* err, int umma) {
   const int rows_half = rows / 2;  // gate/up: I
   const long long per_tile = 1024 + 64;
   const long long units = (long long)E * RB * C * per_tile;
@@ -97,6 +147,10 @@ __global__ void pack_mx_kernel(const uint8_t* __restrict__ codes, const uint8_t*
     const uint8_t* ce = codes + (long long)e * rows * (K / 2);
     const uint8_t* se = scales + (long long)e * rows * kb_total;
     uint8_t* tdst = dst + tile * kMxTileBytes;
+    if (umma) {
+      pack_mx_umma_unit(ce, se, layout, rb, c, rows, rows_half, K, v, tdst, err);
+      continue;
+    }
     uint8_t out[16];
     if (v < 1024) {
       const int lane = v & 31, bp = (v >> 5) & 3, w = v >> 7;
@@ -155,13 +209,13 @@ int launch_pack_dense(const void* src, int K, int N, int layout, int RB, int C, 
 }
 
 int launch_pack_mx(const uint8_t* codes, const uint8_t* scales, int E, int rows, int K, int layout,
-                   int RB, int C, uint8_t* dst, int* err, void* stream) {
+                   int RB, int C, uint8_t* dst, int* err, void* stream, int umma) {
   const long long units = (long long)E * RB * C * (1024 + 64);
   const int threads = 256;
   long long nb = (units + threads - 1) / threads;
   if (nb > 65535LL * 16) nb = 65535LL * 16;
   pack_mx_kernel<<<(int)nb, threads, 0, (cudaStream_t)stream>>>(codes, scales, E, rows, K, layout,
-                                                                 RB, C, dst, err);
+                                                                 RB, C, dst, err, umma);
   return (int)cudaGetLastError();
 }
 

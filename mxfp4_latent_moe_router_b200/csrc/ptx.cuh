@@ -3,6 +3,7 @@
 // launch, warp-level MMA and the e2m1 pair conversion.
 #pragma once
 #include <cstdint>
+#include <cuda_fp16.h>
 
 namespace moe {
 
@@ -80,6 +81,10 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 // and lowers it when this lane's earlier copies have landed.
 __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src_gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
@@ -199,6 +204,23 @@ __device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&r)[4]) 
       " cvt.rn.f16x2.e2m1x2 %2, q2;\n cvt.rn.f16x2.e2m1x2 %3, q3;\n}"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
       : "r"(w));
+}
+
+// fp32 -> e2m1 code (round to nearest even, saturating at +-6), and the
+// value of a code (exact)
+__device__ __forceinline__ uint32_t f32_to_e2m1(float v) {
+  uint32_t r;
+  asm("{\n .reg .b8 q;\n cvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n cvt.u32.u8 %0, q;\n}"
+      : "=r"(r)
+      : "f"(0.f), "f"(v));
+  return r & 0xFu;
+}
+__device__ __forceinline__ float e2m1_to_f32(uint32_t code) {
+  uint32_t h;
+  asm("{\n .reg .b8 q0, q1, q2, q3;\n mov.b32 {q0, q1, q2, q3}, %1;\n cvt.rn.f16x2.e2m1x2 %0, q0;\n}"
+      : "=r"(h)
+      : "r"(code & 0xFu));
+  return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

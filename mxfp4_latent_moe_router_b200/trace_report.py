@@ -26,6 +26,11 @@ START, END, PIECES, FINALIZES, ROUTE_START, ROUTE_END, FIRST_STAGE, FIN_NS = 0, 
 CONS_WAIT, CONS_COMP, CONS_END, PROD_WAIT, PROD_ISSUE, PROD_STAGES, SM = 8, 9, 10, 11, 12, 13, 14
 ROUTE_CLEARED, ROUTE_SELECTED, ROUTE_SCANNED, LOGITS_PUBLISHED = 16, 17, 18, 19
 ROUTE_FIRST_GROUP, ROUTE_STAGED, ROUTE_FIRST_TOKEN = 20, 21, 22
+# expert kernels (slots the front kernel's routing uses): producer cycles in
+# stage set-up (header, weight tile copies) and in the activation copies; the
+# tensor-core MMA warp's waiting and issuing cycles
+PROD_BEGIN, PROD_ACT, MMA_WAIT, MMA_ISSUE = 20, 21, 22, 23
+EXPERT_KERNELS = ("expert_gate_up", "expert_down")
 
 
 def summarize(trace: np.ndarray, names, clock_ghz: float = 1.965) -> list[dict]:
@@ -60,6 +65,9 @@ def summarize(trace: np.ndarray, names, clock_ghz: float = 1.965) -> list[dict]:
             "consumer_us": {"wait": cyc(CONS_WAIT), "compute": cyc(CONS_COMP), "close": cyc(CONS_END)},
             "producer_us": {"wait": cyc(PROD_WAIT), "issue": cyc(PROD_ISSUE)},
             "stages_median": float(np.median(r[:, PROD_STAGES])),
+            **({"producer_split_us": {"begin": cyc(PROD_BEGIN), "act": cyc(PROD_ACT)},
+                "mma_warp_us": {"wait": cyc(MMA_WAIT), "issue": cyc(MMA_ISSUE)}}
+               if name in EXPERT_KERNELS else {}),
             "distinct_sms": int(len(set(r[:, SM].tolist()))),
         }
         route = np.where(rows[:, ROUTE_START] > 0)[0]
@@ -91,6 +99,10 @@ def format_summary(rows: list[dict]) -> str:
         lines.append("    consumer wait %.1f compute %.1f close %.1f | producer wait %.1f issue %.1f (µs, median CTA)"
                      % (s["consumer_us"]["wait"], s["consumer_us"]["compute"], s["consumer_us"]["close"],
                         s["producer_us"]["wait"], s["producer_us"]["issue"]))
+        if "producer_split_us" in s:
+            lines.append("    producer set-up %.1f activations %.1f | MMA warp wait %.1f issue %.1f (µs, median CTA)"
+                         % (s["producer_split_us"]["begin"], s["producer_split_us"]["act"],
+                            s["mma_warp_us"]["wait"], s["mma_warp_us"]["issue"]))
         if "routing_us" in s:
             r = s["routing_us"]
             f = lambda v: "-" if v is None else "%.1f" % v  # noqa: E731

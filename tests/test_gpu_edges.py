@@ -78,16 +78,19 @@ def test_fused_launch_with_staged_tail(monkeypatch):
                                seed=91, scale_exp_lo=-5, scale_exp_hi=-2)
     w = synth.make_weights(shape)
     monkeypatch.setenv("MOE_FUSED", "1")
+    monkeypatch.setenv("MOE_UMMA", "0")  # (the fused launch keeps the warp-level MMA)
     _check(shape, w, synth.make_x(shape), max_tokens=8)
 
 
+@pytest.mark.parametrize("umma", ["1", "0"])
 @pytest.mark.parametrize("B,E,k", [(24, 8, 4), (48, 4, 3)])
-def test_thirty_two_token_expert_groups(B, E, k, monkeypatch):
+def test_thirty_two_token_expert_groups(B, E, k, umma, monkeypatch):
     # with 8-token groups switched off, an expert's slots form groups of up to
     # 32 tokens: ~12 per expert in one group, or 36 per expert in groups of
     # 32 and 4.  The expert kernels run four token tiles at one CTA per SM
     # and gather more than 8 activation rows per stage with 16-byte copies.
     monkeypatch.setenv("MOE_EXPERT_SMALL_MAX_B", "0")
+    monkeypatch.setenv("MOE_UMMA", umma)
     shape = synth.custom_shape("tg32", B, 256, 256, E, k, 256, 64, synth.SCORE_SOFTMAX,
                                seed=101 + B, scale_exp_lo=-5, scale_exp_hi=-2)
     w = synth.make_weights(shape)

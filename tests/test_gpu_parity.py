@@ -82,6 +82,19 @@ def full_check(blk: GpuBlock, x, tokens=None, intermediates=True):
     return out, res, near
 
 
+# Launch modes chosen when a plan is made: the expert kernels on the
+# tensor cores (the default), on the warp-level MMA, and the single fused
+# launch (which keeps the warp-level MMA)
+MODES = {"umma": {"MOE_UMMA": "1", "MOE_FUSED": "0"},
+         "warp": {"MOE_UMMA": "0", "MOE_FUSED": "0"},
+         "fused": {"MOE_UMMA": "0", "MOE_FUSED": "1"}}
+
+
+def set_mode(monkeypatch, mode):
+    for k, v in MODES[mode].items():
+        monkeypatch.setenv(k, v)
+
+
 # ---------------------------------------------------------------------------
 # small shapes: several tiles, ragged tails, every branch
 
@@ -129,12 +142,12 @@ def test_zero_input_gives_exact_zero(tiny):
     np.testing.assert_allclose(wts, 0.5, rtol=0, atol=1e-7)
 
 
-@pytest.mark.parametrize("fused", [0, 1])
-def test_back_to_back_forwards_read_their_own_inputs(tiny, fused, monkeypatch):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_back_to_back_forwards_read_their_own_inputs(tiny, mode, monkeypatch):
     """Two forwards on one stream with different x: a read hoisted above a
     dependency wait would pick up the other step's activations."""
     shape, w = tiny
-    monkeypatch.setenv("MOE_FUSED", str(fused))
+    set_mode(monkeypatch, mode)
     blk = GpuBlock(shape, w, max_tokens=8)
     xa = synth.make_x(shape, tokens=8, step=100)
     xb = synth.make_x(shape, tokens=8, step=101)
@@ -150,10 +163,10 @@ def test_back_to_back_forwards_read_their_own_inputs(tiny, fused, monkeypatch):
         assert_close(bf16_to_f32(o.cpu().numpy().view(np.uint16)), ref["out"], "out")
 
 
-@pytest.mark.parametrize("fused", [0, 1])
-def test_deterministic_and_graph_replay(tiny, fused, monkeypatch):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_deterministic_and_graph_replay(tiny, mode, monkeypatch):
     shape, w = tiny
-    monkeypatch.setenv("MOE_FUSED", str(fused))
+    set_mode(monkeypatch, mode)
     blk = GpuBlock(shape, w, max_tokens=8)
     x = torch.from_numpy(synth.make_x(shape, tokens=8, step=7).view(np.int16)).cuda()
     o1, o2, o3 = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
@@ -216,9 +229,10 @@ def test_fused_launch_matches_multi_kernel_path(tiny, B, monkeypatch):
     The split-K piece boundaries differ, so agreement is to rounding."""
     shape, w = tiny
     x = synth.make_x(shape, tokens=B, step=40 + B)
-    monkeypatch.setenv("MOE_FUSED", "1")
+    set_mode(monkeypatch, "fused")
     fused = GpuBlock(shape, w, max_tokens=8)
     monkeypatch.delenv("MOE_FUSED")
+    monkeypatch.delenv("MOE_UMMA")
     assert fused.plan.info().kernels_per_forward == 1
     multi = GpuBlock(shape, w, max_tokens=8)
     assert multi.plan.info().kernels_per_forward == 4
@@ -231,6 +245,32 @@ def test_fused_launch_matches_multi_kernel_path(tiny, B, monkeypatch):
     ids_f, w_f = fused.plan.routing(B)
     ids_m, w_m = multi.plan.routing(B)
     assert np.array_equal(np.sort(ids_f, axis=1), np.sort(ids_m, axis=1))
+
+
+@pytest.mark.parametrize("case", ["tiny1", "tiny13", "tiny16", "ragged3", "ragged1"])
+def test_expert_mma_paths_agree(tiny, case, monkeypatch):
+    """The expert kernels on the tensor cores (e2m1 x three e4m3 terms of the
+    activations, block-scaled) and on the warp-level MMA (e2m1 decoded to
+    f16 x f16 activations): each within tolerance of the oracle, step by
+    step, and of each other."""
+    if case.startswith("tiny"):
+        shape, w = tiny
+        B = int(case[4:])
+        x = synth.make_x(shape, tokens=B, step=60 + B)
+    else:
+        k = int(case[6:])
+        shape = synth.custom_shape("ragged", 5, 96, 96, 10, k, 96, 32, synth.SCORE_SIGMOID,
+                                   seed=31 + k, scale_exp_lo=-5, scale_exp_hi=-2)
+        w = synth.make_weights(shape)
+        x = synth.make_x(shape, tokens=37, step=5)
+    outs = {}
+    for mode in ("umma", "warp"):
+        set_mode(monkeypatch, mode)
+        blk = GpuBlock(shape, w, max_tokens=max(16, x.shape[0]))
+        outs[mode], _, _ = full_check(blk, x)
+        blk.plan.close()
+    assert_close(bf16_to_f32(outs["umma"]), bf16_to_f32(outs["warp"]), "tensor-core vs warp MMA",
+                 max_rel=1e-2, mean_rel=1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -256,6 +296,17 @@ def test_b1_full_size(full_block):
     shape = synth.SHAPES["b1"]
     _, (mx, mn), near = full_check(full_block, synth.make_x(shape))
     print("b1: max_rel %.3g mean_rel %.3g near-ties %s" % (mx, mn, near))
+
+
+def test_b1_full_size_warp_mma(full_weights, monkeypatch):
+    shape = synth.SHAPES["b1"]
+    set_mode(monkeypatch, "warp")
+    blk = GpuBlock(shape, full_weights, max_tokens=128)
+    try:
+        _, (mx, mn), near = full_check(blk, synth.make_x(shape))
+        print("b1 (warp MMA): max_rel %.3g mean_rel %.3g near-ties %s" % (mx, mn, near))
+    finally:
+        blk.plan.close()
 
 
 # sampled tokens for the whole-block check at B = 64 and 128 (every token's

@@ -79,8 +79,9 @@ def test_every_batch_size_fits_the_kernels(name, cfg, sms):
             else:
                 assert g["grid"] == sms * g["ctas_per_sm"], where
             if g["ctas_per_sm"] == 2:
-                # only the expert kernels at one tile are compiled for two CTAs an SM
-                assert g["kind"] in (1, 2) and g["token_tiles"] == 1, where
+                # only the expert kernels are compiled for two CTAs an SM: at one
+                # token tile, and (tensor-core instantiation) at two
+                assert g["kind"] in (1, 2) and g["token_tiles"] in (1, 2), where
                 assert g["smem_bytes"] <= HALF_SM and g["stages"] >= 3, where
             elif side and g["kind"] in (0, 3, 4, 5):
                 assert g["smem_bytes"] <= HALF_SM and g["stages"] >= 2, where
@@ -110,15 +111,29 @@ def test_every_batch_size_fits_the_kernels(name, cfg, sms):
                 assert per_token == res_k[key]  # the same record size for every B
 
 
+@pytest.mark.parametrize("umma", ["1", "0"])
+def test_expert_kernel_choices(umma, monkeypatch):
+    # 8-token virtual experts up to 64 tokens; above, 16-token ones on the
+    # tensor-core path (two token tiles).  Either MMA path runs two expert
+    # CTAs an SM there (the tensor-core one holding half the SM's tensor
+    # memory each).
+    monkeypatch.setenv("MOE_UMMA", umma)
+    cfg = _cfg(synth.SHAPES["b1"])
+    for B in (1, 8, 64, 65, 128):
+        front, egu, edn, tail = _geometry(cfg, 148, B)[:4]
+        tg = 16 if (umma == "1" and B > 64) else 8
+        assert egu["ctas_per_sm"] == 2 and egu["grid"] == 296
+        assert egu["max_piece_tokens"] == min(B, tg)
+        assert egu["token_tiles"] == tg // 8
+        assert egu["stages"] >= 3 and edn["stages"] >= 3
+
+
 def test_full_size_choices():
-    # the measured configuration at full size: one token per stage at B = 1,
-    # the expert kernels two CTAs an SM with 8-token virtual experts
+    # the measured configuration at full size: one token per stage at B = 1
     cfg = _cfg(synth.SHAPES["b1"])
     for B, front_tiles in ((1, 1), (8, 1), (64, 8), (128, 16)):
         front, egu, edn, tail = _geometry(cfg, 148, B)[:4]
         assert front["token_tiles"] == front_tiles
-        assert egu["ctas_per_sm"] == 2 and egu["grid"] == 296
-        assert egu["max_piece_tokens"] == min(B, 8)
     front, egu, edn, tail, side_front, side_tail = _geometry(cfg, 148, 1)
     assert tail["resident_tail_bytes"] > 0  # B = 1 keeps c and h_s in shared memory
     assert front["pieces_per_row_block"] > 1  # the dense front splits K
