@@ -168,6 +168,8 @@ typedef struct moe_plan_info {
  *   MOE_SIDE_LANE=0         no side lane, whatever shared_sms says
  *   MOE_TAIL_SPLIT=0        the tail's shared-expert part is not scheduled first
  *   MOE_Z_FLAG=0            expert gate/up waits for the whole front kernel
+ *   MOE_H_FLAG=0            expert down waits for the whole gate/up kernel (default:
+ *                           per virtual expert, for its gate/up row blocks)
  *   MOE_PREFETCH_MB=n       L2 prefetch of the chosen experts' tiles by the
  *                           routing CTA once they are known, at most n MB
  *                           (default 0 = off: one SM issues them too slowly)

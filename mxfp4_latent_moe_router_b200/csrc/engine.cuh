@@ -104,6 +104,12 @@ struct Params {
   // expert gate/up kernel reads z once it reaches RB_lat instead of waiting
   // for the whole front grid (whose last CTAs stream shared-expert rows)
   int* z_done;
+  // per virtual expert: EGU's row-block finalisations of its h count up
+  // here (release); the expert down kernel streams a virtual expert's
+  // activations once its count reaches RB_egu instead of waiting for the
+  // whole gate/up grid.  Zeroed by the routing with the tables.
+  int* h_done;
+  int RB_egu;
   int RB_router;      // FRONT: leading row blocks holding router rows
   int RB_lat;         // FRONT: row blocks of the latent projection (after the router's);
                       // the shared expert's gate/up row blocks follow

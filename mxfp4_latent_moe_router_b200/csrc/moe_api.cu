@@ -155,7 +155,12 @@ struct moe_plan_s {
   // expert gate/up waits for the latent row blocks' count, not the whole
   // front grid (environment MOE_Z_FLAG=0 turns it off)
   bool z_flag = true;
+  // the expert down kernel starts a virtual expert once the gate/up kernel's
+  // row blocks of it are done, not after the whole gate/up grid
+  // (environment MOE_H_FLAG=0 turns it off)
+  bool h_flag = true;
   int* z_done = nullptr;
+  int* h_done = nullptr;  // per virtual expert (ve_max)
   // one launch per forward for B <= kFusedMaxTokens (environment MOE_FUSED=1);
   // off by default: measured slower than the four-launch chain at B = 1
   bool use_fused = false;
@@ -368,6 +373,8 @@ Params base_params(const moe_plan_s* p, int B) {
   q.route_ready = p->route_ready;
   q.err = p->err;
   q.z_done = p->z_flag ? p->z_done : nullptr;
+  q.h_done = p->h_flag ? p->h_done : nullptr;
+  q.RB_egu = p->g[KIND_EGU].RB;
   q.t_ready = p->t_ready;
   q.route_cnt = p->route_cnt;
   q.RB_lat = p->RB_lat;
@@ -582,6 +589,7 @@ void read_env(moe_plan_s* p) {
   if (const char* e = getenv("MOE_PROD_SLEEP")) p->prod_sleep = std::max(0, std::min(2000, atoi(e)));
   if (const char* e = getenv("MOE_TAIL_SPLIT")) p->tail_split = atoi(e) != 0;
   if (const char* e = getenv("MOE_Z_FLAG")) p->z_flag = atoi(e) != 0;
+  if (const char* e = getenv("MOE_H_FLAG")) p->h_flag = atoi(e) != 0;
   if (const char* e = getenv("MOE_SIDE_LANE")) p->side_env_off = atoi(e) == 0;
   if (const char* e = getenv("MOE_PREFETCH_MB")) p->prefetch_bytes = std::max(0LL, (long long)atoi(e)) << 20;
   if (const char* e = getenv("MOE_DIRECT_ROUTE")) p->direct_route = atoi(e) != 0;
@@ -664,6 +672,9 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->slots_sorted = (int*)v;
   TRY(alloc(p, &v, sizeof(VExpert) * p->ve_max, false));
   p->ve = (VExpert*)v;
+  TRY(alloc(p, &v, sizeof(int) * p->ve_max, false));
+  p->h_done = (int*)v;
+  CUDA_TRY(cudaMemset(v, 0, sizeof(int) * p->ve_max));
   // small control block: nve, router_done, err, Ctl[KIND_COUNT]
   TRY(alloc(p, &v, kControlBytes, false));
   p->nve = (int*)v;
@@ -771,6 +782,7 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
     q.table_off = kStageOff;
     q.ctl = p->ctl + kFused;
     q.z_done = nullptr;  // the single launch counts phases in `done`
+    q.h_done = nullptr;
     q.trace = p->trace ? p->trace + (size_t)kFused * 2 * p->num_sms * 24 : nullptr;
     q.done = p->done;
     q.need_rb_edn = p->g[KIND_EDN].RB;

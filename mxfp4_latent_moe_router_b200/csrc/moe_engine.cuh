@@ -451,6 +451,9 @@ __device__ __forceinline__ bool wait_count(const int* counter, int target, int* 
 //                     completion implies the front's (the tail reads h_s and
 //                     the combine weights after waiting only for its own
 //                     predecessor).
+//   EDN with h_done:  per piece, its virtual expert's h rows (the gate/up
+//                     kernel's row-block count of that expert; see the
+//                     producer), likewise with the exit wait.
 template <int KIND>
 __device__ __forceinline__ bool producer_dep_wait(const Params& p, int lane) {
   if (KIND == KIND_TAIL && p.t_rec) {
@@ -485,7 +488,12 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   // CTAs take pieces (and keep a grab in flight) from the start; the first
   // latent piece they hold waits for it.
   const bool free_start = KIND == KIND_TAIL && p.tail_split && !p.tail_part;
-  if (KIND == KIND_EGU && p.z_done) pdl_trigger();
+  // The expert down kernel with per-expert counts: a piece's activations are
+  // issued at once when its virtual expert's h is complete, else after its
+  // weight tiles, once the count is reached (pending stages stay contiguous
+  // in the ring: after one is deferred, the rest of the piece is too).
+  const bool ve_dep = KIND == KIND_EDN && p.h_done != nullptr;
+  if ((KIND == KIND_EGU && p.z_done) || ve_dep) pdl_trigger();
   // routing tables in shared memory: the per-stage lookups then cost no
   // global round trip (they are visible to the consumers through the first
   // full-barrier completion).  The whole capacity is copied so that these
@@ -515,6 +523,22 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
 
   // Resolve the dependency and issue the pending stages' activations.
   auto resolve = [&]() {
+    if (ve_dep) {
+      int v_ok = -1;
+      for (int j = 0; j < prefetched; ++j) {
+        const int s = (pend_first + j) % p.nstages;
+        uint8_t* sb = stage_base + (size_t)s * p.stage_bytes;
+        const Hdr& hs = *reinterpret_cast<const Hdr*>(sb);
+        if (hs.v != v_ok) {
+          if (!wait_count(p.h_done + hs.v, p.RB_egu, p.err, lane)) sp.total = 0;
+          fence_proxy_async_global();  // (bulk copies read the records)
+          v_ok = hs.v;
+        }
+        issue_act<KIND>(p, hs, sb + p.act_off, &full[s], lane, slot_tab);
+      }
+      prefetched = 0;
+      return;
+    }
     if (!producer_dep_wait<KIND>(p, lane)) sp.total = 0;  // gave up: no further pieces
     waited = true;
     for (int j = 0; j < prefetched; ++j) {
@@ -538,7 +562,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
   bool in_flight = false;
   const int workers = (int)gridDim.x - (KIND == KIND_FRONT ? p.route_cta : 0);
   int piece = blockIdx.x;
-  if ((waited || free_start) && piece < sp.total) {
+  if ((waited || free_start || ve_dep) && piece < sp.total) {
     if (lane == 0) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
     in_flight = true;
   }
@@ -547,6 +571,13 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
     Hdr ph;
     piece_header<KIND>(p, sp, piece, ph, ve_tab);
     const int c_first = ph.c_first, c_last = ph.c_last;
+    if (ve_dep) {
+      // its virtual expert's h complete already?
+      int cnt = 0;
+      if (lane == 0) cnt = ld_acquire(p.h_done + ph.v);
+      ph.dep = __shfl_sync(0xffffffffu, cnt, 0) < p.RB_egu ? 1 : 0;
+      if (!ph.dep) fence_proxy_async_global();
+    }
     for (int c = c_first; c < c_last; ++c) {
       // before the dependency resolves, fill at most one ring of weight-only
       // stages: the slot to reuse next would otherwise be a pending one
@@ -562,7 +593,7 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       __syncwarp();
       const long long tb = clock64();
       pb += tb - tw1;
-      if (waited || !h.dep) {
+      if ((waited || !h.dep) && !(ve_dep && prefetched > 0)) {
         issue_act<KIND>(p, h, sb + p.act_off, &full[stage], lane, slot_tab);
         pa += clock64() - tb;
       } else {
@@ -577,13 +608,13 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
       ++nst;
     }
     // a piece issued with pending activations: stop prefetching here
-    if (!waited && (prefetched > 0 || !free_start)) resolve();
+    if (!waited && (prefetched > 0 || (!free_start && !ve_dep))) resolve();
     if (!in_flight && lane == 0) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
     piece = __shfl_sync(0xffffffffu, grabbed, 0);
     in_flight = piece < sp.total;
     if (lane == 0 && in_flight) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
   }
-  if (!waited && (prefetched > 0 || !free_start)) resolve();
+  if (!waited && (prefetched > 0 || (!free_start && !ve_dep))) resolve();
   if (p.trace && lane == 0) {
     unsigned long long* tr = p.trace + (size_t)blockIdx.x * kTraceStride;
     tr[11] = (unsigned long long)pw;
@@ -1304,6 +1335,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const Hdr& h, float (&
                          i < p.I, false);  // ends with a barrier
     }
     if (p.done && tid == 0) red_release_add(p.done + 2, 1);
+    // every thread's records precede the release (barrier cumulativity)
+    if (p.h_done && tid == 0) red_release_add(p.h_done + h.v, 1);
   } else if (KIND == KIND_EDN) {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
@@ -1535,7 +1568,10 @@ __device__ __forceinline__ bool route_tokens(const Params& p, const float* bias,
         ve.start = bc + gi * tg;
         ve.count = min(tg, c[i] - gi * tg);
         ve.pad = 0;
-        if (bg + gi < p.ve_max) p.ve[bg + gi] = ve;
+        if (bg + gi < p.ve_max) {
+          p.ve[bg + gi] = ve;
+          if (p.h_done) p.h_done[bg + gi] = 0;
+        }
       }
     }
     bc += c[i];
@@ -1977,7 +2013,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   //     kernel but what its producer copies after that count; it waits for
   //     the front grid only before exiting.
   const bool lazy = KIND == KIND_TAIL && p.tail_split && !p.tail_part;
-  const bool late = KIND == KIND_EGU && p.z_done;
+  const bool late = (KIND == KIND_EGU && p.z_done) || (KIND == KIND_EDN && p.h_done);
   uint8_t* res = stage_base - p.stage_off + p.res_off;  // shared-memory base + offset
   const int klat = p.C_lat * 64;
   // Past the wait every earlier kernel of the forward has finished, so no
