@@ -338,24 +338,25 @@ __device__ __forceinline__ void copy_records_umma(const Params& p, const Hdr& h,
   uint8_t* B = sb + kUBOff;
   uint8_t* sfb = B + rows * kUTermBytes;
   const int cz = (p.L + kMxChunkK - 1) / kMxChunkK;
-  constexpr int kPerTerm = kMxChunkK / 32 + 2;  // 8 K blocks of 16 bytes, 2 scale words
-  constexpr int kPerTok = kUTerms * kPerTerm;
-  const int items = h.ntok * kPerTok;
-  for (int it = lane; it < items; it += 32) {
-    const int tok = it / kPerTok, rem = it - tok * kPerTok;
-    const int t = rem / kPerTerm, q = rem - t * kPerTerm;
+  // lane -> (token, term) rows, the token fastest: one record pointer a row,
+  // then its 8 K blocks of 16 bytes and 2 scale words
+  for (int it = lane; it < per_tok * kUTerms; it += 32) {
+    const int tok = it & (per_tok - 1), t = it / per_tok;
+    if (tok >= h.ntok) continue;
     const uint8_t* rec;
     if (KIND == KIND_EGU)
       rec = p.z_mx + ((long long)(slot_tab[h.tok0 + tok] / p.topk) * cz + h.chunk) * p.act_rec;
     else
       rec = p.h_mx + ((long long)h.chunk * p.ld_slots + h.tok0 + tok) * p.act_rec;
     const int n = t * per_tok + tok;
-    if (q < kPerTerm - 2) {
-      cp_async16(B + (q * ng + (n >> 3)) * 128 + (n & 7) * 16, rec + t * kUTermBytes + q * 16);
-    } else {
-      const int u = q - (kPerTerm - 2);
-      cp_async4(sfb + u * 512 + (n & 31) * 16 + (n >> 5) * 4, rec + kUTerms * kUTermBytes + t * 8 + u * 4);
-    }
+    uint8_t* dst = B + (n >> 3) * 128 + (n & 7) * 16;
+    const uint8_t* src = rec + t * kUTermBytes;
+#pragma unroll
+    for (int q = 0; q < kMxChunkK / 32; ++q) cp_async16(dst + q * ng * 128, src + q * 16);
+    const uint8_t* ssrc = rec + kUTerms * kUTermBytes + t * 8;
+    uint8_t* sdst = sfb + (n & 31) * 16 + (n >> 5) * 4;
+    cp_async4(sdst, ssrc);
+    cp_async4(sdst + 512, ssrc + 4);
   }
   rows_async_done(bar, lane);
 }
