@@ -24,6 +24,10 @@ namespace {
 constexpr int kScratchOff = 1024;
 constexpr int kScratchBytes = 20480;
 constexpr int kStageOff = kScratchOff + kScratchBytes;
+// The tensor-core expert kernels at up to two token tiles use at most 8.5 KB
+// of the consumers' scratch (the accumulator staging, 128 rows x 17 floats;
+// the split-K sums, 16 columns x 128 rows): the rest goes to the ring.
+constexpr int kScratchBytesUmmaSmall = 9216;
 constexpr int kHdr = 128;
 // per-kind slots (scheduling state, profile, trace), one for the fused
 // single launch, and two for the side lane's kernels (the shared expert's
@@ -146,6 +150,7 @@ struct moe_plan_s {
   int expert_per_sm_max = 2;     // environment MOE_EXPERT_CTAS_PER_SM
   int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
   int expert_tg_fixed = 0;       // environment MOE_EXPERT_TG (8, 16 or 32; 0: by batch size)
+  int expert_ppr_fixed = 0;      // environment MOE_EXPERT_PPR (split-K factor; 0: makespan model)
   bool use_pdl = true;
   int fail_alloc_after = -1;     // environment MOE_FAIL_ALLOC_AFTER (tests only)
   int prod_sleep = 200, cons_sleep = 32;  // environment MOE_PROD_SLEEP / MOE_CONS_SLEEP (ns)
@@ -182,6 +187,12 @@ int expert_tg(const moe_plan_s* p, int B) {
   // near-uniform tokens, where few experts see more than 8, 536 vs 515)
   if (p->umma && B > 64 && B <= p->expert_small_max_b) return kExpertTgUmmaLarge;
   return B <= p->expert_small_max_b ? kExpertTgSmall : kExpertTgLarge;
+}
+
+// Most virtual experts a forward with `slots` = B * k expert slots can have:
+// an expert per slot (at most E) plus one group boundary per 8 slots.
+int ve_bound(const moe_plan_s* p, int slots) {
+  return std::min(p->ve_max, std::min(p->cfg.num_experts, slots) + ceil_div(slots, kExpertTgSmall) + 1);
 }
 
 // Whether a forward of B tokens runs the shared expert as a side lane.
@@ -231,8 +242,14 @@ moe_status alloc(moe_plan p, void** out, size_t bytes, bool packed) {
 
 bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
 
+int scratch_bytes(const moe_plan_s* p, int kind, int nt) {
+  return ((kind == KIND_EGU || kind == KIND_EDN) && p->umma && nt <= 2) ? kScratchBytesUmmaSmall
+                                                                          : kScratchBytes;
+}
+
 struct SmemGeom {
   int stage_bytes, nstages, act_off, act_stride, table_bytes, stage_off, res_bytes;
+  int table_off;  // after the consumers' scratch
   size_t total;
 };
 
@@ -242,14 +259,15 @@ int resident_stride(int res_k) { return res_k * 4 + 64; }
 
 SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int slots,
                    int res_bytes = 0, int budget = kBigSmem, bool formed = false) {
-  const int topk = p->cfg.top_k, ve_max = p->ve_max;
+  const int topk = p->cfg.top_k, ve_max = ve_bound(p, slots);
   SmemGeom s;
   // routing tables (virtual experts + expert-sorted slots) for the expert kernels
   s.table_bytes = 0;
   if (kind == KIND_EGU || kind == KIND_EDN)
     s.table_bytes = ((ve_max * (int)sizeof(VExpert) + slots * 4) + 127) / 128 * 128;
   s.res_bytes = res_bytes;
-  const int stage_off = kStageOff + s.table_bytes + res_bytes;
+  s.table_off = kScratchOff + scratch_bytes(p, kind, nt);
+  const int stage_off = s.table_off + s.table_bytes + res_bytes;
   int act = 0;
   s.act_stride = 0;
   if (kind == KIND_FRONT) {
@@ -368,7 +386,7 @@ Params base_params(const moe_plan_s* p, int B) {
   q.slots_sorted = p->slots_sorted;
   q.ve = p->ve;
   q.nve = p->nve;
-  q.ve_max = p->ve_max;
+  q.ve_max = ve_bound(p, B * c.top_k);
   q.router_done = p->router_done;
   q.route_ready = p->route_ready;
   q.err = p->err;
@@ -400,7 +418,7 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
   q.stage_bytes = s.stage_bytes;
   q.act_off = s.act_off;
   q.act_stride = s.act_stride;
-  q.table_off = kStageOff;
+  q.table_off = s.table_off;
   q.stage_off = s.stage_off;
   q.matrix_bytes = (long long)p->g[kind].weight_bytes;
   switch (kind) {
@@ -420,8 +438,8 @@ void set_kind(Params& q, const moe_plan_s* p, int kind, const SmemGeom& s) {
       q.route_cta = 1;
       break;
     }
-    case KIND_EGU: q.wt = p->w_egu; q.tg = expert_tg(p, q.B); break;
-    case KIND_EDN: q.wt = p->w_edn; q.tg = expert_tg(p, q.B); break;
+    case KIND_EGU: q.wt = p->w_egu; q.tg = expert_tg(p, q.B); q.PPR = p->expert_ppr_fixed; break;
+    case KIND_EDN: q.wt = p->w_edn; q.tg = expert_tg(p, q.B); q.PPR = p->expert_ppr_fixed; break;
     default: q.wt = p->w_tail; q.tg = p->tail_tg; break;
   }
 }
@@ -434,6 +452,14 @@ int split_cost_for(const moe_plan_s* p, int nt) { return p->split_cost * (1 + st
 // split-K factor of a kind whose row-block count the host knows
 int ppr_for(const moe_plan_s* p, int mats, int C, int ctas, int nt) {
   return best_ppr(mats, C, ctas, split_cost_for(p, nt));
+}
+
+// The expert kernels' split-K factor for `mats` row blocks (the device
+// computes the same from the routing's count of virtual experts), or the
+// fixed one of MOE_EXPERT_PPR (at most the chunk count).
+int expert_ppr(const moe_plan_s* p, int mats, int C, int ctas, int nt) {
+  if (p->expert_ppr_fixed > 0) return std::min(p->expert_ppr_fixed, C);
+  return ppr_for(p, mats, C, ctas, nt);
 }
 
 // Router row blocks are the first pieces handed out and the routing waits
@@ -499,7 +525,7 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
       // the split depends on the routing: take the largest over every
       // possible count of virtual experts
       for (int V = 1; V <= p->ve_max; ++V)
-        pieces = std::max(pieces, (size_t)V * g.RB * ppr_for(p, V * g.RB, g.C, f.expert_grid, nt));
+        pieces = std::max(pieces, (size_t)V * g.RB * expert_ppr(p, V * g.RB, g.C, f.expert_grid, nt));
     }
     best = std::max(best, pieces * (size_t)nt * 1024);
   }
@@ -578,6 +604,7 @@ void read_env(moe_plan_s* p) {
   if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
   if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_EXPERT_PPR")) p->expert_ppr_fixed = std::max(0, std::min(8, atoi(e)));
   if (const char* e = getenv("MOE_EXPERT_TG")) {
     const int v = atoi(e);
     p->expert_tg_fixed = (v == 8 || v == 16 || v == 32) ? v : 0;
@@ -1400,10 +1427,10 @@ moe_status moe_debug_geometry(const moe_config* cfg, int32_t num_sms, int32_t nu
       o.ctas_per_sm = f.expert_per_sm;
       o.token_tiles = f.nt_e;
       o.max_piece_tokens = std::min(B, expert_tg(p, B));
-      o.pieces_per_row_block = ppr_for(p, p->ve_max * g.RB, g.C, f.expert_grid, f.nt_e);
+      o.pieces_per_row_block = expert_ppr(p, ve_bound(p, B * K) * g.RB, g.C, f.expert_grid, f.nt_e);
       int64_t most = 0;
       for (int V = 1; V <= p->ve_max; ++V)
-        most = std::max(most, (int64_t)V * g.RB * ppr_for(p, V * g.RB, g.C, f.expert_grid, f.nt_e));
+        most = std::max(most, (int64_t)V * g.RB * expert_ppr(p, V * g.RB, g.C, f.expert_grid, f.nt_e));
       o.partial_floats_needed = most * f.nt_e * 1024;
     } else {
       const TailLaunch l = tail_launch(p, f, B, k == 5 ? 2 : (f.side ? 1 : 0));

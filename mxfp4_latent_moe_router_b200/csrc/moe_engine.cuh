@@ -102,7 +102,7 @@ __device__ __forceinline__ Space make_space(const Params& p, int V = 0) {
   Space s;
   if (KIND == KIND_EGU || KIND == KIND_EDN) {
     const int mats = V * p.RB;
-    const int ppr = best_ppr(mats, p.C, p.piece_ctas, p.split_cost);
+    const int ppr = p.PPR > 0 ? min(p.PPR, p.C) : best_ppr(mats, p.C, p.piece_ctas, p.split_cost);
     s.ppr = ppr;
     s.total = mats * ppr;
   } else if (KIND == KIND_TAIL) {
@@ -1861,11 +1861,11 @@ static_assert(tmem_sf<4>() + 16 * kMaxStages <= tmem_cols<4>(), "scale columns o
 // shared-memory handover: tensor-memory base at flag word kUTmemWord,
 // accumulator-full barriers (MMA completion + the header's release) at words
 // kUDfullWord + 2 b, accumulator-free barriers at kUDfreeWord + 2 b, the MMA
-// warp's drain barrier at kUDrainWord; the finished pieces' headers at the
-// end of the scratch area
+// warp's drain barrier at kUDrainWord; the finished pieces' headers at byte
+// kUPqByte of shared memory (between the flags and the scratch)
 constexpr int kUTmemWord = 48, kUDfullWord = 50, kUDfreeWord = 54, kUDrainWord = 58;
-constexpr int kUPqOff = 19456;
-static_assert(2 * sizeof(Hdr) <= 1024, "two piece headers behind the consumers' scratch");
+constexpr int kUPqByte = 512;
+static_assert(kUPqByte + 2 * sizeof(Hdr) <= 1024, "two piece headers before the consumers' scratch");
 constexpr int kThreadsU = kThreads + 32;  // + the MMA warp
 constexpr int kMmaWarp = kConsumerWarps + 1;
 
@@ -2057,7 +2057,7 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
   const uint32_t tmem = UM ? *reinterpret_cast<volatile uint32_t*>(sm_flag + kUTmemWord) : 0u;
   uint64_t* dfull = reinterpret_cast<uint64_t*>(sm_flag + kUDfullWord);
   uint64_t* dfree = reinterpret_cast<uint64_t*>(sm_flag + kUDfreeWord);
-  const Hdr* pq = reinterpret_cast<const Hdr*>(scratch + kUPqOff);
+  const Hdr* pq = reinterpret_cast<const Hdr*>(stage_base - p.stage_off + kUPqByte);
   // a piece's sums are in acc (+ acc2): split-K partials, tickets,
   // finalisation, epilogue
   auto piece_done = [&](const Hdr& h) {
@@ -2225,7 +2225,8 @@ template <int KIND, int NT, int MINB, bool UM>
 __global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
     moe_kernel(const __grid_constant__ Params p) {
   // shared memory: [0,128) full barriers, [128,256) empty barriers,
-  // [256,512) flags, [scratch_off, ...) scratch, [table_off, ...) routing
+  // [256,512) flags, [512,1024) the tensor-core kernels' piece headers,
+  // [scratch_off, ...) scratch, [table_off, ...) routing
   // tables (expert kernels), [stage_off, ...) ring
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -2284,7 +2285,7 @@ __global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
   } else if (UM && warp == kMmaWarp) {
     if (lane == 0)
       mma_issuer<NT>(p, stages, full, empty, dfull, dfree, drain,
-                     reinterpret_cast<Hdr*>(scratch + kUPqOff), *tmem_slot);
+                     reinterpret_cast<Hdr*>(smem + kUPqByte), *tmem_slot);
   } else {
     consumer<KIND, NT, UM>(p, stages, full, empty, scratch, sm_flag, slot_tab, warp, lane);
   }
