@@ -520,7 +520,10 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us_step / 1e3, "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f16 MMA on bf16 + MXFP4 weights, fp32 accumulate",
+            "scaling": "weak", "vs_baseline": None, "dtype": ("bf16 MMA (dense rows), e2m1 x e2m1 block-scaled MMA (MXFP4 experts, "
+                      "activations as 4 e2m1 terms), fp32 accumulate"
+                      if os.environ.get("MOE_UMMA", "1") != "0" else
+                      "bf16 MMA (dense rows), f16 MMA on decoded MXFP4 (experts), fp32 accumulate"),
             "data": "synthetic",
             "config": {"workload": _workload_desc(shape), "tokens_per_step": B,
                        "weight_instances": args.instances,
