@@ -190,7 +190,7 @@ int launch_expire_wait(int* never, int* err, int* router_done, int* ticket, Ctl*
 int set_smem_limits(size_t bytes);
 
 int launch_pack_dense(const void* src, int K, int N, int layout, int RB, int C, int rows_valid,
-                      uint8_t* dst, void* stream, const void* src2, int K2, int C_first);
+                      uint8_t* dst, void* stream, const void* src2, int K2, int C_first, int umma = 0);
 int launch_pack_mx(const uint8_t* codes, const uint8_t* scales, int E, int rows, int K,
                    int layout, int RB, int C, uint8_t* dst, int* err, void* stream, int umma);
 

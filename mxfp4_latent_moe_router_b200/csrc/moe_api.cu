@@ -95,6 +95,7 @@ struct moe_plan_s {
   uint8_t* w_egu = nullptr;
   uint8_t* w_edn = nullptr;
   uint8_t* w_tail = nullptr;
+  uint8_t* w_tail_um = nullptr;  // the tail's tiles in the tensor-core order (umma_tail)
   float* bias = nullptr;
 
   float* logits = nullptr;
@@ -137,6 +138,10 @@ struct moe_plan_s {
   // activation records' form, so it is fixed when the plan is made
   bool umma = true;
   int act_rec = kActRecBytesU;
+  // the tail on the tensor cores (bf16 MMA of the formed records' hi and lo
+  // parts) whenever its activation is staged from formed records; needs a
+  // second copy of the tail's tiles (environment MOE_UMMA_TAIL=0 turns it off)
+  bool umma_tail = true;
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* out_stage = nullptr;
@@ -282,9 +287,12 @@ SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int s
     s.act_stride = 576;
     act = 8 * nt * s.act_stride;
   } else {
-    // resident: none; formed records: 256 bytes a token; else the k slots'
+    // resident: none; formed records: 256 bytes a token (the tensor-core
+    // tail: its 8 NT token rows, two 128-byte parts each); else the k slots'
     // y rows a token (the fused single launch)
-    act = res_bytes ? 0 : formed ? tail_tg_eff * 256 : tail_tg_eff * std::max(1, topk) * 256;
+    act = res_bytes ? 0
+          : formed  ? (p->umma_tail ? 8 * nt * 256 : tail_tg_eff * 256)
+                    : tail_tg_eff * std::max(1, topk) * 256;
   }
   const int tile = (kind == KIND_EGU || kind == KIND_EDN) ? kMxTileBytes : kDenseTileBytes;
   if (!((kind == KIND_EGU || kind == KIND_EDN) && p->umma)) {
@@ -622,6 +630,8 @@ void read_env(moe_plan_s* p) {
   if (const char* e = getenv("MOE_DIRECT_ROUTE")) p->direct_route = atoi(e) != 0;
   if (const char* e = getenv("MOE_CONS_SLEEP")) p->cons_sleep = std::max(0, std::min(2000, atoi(e)));
   if (const char* e = getenv("MOE_UMMA")) p->umma = atoi(e) != 0;
+  if (const char* e = getenv("MOE_UMMA_TAIL")) p->umma_tail = atoi(e) != 0;
+  p->umma_tail = p->umma_tail && p->umma;
   p->act_rec = p->umma ? kActRecBytesU : kActRecBytes;
   if (p->umma) p->use_fused = false;  // the single launch keeps the warp-level MMA
 }
@@ -675,6 +685,10 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   p->w_edn = (uint8_t*)v;
   TRY(alloc(p, &v, tl.weight_bytes, true));
   p->w_tail = (uint8_t*)v;
+  if (p->umma_tail) {
+    TRY(alloc(p, &v, tl.weight_bytes, true));
+    p->w_tail_um = (uint8_t*)v;
+  }
   TRY(alloc(p, &v, sizeof(float) * E, true));
   p->bias = (float*)v;
 
@@ -996,6 +1010,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       q.tail_split = l.split;
       q.tail_part = 2;
       q.half_sm = 1;
+      q.umma = 0;  // (the side lane's tail keeps the warp-level MMA)
       TRY(launch_timed(p, kSideTail, KIND_TAIL, f.nt_tail, q, l.grid, l.sm.total, p->side));
     }
     CUDA_TRY(cudaEventRecord(p->ev_join, p->side));
@@ -1027,6 +1042,9 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     q.tail_part = f.side ? 1 : 0;
     q.half_sm = f.side ? 1 : 0;
     if (l.formed) q.t_rec = p->t_rec;
+    // the tensor-core tail: formed records, the whole K range, no side lane
+    q.umma = (p->umma_tail && l.formed && !l.split && !f.side) ? 1 : 0;
+    if (q.umma) q.wt = p->w_tail_um;
     TRY(launch_timed(p, KIND_TAIL, KIND_TAIL, f.nt_tail, q, f.tail_grid, l.sm.total, s));
   }
   if (f.side) CUDA_TRY(cudaStreamWaitEvent(s, p->ev_join, 0));
@@ -1141,6 +1159,9 @@ moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
   const KindGeom& tl = p->g[KIND_TAIL];
   CUDA_TRY((cudaError_t)launch_pack_dense(w->w_out, L, H, 2, tl.RB, tl.C, H, p->w_tail, s,
                                           Is > 0 ? w->sh_down : w->w_out, Is, p->C_lat));
+  if (p->w_tail_um)
+    CUDA_TRY((cudaError_t)launch_pack_dense(w->w_out, L, H, 2, tl.RB, tl.C, H, p->w_tail_um, s,
+                                            Is > 0 ? w->sh_down : w->w_out, Is, p->C_lat, 1));
   const KindGeom& eg = p->g[KIND_EGU];
   CUDA_TRY((cudaError_t)launch_pack_mx(w->gu_codes, w->gu_scales, E, 2 * I, L, 1, eg.RB, eg.C,
                                        p->w_egu, p->err, s, p->umma ? 1 : 0));

@@ -255,7 +255,8 @@ __device__ __forceinline__ const uint8_t* weight_src(const Params& p, const Hdr&
 constexpr int kBulkRowsMax = 8;
 template <int KIND>
 __device__ __forceinline__ bool rows_async(const Params& p, const Hdr& h) {
-  if ((KIND == KIND_EGU || KIND == KIND_EDN) && p.umma) return true;  // scattered into the MMA's B layout
+  if ((KIND == KIND_EGU || KIND == KIND_EDN || KIND == KIND_TAIL) && p.umma)
+    return true;  // scattered into the MMA's B layout
   return (KIND == KIND_FRONT || KIND == KIND_EGU || KIND == KIND_EDN) && h.ntok > kBulkRowsMax;
 }
 
@@ -361,12 +362,34 @@ __device__ __forceinline__ void copy_records_umma(const Params& p, const Hdr& h,
   rows_async_done(bar, lane);
 }
 
+// Tensor-core tail stage: every token's formed record (bf16 hi and lo parts
+// of one 64-wide chunk) as two rows of the B operand (row n = part * 8 NT +
+// token; K block kb of row n at (kb * ng + n / 8) * 128 + (n % 8) * 16).
+__device__ __forceinline__ void copy_tail_records_umma(const Params& p, const Hdr& h, uint8_t* B,
+                                                       uint64_t* bar, int lane, int nt) {
+  const int per_tok = 8 * nt, ng = 2 * per_tok / 8;
+  for (int it = lane; it < 2 * per_tok; it += 32) {
+    const int tok = it & (per_tok - 1), part = it / per_tok;
+    if (tok >= h.ntok) continue;
+    const uint8_t* src = p.t_rec + ((long long)h.chunk * p.B + h.tok0 + tok) * 256 + part * 128;
+    const int n = part * per_tok + tok;
+    uint8_t* dst = B + (n >> 3) * 128 + (n & 7) * 16;
+#pragma unroll
+    for (int q = 0; q < kDenseChunkK / 8; ++q) cp_async16(dst + q * ng * 128, src + q * 16);
+  }
+  rows_async_done(bar, lane);
+}
+
 // Issue this stage's activation copies (all 32 producer lanes).
 template <int KIND>
 __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t* act, uint64_t* bar,
                                           int lane, const int* slot_tab) {
   if ((KIND == KIND_EGU || KIND == KIND_EDN) && p.umma) {
     copy_records_umma<KIND>(p, h, act - p.act_off, bar, lane, slot_tab, p.umma);  // (umma = NT)
+    return;
+  }
+  if (KIND == KIND_TAIL && p.umma) {
+    copy_tail_records_umma(p, h, act, bar, lane, p.umma);  // (umma = NT)
     return;
   }
   if (rows_async<KIND>(p, h)) {
@@ -1849,15 +1872,23 @@ __device__ __forceinline__ void finalize(const Params& p, const Hdr& h, float (&
 // after the MMAs that read them have completed (they release the slot).
 // Up to two token tiles the CTA takes 256 columns (two CTAs can share an
 // SM), at four 512.
-template <int NT>
-__host__ __device__ constexpr uint32_t tmem_dcols() { return (uint32_t)umma_rows(NT); }
-template <int NT>
-__host__ __device__ constexpr uint32_t tmem_sf() { return 2 * tmem_dcols<NT>(); }
-template <int NT>
-__host__ __device__ constexpr uint32_t tmem_cols() { return NT <= 2 ? 256u : 512u; }
-static_assert(tmem_sf<1>() + 16 * kMaxStages <= tmem_cols<1>(), "scale columns of every ring slot");
-static_assert(tmem_sf<2>() + 16 * kMaxStages <= tmem_cols<2>(), "scale columns of every ring slot");
-static_assert(tmem_sf<4>() + 16 * kMaxStages <= tmem_cols<4>(), "scale columns of every ring slot");
+// The tail's bf16 MMA (its activation as hi and lo parts, two rows a token)
+// needs no scale columns: 2 x 16 NT accumulator columns.
+template <int KIND>
+__host__ __device__ constexpr int umma_terms() { return KIND == KIND_TAIL ? 2 : kUTerms; }
+template <int KIND, int NT>
+__host__ __device__ constexpr uint32_t tmem_dcols() { return (uint32_t)(umma_terms<KIND>() * 8 * NT); }
+template <int KIND, int NT>
+__host__ __device__ constexpr uint32_t tmem_sf() { return 2 * tmem_dcols<KIND, NT>(); }
+template <int KIND, int NT>
+__host__ __device__ constexpr uint32_t tmem_cols() {
+  return KIND == KIND_TAIL ? (NT <= 4 ? 128u : 256u) : (NT <= 2 ? 256u : 512u);
+}
+static_assert(tmem_sf<KIND_EGU, 1>() + 16 * kMaxStages <= tmem_cols<KIND_EGU, 1>(), "scale columns");
+static_assert(tmem_sf<KIND_EGU, 2>() + 16 * kMaxStages <= tmem_cols<KIND_EGU, 2>(), "scale columns");
+static_assert(tmem_sf<KIND_EGU, 4>() + 16 * kMaxStages <= tmem_cols<KIND_EGU, 4>(), "scale columns");
+static_assert(tmem_sf<KIND_TAIL, 8>() <= tmem_cols<KIND_TAIL, 8>(), "two accumulator buffers");
+static_assert(tmem_sf<KIND_TAIL, 4>() <= tmem_cols<KIND_TAIL, 4>(), "two accumulator buffers");
 // shared-memory handover: tensor-memory base at flag word kUTmemWord,
 // accumulator-full barriers (MMA completion + the header's release) at words
 // kUDfullWord + 2 b, accumulator-free barriers at kUDfreeWord + 2 b, the MMA
@@ -1869,10 +1900,10 @@ static_assert(kUPqByte + 2 * sizeof(Hdr) <= 1024, "two piece headers before the 
 constexpr int kThreadsU = kThreads + 32;  // + the MMA warp
 constexpr int kMmaWarp = kConsumerWarps + 1;
 
-template <int NT>
+template <int KIND, int NT>
 __device__ void mma_issuer(const Params& p, uint8_t* stage_base, uint64_t* full, uint64_t* empty,
                            uint64_t* dfull, uint64_t* dfree, uint64_t* drain, Hdr* pq, uint32_t tmem) {
-  constexpr int kRows = umma_rows(NT), kNg = kRows / 8;
+  constexpr int kRows = umma_terms<KIND>() * 8 * NT, kNg = kRows / 8;
   int stage = 0, buf = 0;
   uint32_t phase = 0, uses[2] = {0u, 0u};
   long long mw = 0, mi = 0, t0 = clock64();
@@ -1897,21 +1928,33 @@ __device__ void mma_issuer(const Params& p, uint8_t* stage_base, uint64_t* full,
     }
     fence_proxy_async_smem();  // the activation rows came in by cp.async
     umma::fence_after_sync();
-    const uint8_t* A = sb + kUAOff;
-    const uint8_t* B = sb + kUBOff;
-    const uint32_t sfa_t = tmem + tmem_sf<NT>() + 16u * (uint32_t)stage, sfb_t = sfa_t + 8;
+    const uint32_t d = tmem + (uint32_t)buf * tmem_dcols<KIND, NT>();
+    if constexpr (KIND == KIND_TAIL) {
+      // bf16 weights (128 x 64 K) x the records' hi and lo rows: four K = 16
+      const uint8_t* A = sb + kHdrBytes;
+      const uint8_t* B = sb + p.act_off;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      umma::cp_scales(sfa_t + 4 * u, umma::smem_desc(sb + kUSfaOff + 512 * u, 128, 128));
-      umma::cp_scales(sfb_t + 4 * u, umma::smem_desc(B + kRows * kUTermBytes + 512 * u, 128, 128));
-    }
-    const uint32_t d = tmem + (uint32_t)buf * tmem_dcols<NT>();
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t ad = umma::smem_desc(A + j * 4096, 2048, 128);
+        const uint64_t bd = umma::smem_desc(B + j * 2 * kNg * 128, kNg * 128, 128);
+        umma::mma_bf16(d, ad, bd, umma::idesc_bf16(128, kRows), !(first && j == 0));
+      }
+    } else {
+      const uint8_t* A = sb + kUAOff;
+      const uint8_t* B = sb + kUBOff;
+      const uint32_t sfa_t = tmem + tmem_sf<KIND, NT>() + 16u * (uint32_t)stage, sfb_t = sfa_t + 8;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint64_t ad = umma::smem_desc(A + j * 4096, 2048, 128);
-      const uint64_t bd = umma::smem_desc(B + j * 2 * kNg * 128, kNg * 128, 128);
-      umma::mma_mxf4(d, ad, bd, umma::idesc_mxf4(128, kRows, 2 * (j & 1), 2 * (j & 1)),
-                     sfa_t + 4 * (j >> 1), sfb_t + 4 * (j >> 1), !(first && j == 0));
+      for (int u = 0; u < 2; ++u) {
+        umma::cp_scales(sfa_t + 4 * u, umma::smem_desc(sb + kUSfaOff + 512 * u, 128, 128));
+        umma::cp_scales(sfb_t + 4 * u, umma::smem_desc(B + kRows * kUTermBytes + 512 * u, 128, 128));
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t ad = umma::smem_desc(A + j * 4096, 2048, 128);
+        const uint64_t bd = umma::smem_desc(B + j * 2 * kNg * 128, kNg * 128, 128);
+        umma::mma_mxf4(d, ad, bd, umma::idesc_mxf4(128, kRows, 2 * (j & 1), 2 * (j & 1)),
+                       sfa_t + 4 * (j >> 1), sfb_t + 4 * (j >> 1), !(first && j == 0));
+      }
     }
     umma::commit(&empty[stage]);  // the slot is free once these MMAs have read it
     if (h.flags & HDR_LAST) {
@@ -1941,46 +1984,51 @@ __device__ void mma_issuer(const Params& p, uint8_t* stage_base, uint64_t* full,
 
 // A finished piece's sums out of tensor memory into the MMA-fragment
 // registers the epilogues take: warps 0-3 read their 32 rows (lane quarter
-// = warp), add the kUTerms terms of each token and stage the sums in shared
-// memory (128 rows x 8 NT tokens); the buffer is then released to the MMA
-// warp and every warp picks its fragment.
-template <int NT>
+// = warp), add the TERMS terms of each token and stage the sums in shared
+// memory (128 rows x up to 32 tokens at a time); the buffer is released to
+// the MMA warp once read, and every warp picks its fragments.
+template <int NT, int TERMS>
 __device__ __forceinline__ void umma_read_acc(uint32_t d, float* stage_s, float (&acc)[NT][4], int warp,
                                              int lane, int tid, uint64_t* dfree_bar) {
   umma::fence_after_sync();
-  constexpr int kTok = 8 * NT, kLd = kTok + 1;  // (row stride padded: no bank conflicts)
-  if (warp < 4) {
-    const int row = 32 * warp + lane;
-    const uint32_t lane_addr = d + ((uint32_t)(32 * warp) << 16);
-#pragma unroll
-    for (int c = 0; c < NT; ++c) {
-      float sum[8], t[8];
-      umma::ld_32x32b_x8(lane_addr + 8 * c, sum);
-      umma::wait_ld();
-#pragma unroll
-      for (int term = 1; term < kUTerms; ++term) {
-        umma::ld_32x32b_x8(lane_addr + term * kTok + 8 * c, t);
-        umma::wait_ld();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sum[i] += t[i];
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) stage_s[row * kLd + 8 * c + i] = sum[i];
-    }
-  }
-  umma::fence_before_sync();
-  named_sync(1, kConsumerThreads);
-  if (tid == 0) mbar_arrive(dfree_bar);
+  constexpr int kTok = 8 * NT;                 // columns of one term
+  constexpr int kGrp = NT < 4 ? NT : 4;        // token tiles staged at a time
+  constexpr int kLd = 8 * kGrp + 1;            // (row stride padded: no bank conflicts)
   const int g = lane >> 2, tig = lane & 3;
 #pragma unroll
-  for (int t = 0; t < NT; ++t)
+  for (int t0 = 0; t0 < NT; t0 += kGrp) {
+    if (warp < 4) {
+      const int row = 32 * warp + lane;
+      const uint32_t lane_addr = d + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int col = 8 * t + 2 * tig + (q & 1);
-      const int row = 16 * warp + ((q & 2) ? g + 8 : g);
-      acc[t][q] = stage_s[row * kLd + col];
+      for (int c = 0; c < kGrp; ++c) {
+        float sum[8], t[8];
+        umma::ld_32x32b_x8(lane_addr + 8 * (t0 + c), sum);
+        umma::wait_ld();
+#pragma unroll
+        for (int term = 1; term < TERMS; ++term) {
+          umma::ld_32x32b_x8(lane_addr + term * kTok + 8 * (t0 + c), t);
+          umma::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sum[i] += t[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) stage_s[row * kLd + 8 * c + i] = sum[i];
+      }
     }
-  named_sync(1, kConsumerThreads);
+    if (t0 + kGrp >= NT) umma::fence_before_sync();
+    named_sync(1, kConsumerThreads);
+    if (t0 + kGrp >= NT && tid == 0) mbar_arrive(dfree_bar);
+#pragma unroll
+    for (int c = 0; c < kGrp; ++c)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col = 8 * c + 2 * tig + (q & 1);
+        const int row = 16 * warp + ((q & 2) ? g + 8 : g);
+        acc[t0 + c][q] = stage_s[row * kLd + col];
+      }
+    named_sync(1, kConsumerThreads);
+  }
 }
 
 template <int KIND, int NT, bool UM>
@@ -2142,7 +2190,8 @@ __device__ void consumer(const Params& p, uint8_t* stage_base, uint64_t* full, u
       if (h.flags & HDR_END) break;
       if (tr && tid == 0 && n_pieces == 0) tr[6] = global_ns();
       zero_acc(acc2);
-      umma_read_acc<NT>(tmem + (uint32_t)buf * tmem_dcols<NT>(), reinterpret_cast<float*>(scratch), acc, warp,
+      umma_read_acc<NT, umma_terms<KIND>()>(tmem + (uint32_t)buf * tmem_dcols<KIND, NT>(),
+                                            reinterpret_cast<float*>(scratch), acc, warp,
                         lane, tid, &dfree[buf]);
       ++uses[buf];
       buf ^= 1;
@@ -2249,7 +2298,7 @@ __global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
   // completed and the MMA warp has written the piece's header (two
   // arrivals), free once the consumers have read it (one); tensor memory for
   // the accumulators and the scales
-  static_assert(!UM || KIND == KIND_EGU || KIND == KIND_EDN, "tensor-core path: expert kernels only");
+  static_assert(!UM || KIND != KIND_FRONT, "tensor-core path: expert and tail kernels");
   constexpr bool um = UM;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm_flag + kUTmemWord);
   uint64_t* dfull = reinterpret_cast<uint64_t*>(sm_flag + kUDfullWord);
@@ -2269,7 +2318,7 @@ __global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
     }
     fence_mbar_init();
   }
-  if (um && warp == 0) umma::tmem_alloc(tmem_slot, tmem_cols<NT>());
+  if (um && warp == 0) umma::tmem_alloc(tmem_slot, tmem_cols<KIND, NT>());
   if (um) umma::fence_before_sync();
   __syncthreads();
   if (um) umma::fence_after_sync();
@@ -2284,7 +2333,7 @@ __global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
     producer<KIND>(p, ctl, stages, tables, full, empty, lane);
   } else if (UM && warp == kMmaWarp) {
     if (lane == 0)
-      mma_issuer<NT>(p, stages, full, empty, dfull, dfree, drain,
+      mma_issuer<KIND, NT>(p, stages, full, empty, dfull, dfree, drain,
                      reinterpret_cast<Hdr*>(smem + kUPqByte), *tmem_slot);
   } else {
     consumer<KIND, NT, UM>(p, stages, full, empty, scratch, sm_flag, slot_tab, warp, lane);
@@ -2293,7 +2342,7 @@ __global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
   __syncthreads();
   if (um && warp == 0) {
     umma::fence_after_sync();
-    umma::tmem_dealloc(*tmem_slot, tmem_cols<NT>());
+    umma::tmem_dealloc(*tmem_slot, tmem_cols<KIND, NT>());
   }
   if (p.trace && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * kTraceStride + 1] = global_ns();
   if (threadIdx.x == 0) {
@@ -2359,6 +2408,18 @@ static int launch_kind_nt(int nt, const Params& p0, int grid, size_t smem, cudaS
     }
   }
   constexpr bool kHalf = (KIND == KIND_FRONT || KIND == KIND_TAIL);
+  if constexpr (KIND == KIND_TAIL) {
+    if (p.umma) {  // the tensor-core tail (formed records)
+      p.umma = nt;
+      switch (nt) {
+        case 1: return launch_one<KIND, 1, 1, true>(p, grid, smem, s, pdl);
+        case 2: return launch_one<KIND, 2, 1, true>(p, grid, smem, s, pdl);
+        case 4: return launch_one<KIND, 4, 1, true>(p, grid, smem, s, pdl);
+        case 8: return launch_one<KIND, 8, 1, true>(p, grid, smem, s, pdl);
+        default: return (int)cudaErrorInvalidValue;
+      }
+    }
+  }
   if constexpr (kHalf) {
     if (p.half_sm) return nt == 1 ? launch_one<KIND, 1, 2>(p, grid, smem, s, pdl) : (int)cudaErrorInvalidValue;
   }
@@ -2387,6 +2448,9 @@ static int set_attr_kind(size_t bytes) {
     e |= set_attr<KIND, 1, 1, true>(bytes) | set_attr<KIND, 2, 1, true>(bytes) |
          set_attr<KIND, 4, 1, true>(bytes) | set_attr<KIND, 1, 2, true>(bytes) |
          set_attr<KIND, 2, 2, true>(bytes);
+  if constexpr (KIND == KIND_TAIL)
+    e |= set_attr<KIND, 1, 1, true>(bytes) | set_attr<KIND, 2, 1, true>(bytes) |
+         set_attr<KIND, 4, 1, true>(bytes) | set_attr<KIND, 8, 1, true>(bytes);
   return e;
 }
 

@@ -15,23 +15,38 @@ enum : int { DENSE_PLAIN = 0, DENSE_GATE_UP = 1, DENSE_TWO_K = 2 };
 // MXFP4 layouts
 enum : int { MX_PLAIN = 0, MX_GATE_UP = 1 };
 
+// Unit u of a tile is 16 bytes: 8 bf16 values.  Warp-MMA order: lane, k16
+// step, 32-block and warp tile of the m16n8k16 A fragments.  Tensor-core
+// order (umma): core-matrix slot u = (kb * 16 + rg) * 8 + rr holds row
+// 8 rg + rr, K elements 8 kb .. 8 kb + 7 of the chunk (row groups 128 bytes
+// apart, K blocks 2048).  Either way a row of the tile is row r of warp tile
+// w (16 rows each), as the epilogues expect.
 __global__ void pack_dense_kernel(const uint16_t* __restrict__ src, int K, int N, int layout,
                                   int RB, int C, uint8_t* __restrict__ dst,
-                                  const uint16_t* __restrict__ src2, int K2, int C_first) {
+                                  const uint16_t* __restrict__ src2, int K2, int C_first, int umma) {
   const long long units = (long long)RB * C * 1024;
   for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
        u += (long long)gridDim.x * blockDim.x) {
-    const int lane = u & 31, s = (u >> 5) & 1, b = (u >> 6) & 1, w = (u >> 7) & 7;
+    const int lane = u & 31, s = (u >> 5) & 1, b = (u >> 6) & 1, w0 = (u >> 7) & 7;
     const long long tile = u >> 10;
     const int rb = (int)(tile / C), c = (int)(tile % C);
     const int g = lane >> 2, t = lane & 3;
+    const int slot = (int)(u & 1023);
     uint16_t v[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int r = frag_row(g, q);  // row within the warp tile
-        const int kk = 32 * b + frag_k(t, s, q, e);
+        int w = w0, r, kk;
+        if (umma) {
+          const int row = ((slot >> 3) & 15) * 8 + (slot & 7);  // row within the tile
+          w = row >> 4;
+          r = row & 15;
+          kk = 8 * (slot >> 7) + 2 * q + e;
+        } else {
+          r = frag_row(g, q);  // row within the warp tile
+          kk = 32 * b + frag_k(t, s, q, e);
+        }
         const uint16_t* m = src;
         int col = -1, k = -1, kmax = K;
         if (layout == DENSE_PLAIN) {
@@ -61,8 +76,9 @@ __global__ void pack_dense_kernel(const uint16_t* __restrict__ src, int K, int N
     o.y = v[2] | ((uint32_t)v[3] << 16);
     o.z = v[4] | ((uint32_t)v[5] << 16);
     o.w = v[6] | ((uint32_t)v[7] << 16);
-    // [warp][blk][step][lane][16 B]
-    uint8_t* d = dst + tile * kDenseTileBytes + (((w * 2 + b) * 2 + s) * 32 + lane) * 16;
+    // [warp][blk][step][lane][16 B], or the core-matrix slot
+    uint8_t* d = dst + tile * kDenseTileBytes +
+                 (umma ? slot * 16 : (((w0 * 2 + b) * 2 + s) * 32 + lane) * 16);
     *reinterpret_cast<uint4*>(d) = o;
   }
 }
@@ -198,13 +214,13 @@ __global__ void pack_mx_kernel(const uint8_t* __restrict__ codes, const uint8_t*
 }
 
 int launch_pack_dense(const void* src, int K, int N, int layout, int RB, int C, int /*rows_valid*/,
-                      uint8_t* dst, void* stream, const void* src2, int K2, int C_first) {
+                      uint8_t* dst, void* stream, const void* src2, int K2, int C_first, int umma) {
   const long long units = (long long)RB * C * 1024;
   const int threads = 256;
   const int blocks = (int)((units + threads - 1) / threads < 65535 * 8 ? (units + threads - 1) / threads
                                                                          : 65535 * 8);
   pack_dense_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
-      (const uint16_t*)src, K, N, layout, RB, C, dst, (const uint16_t*)src2, K2, C_first);
+      (const uint16_t*)src, K, N, layout, RB, C, dst, (const uint16_t*)src2, K2, C_first, umma);
   return (int)cudaGetLastError();
 }
 

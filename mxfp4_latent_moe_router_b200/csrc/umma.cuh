@@ -2,8 +2,8 @@
 // sm_100a (tcgen05): tensor-memory allocation, shared-memory operand
 // descriptors, the block-scaled MMA with e2m1 operands on both sides
 // (kind::mxf4, one e8m0 scale per 32 K elements on each side, K = 64 per
-// instruction), scale copies into tensor memory, commit to an mbarrier and
-// loads of the fp32 accumulator.
+// instruction), the bf16 MMA (kind::f16, K = 16), scale copies into tensor
+// memory, commit to an mbarrier and loads of the fp32 accumulator.
 //
 // Layouts used here (all K-major, no swizzle):
 //   - an operand is a grid of "core matrices", each 8 rows x 16 bytes stored
@@ -11,7 +11,8 @@
 //     byte distance between core matrices adjacent along K (leading, LBO)
 //     and along M/N (stride, SBO);
 //   - e2m1 operands are packed: 16 bytes of a core-matrix row hold 32
-//     elements, element 2t in the low nibble of byte t;
+//     elements, element 2t in the low nibble of byte t; bf16 operands hold
+//     8 elements a core-matrix row;
 //   - scale factors: one byte per (row, 32-wide K block); four K blocks of
 //     128 rows form a 512-byte unit, byte (m % 32) * 16 + (m / 32) * 4 + kb,
 //     which one copy broadcasts into tensor-memory lanes 0-127, 4 columns:
@@ -78,6 +79,23 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint6
       " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate), "r"(sfa_tmem),
       "r"(sfb_tmem)
+      : "memory");
+}
+
+// ---- instruction descriptor, kind::f16 with bf16 operands ----------------------
+// bits 4-5 D format (1: f32), 7-9 A format (1: bf16), 10-12 B format (1: bf16),
+// 15/16 A/B major (0: K), 17-22 N >> 3, 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return 1u << 4 | 1u << 7 | 1u << 10 | (uint32_t)(N >> 3) << 17 | (uint32_t)(M >> 4) << 24;
+}
+
+// D[tmem] (+)= A . B^T, bf16 operands, K = 16; issued by one thread.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem), "l"(a_desc),
+      "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
       : "memory");
 }
 

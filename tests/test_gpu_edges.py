@@ -1,7 +1,8 @@
 """Edge cases of the CUDA path against the CPU oracle: the largest expert count
 and top-k the library takes, the largest batch, sigmoid scoring without a
 selection bias, the fused single launch with a tail activation too large to
-keep in shared memory, 32-token virtual experts, raw (unrenormalised)
+keep in shared memory, the tail on formed records (tensor-core and warp-level
+MMA), 32-token virtual experts, raw (unrenormalised)
 scores with a routed scale, and the host-side geometry query against a real
 plan."""
 import numpy as np
@@ -80,6 +81,20 @@ def test_fused_launch_with_staged_tail(monkeypatch):
     monkeypatch.setenv("MOE_FUSED", "1")
     monkeypatch.setenv("MOE_UMMA", "0")  # (the fused launch keeps the warp-level MMA)
     _check(shape, w, synth.make_x(shape), max_tokens=8)
+
+
+@pytest.mark.parametrize("umma_tail", ["1", "0"])
+@pytest.mark.parametrize("B", [5, 8, 37, 64, 77])
+def test_tail_from_formed_records(B, umma_tail, monkeypatch):
+    # L + I_s = 3072: the tail's activation is formed once per token group as
+    # bf16 hi/lo records (too large to keep resident from 6 tokens on); on the
+    # tensor cores the tail multiplies them with a bf16 MMA, the records' two
+    # parts as two rows a token.  1 to 8 token tiles, two passes at 77 tokens.
+    monkeypatch.setenv("MOE_UMMA_TAIL", umma_tail)
+    shape = synth.custom_shape("formed", B, 256, 1024, 16, 2, 128, 2048, synth.SCORE_SOFTMAX,
+                               seed=61 + B, scale_exp_lo=-5, scale_exp_hi=-2)
+    w = synth.make_weights(shape)
+    _check(shape, w, synth.make_x(shape), max_tokens=max(B, 8))
 
 
 @pytest.mark.parametrize("umma", ["1", "0"])
