@@ -99,6 +99,9 @@ struct Params {
   // records in that form.  0: the warp-level MMA; else nonzero, and at an
   // expert kernel's launch the token tiles of its stages (its NT)
   int umma;
+  // FRONT on the tensor cores (bf16 MMA of the weight rows with x): 0, or its
+  // token tiles (set at launch)
+  int front_umma;
   int act_rec;  // bytes of one activation record (kActRecBytes or kActRecBytesU)
   // EGU: the latent row blocks' finalisations count up here (release); the
   // expert gate/up kernel reads z once it reaches RB_lat instead of waiting

@@ -95,7 +95,8 @@ struct moe_plan_s {
   uint8_t* w_egu = nullptr;
   uint8_t* w_edn = nullptr;
   uint8_t* w_tail = nullptr;
-  uint8_t* w_tail_um = nullptr;  // the tail's tiles in the tensor-core order (umma_tail)
+  uint8_t* w_tail_um = nullptr;   // the tail's tiles in the tensor-core order (umma_tail)
+  uint8_t* w_front_um = nullptr;  // the front's tiles in the tensor-core order (umma_front)
   float* bias = nullptr;
 
   float* logits = nullptr;
@@ -142,6 +143,10 @@ struct moe_plan_s {
   // parts) whenever its activation is staged from formed records; needs a
   // second copy of the tail's tiles (environment MOE_UMMA_TAIL=0 turns it off)
   bool umma_tail = true;
+  // the front on the tensor cores (bf16 MMA with x) from two token tiles on;
+  // a second copy of the front's tiles (environment MOE_UMMA_FRONT=0 turns it off)
+  bool umma_front = true;
+  bool w_front_um_ok = false;  // umma_front, and the plan takes more than 8 tokens
   int* err = nullptr;
   uint16_t* x_stage = nullptr;
   uint16_t* out_stage = nullptr;
@@ -247,6 +252,12 @@ moe_status alloc(moe_plan p, void** out, size_t bytes, bool packed) {
 
 bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
 
+// Whether the front runs on the tensor cores: two token tiles or more (its
+// MMA needs N >= 16), the whole SM (no side lane).
+bool front_umma_for(const moe_plan_s* p, int nt, int budget) {
+  return p->w_front_um_ok && nt >= 2 && budget > kHalfSmem;
+}
+
 int scratch_bytes(const moe_plan_s* p, int kind, int nt) {
   return ((kind == KIND_EGU || kind == KIND_EDN) && p->umma && nt <= 2) ? kScratchBytesUmmaSmall
                                                                           : kScratchBytes;
@@ -277,7 +288,8 @@ SmemGeom smem_geom(const moe_plan_s* p, int kind, int nt, int tail_tg_eff, int s
   s.act_stride = 0;
   if (kind == KIND_FRONT) {
     s.act_stride = 192;
-    act = 8 * nt * s.act_stride;
+    // (the tensor-core front: 128 bytes a token, in core matrices)
+    act = front_umma_for(p, nt, budget) ? 8 * nt * 128 : 8 * nt * s.act_stride;
   } else if ((kind == KIND_EGU || kind == KIND_EDN) && p->umma) {
     // tensor-core stage: unpacked codes, scales, the token-term rows
     s.act_stride = 0;
@@ -632,6 +644,9 @@ void read_env(moe_plan_s* p) {
   if (const char* e = getenv("MOE_UMMA")) p->umma = atoi(e) != 0;
   if (const char* e = getenv("MOE_UMMA_TAIL")) p->umma_tail = atoi(e) != 0;
   p->umma_tail = p->umma_tail && p->umma;
+  if (const char* e = getenv("MOE_UMMA_FRONT")) p->umma_front = atoi(e) != 0;
+  p->umma_front = p->umma_front && p->umma;
+  p->w_front_um_ok = p->umma_front && p->cfg.max_tokens > 8;
   p->act_rec = p->umma ? kActRecBytesU : kActRecBytes;
   if (p->umma) p->use_fused = false;  // the single launch keeps the warp-level MMA
 }
@@ -679,6 +694,10 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
   void* v;
   TRY(alloc(p, &v, fr.weight_bytes, true));
   p->w_front = (uint8_t*)v;
+  if (p->w_front_um_ok) {  // (the tensor-core front takes more than 8 tokens)
+    TRY(alloc(p, &v, fr.weight_bytes, true));
+    p->w_front_um = (uint8_t*)v;
+  }
   TRY(alloc(p, &v, (size_t)E * eg.weight_bytes, true));
   p->w_egu = (uint8_t*)v;
   TRY(alloc(p, &v, (size_t)E * ed.weight_bytes, true));
@@ -974,6 +993,10 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       q.rpart = p->rpart;
       q.PPR_r = std::min(q.C, 16);
     }
+    if (front_umma_for(p, f.nt_front, f.budget) && !f.side && !q.rpart) {
+      q.front_umma = 1;
+      q.wt = p->w_front_um;
+    }
     TRY(launch_timed(p, KIND_FRONT, KIND_FRONT, f.nt_front, q, l.grid, l.sm.total, s));
   }
   {
@@ -1147,15 +1170,18 @@ moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
   // from [H][N] tensors
   const KindGeom& fr = p->g[KIND_FRONT];
   const size_t rb_bytes = (size_t)fr.C * kDenseTileBytes;
-  CUDA_TRY((cudaError_t)launch_pack_dense(w->router_w, H, E, 0, p->RB_router, fr.C, E, p->w_front,
-                                          s, nullptr, 0, 0));
-  CUDA_TRY((cudaError_t)launch_pack_dense(w->w_in, H, L, 0, p->RB_lat, fr.C, L,
-                                          p->w_front + p->RB_router * rb_bytes, s, nullptr, 0, 0));
-  if (Is > 0)
-    CUDA_TRY((cudaError_t)launch_pack_dense(w->sh_gate, H, Is, 1, fr.RB - p->RB_router - p->RB_lat,
-                                            fr.C, Is,
-                                            p->w_front + (p->RB_router + p->RB_lat) * rb_bytes, s,
-                                            w->sh_up, 0, 0));
+  // the front's tiles, and their tensor-core copy when the plan has one
+  for (int um = 0; um < (p->w_front_um ? 2 : 1); ++um) {
+    uint8_t* wf = um ? p->w_front_um : p->w_front;
+    CUDA_TRY((cudaError_t)launch_pack_dense(w->router_w, H, E, 0, p->RB_router, fr.C, E, wf, s,
+                                            nullptr, 0, 0, um));
+    CUDA_TRY((cudaError_t)launch_pack_dense(w->w_in, H, L, 0, p->RB_lat, fr.C, L,
+                                            wf + p->RB_router * rb_bytes, s, nullptr, 0, 0, um));
+    if (Is > 0)
+      CUDA_TRY((cudaError_t)launch_pack_dense(w->sh_gate, H, Is, 1, fr.RB - p->RB_router - p->RB_lat,
+                                              fr.C, Is, wf + (p->RB_router + p->RB_lat) * rb_bytes, s,
+                                              w->sh_up, 0, 0, um));
+  }
   const KindGeom& tl = p->g[KIND_TAIL];
   CUDA_TRY((cudaError_t)launch_pack_dense(w->w_out, L, H, 2, tl.RB, tl.C, H, p->w_tail, s,
                                           Is > 0 ? w->sh_down : w->w_out, Is, p->C_lat));

@@ -257,6 +257,7 @@ template <int KIND>
 __device__ __forceinline__ bool rows_async(const Params& p, const Hdr& h) {
   if ((KIND == KIND_EGU || KIND == KIND_EDN || KIND == KIND_TAIL) && p.umma)
     return true;  // scattered into the MMA's B layout
+  if (KIND == KIND_FRONT && p.front_umma) return true;
   return (KIND == KIND_FRONT || KIND == KIND_EGU || KIND == KIND_EDN) && h.ntok > kBulkRowsMax;
 }
 
@@ -380,6 +381,24 @@ __device__ __forceinline__ void copy_tail_records_umma(const Params& p, const Hd
   rows_async_done(bar, lane);
 }
 
+// Tensor-core front stage: the tokens' x rows of this 64-wide chunk into the
+// B operand's core-matrix layout (token n's K block kb at (kb * NT + n / 8) *
+// 128 + (n % 8) * 16); K blocks past the chunk's valid blocks (a ragged last
+// chunk) are zero-filled, reading nothing.
+__device__ __forceinline__ void copy_x_rows_umma(const Params& p, const Hdr& h, uint8_t* B,
+                                                 uint64_t* bar, int lane, int nt) {
+  const uint8_t* x = reinterpret_cast<const uint8_t*>(p.x + h.chunk * kDenseChunkK);
+  const int kb_valid = h.nb * 4;  // 16-byte K blocks holding real columns
+  for (int tok = lane; tok < h.ntok; tok += 32) {
+    const uint8_t* src = x + (long long)tok * p.H * 2;
+    uint8_t* dst = B + (tok >> 3) * 128 + (tok & 7) * 16;
+#pragma unroll
+    for (int q = 0; q < kDenseChunkK / 8; ++q)
+      cp_async16_zfill(dst + q * nt * 128, q < kb_valid ? src + q * 16 : src, q < kb_valid ? 16u : 0u);
+  }
+  rows_async_done(bar, lane);
+}
+
 // Issue this stage's activation copies (all 32 producer lanes).
 template <int KIND>
 __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t* act, uint64_t* bar,
@@ -390,6 +409,10 @@ __device__ __forceinline__ void issue_act(const Params& p, const Hdr& h, uint8_t
   }
   if (KIND == KIND_TAIL && p.umma) {
     copy_tail_records_umma(p, h, act, bar, lane, p.umma);  // (umma = NT)
+    return;
+  }
+  if (KIND == KIND_FRONT && p.front_umma) {
+    copy_x_rows_umma(p, h, act, bar, lane, p.front_umma);  // (front_umma = NT)
     return;
   }
   if (rows_async<KIND>(p, h)) {
@@ -1874,16 +1897,25 @@ __device__ __forceinline__ void finalize(const Params& p, const Hdr& h, float (&
 // SM), at four 512.
 // The tail's bf16 MMA (its activation as hi and lo parts, two rows a token)
 // needs no scale columns: 2 x 16 NT accumulator columns.
+// (the front's bf16 MMA: x once, one row a token)
 template <int KIND>
-__host__ __device__ constexpr int umma_terms() { return KIND == KIND_TAIL ? 2 : kUTerms; }
+__host__ __device__ constexpr int umma_terms() {
+  return KIND == KIND_TAIL ? 2 : KIND == KIND_FRONT ? 1 : kUTerms;
+}
 template <int KIND, int NT>
 __host__ __device__ constexpr uint32_t tmem_dcols() { return (uint32_t)(umma_terms<KIND>() * 8 * NT); }
 template <int KIND, int NT>
 __host__ __device__ constexpr uint32_t tmem_sf() { return 2 * tmem_dcols<KIND, NT>(); }
 template <int KIND, int NT>
 __host__ __device__ constexpr uint32_t tmem_cols() {
-  return KIND == KIND_TAIL ? (NT <= 4 ? 128u : 256u) : (NT <= 2 ? 256u : 512u);
+  // (a power of two, at least 32: two accumulator buffers, and the expert
+  // kernels' scale columns)
+  return KIND == KIND_FRONT ? (NT <= 2 ? 32u : NT == 4 ? 64u : NT == 8 ? 128u : 256u)
+         : KIND == KIND_TAIL ? (NT <= 4 ? 128u : 256u)
+                             : (NT <= 2 ? 256u : 512u);
 }
+static_assert(tmem_sf<KIND_FRONT, 16>() <= tmem_cols<KIND_FRONT, 16>(), "two accumulator buffers");
+static_assert(tmem_sf<KIND_FRONT, 2>() <= tmem_cols<KIND_FRONT, 2>(), "two accumulator buffers");
 static_assert(tmem_sf<KIND_EGU, 1>() + 16 * kMaxStages <= tmem_cols<KIND_EGU, 1>(), "scale columns");
 static_assert(tmem_sf<KIND_EGU, 2>() + 16 * kMaxStages <= tmem_cols<KIND_EGU, 2>(), "scale columns");
 static_assert(tmem_sf<KIND_EGU, 4>() + 16 * kMaxStages <= tmem_cols<KIND_EGU, 4>(), "scale columns");
@@ -1929,8 +1961,9 @@ __device__ void mma_issuer(const Params& p, uint8_t* stage_base, uint64_t* full,
     fence_proxy_async_smem();  // the activation rows came in by cp.async
     umma::fence_after_sync();
     const uint32_t d = tmem + (uint32_t)buf * tmem_dcols<KIND, NT>();
-    if constexpr (KIND == KIND_TAIL) {
-      // bf16 weights (128 x 64 K) x the records' hi and lo rows: four K = 16
+    if constexpr (KIND == KIND_TAIL || KIND == KIND_FRONT) {
+      // bf16 weights (128 x 64 K) x the records' hi and lo rows (tail) or the
+      // x rows (front): four K = 16
       const uint8_t* A = sb + kHdrBytes;
       const uint8_t* B = sb + p.act_off;
 #pragma unroll
@@ -2298,7 +2331,8 @@ __global__ void __launch_bounds__(UM ? kThreadsU : kThreads, MINB)
   // completed and the MMA warp has written the piece's header (two
   // arrivals), free once the consumers have read it (one); tensor memory for
   // the accumulators and the scales
-  static_assert(!UM || KIND != KIND_FRONT, "tensor-core path: expert and tail kernels");
+  static_assert(!UM || MINB == 1 || KIND == KIND_EGU || KIND == KIND_EDN,
+                "two tensor-core CTAs an SM: expert kernels only");
   constexpr bool um = UM;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm_flag + kUTmemWord);
   uint64_t* dfull = reinterpret_cast<uint64_t*>(sm_flag + kUDfullWord);
@@ -2408,6 +2442,18 @@ static int launch_kind_nt(int nt, const Params& p0, int grid, size_t smem, cudaS
     }
   }
   constexpr bool kHalf = (KIND == KIND_FRONT || KIND == KIND_TAIL);
+  if constexpr (KIND == KIND_FRONT) {
+    if (p.front_umma) {  // the tensor-core front (two token tiles or more)
+      p.front_umma = nt;
+      switch (nt) {
+        case 2: return launch_one<KIND, 2, 1, true>(p, grid, smem, s, pdl);
+        case 4: return launch_one<KIND, 4, 1, true>(p, grid, smem, s, pdl);
+        case 8: return launch_one<KIND, 8, 1, true>(p, grid, smem, s, pdl);
+        case 16: return launch_one<KIND, 16, 1, true>(p, grid, smem, s, pdl);
+        default: return (int)cudaErrorInvalidValue;
+      }
+    }
+  }
   if constexpr (KIND == KIND_TAIL) {
     if (p.umma) {  // the tensor-core tail (formed records)
       p.umma = nt;
@@ -2451,6 +2497,9 @@ static int set_attr_kind(size_t bytes) {
   if constexpr (KIND == KIND_TAIL)
     e |= set_attr<KIND, 1, 1, true>(bytes) | set_attr<KIND, 2, 1, true>(bytes) |
          set_attr<KIND, 4, 1, true>(bytes) | set_attr<KIND, 8, 1, true>(bytes);
+  if constexpr (KIND == KIND_FRONT)
+    e |= set_attr<KIND, 2, 1, true>(bytes) | set_attr<KIND, 4, 1, true>(bytes) |
+         set_attr<KIND, 8, 1, true>(bytes) | set_attr<KIND, 16, 1, true>(bytes);
   return e;
 }
 

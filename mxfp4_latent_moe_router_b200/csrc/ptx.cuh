@@ -83,6 +83,13 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem)
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
                : "memory");
 }
+// 16 bytes of which the first src_bytes (0 or 16) come from global memory and
+// the rest are zero (with 0 nothing is read)
+__device__ __forceinline__ void cp_async16_zfill(void* dst_smem, const void* src_gmem, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem),
+               "r"(src_bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src_gmem) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
                : "memory");
