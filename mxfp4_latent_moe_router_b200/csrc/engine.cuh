@@ -117,6 +117,7 @@ struct Params {
   int RB_lat;         // FRONT: row blocks of the latent projection (after the router's);
                       // the shared expert's gate/up row blocks follow
   int route_cta;      // FRONT: routing CTAs, the grid's last ones (no pieces); 0: none
+  int route_few;      // FRONT, B * k <= 32 with direct logits: the one-warp table build
   int tg;             // tokens per group (EGU/EDN/TAIL)
   int KL;             // K extent of the chunked dimension (for ragged last chunk)
   int KS;             // TAIL: K extent of the shared part (I_s)

@@ -138,6 +138,9 @@ struct moe_plan_s {
   // b64 452.2 us with 8 tokens a CTA against 458.2 with 16; b8 and b128 the
   // same within noise (b128 351.7 vs 351.5)
   int route_tpc = 8, route_max_ctas = 16;
+  // few tokens: the selection and table build of route_few (environment
+  // MOE_ROUTE_FEW=0: the general path)
+  bool route_few = true;
   // expert kernels on the 5th-generation tensor cores (block-scaled MMA of
   // e2m1 weights and e4m3 activation terms; environment MOE_UMMA=0 keeps
   // the warp-level MMA): decides the expert tiles' packed order and the
@@ -646,6 +649,7 @@ void read_env(moe_plan_s* p) {
   if (const char* e = getenv("MOE_SIDE_LANE")) p->side_env_off = atoi(e) == 0;
   if (const char* e = getenv("MOE_PREFETCH_MB")) p->prefetch_bytes = std::max(0LL, (long long)atoi(e)) << 20;
   if (const char* e = getenv("MOE_DIRECT_ROUTE")) p->direct_route = atoi(e) != 0;
+  if (const char* e = getenv("MOE_ROUTE_FEW")) p->route_few = atoi(e) != 0;
   if (const char* e = getenv("MOE_ROUTE_TPC")) p->route_tpc = std::max(1, std::min(128, atoi(e)));
   if (const char* e = getenv("MOE_ROUTE_MAX_CTAS")) p->route_max_ctas = std::max(1, std::min(32, atoi(e)));
   if (const char* e = getenv("MOE_CONS_SLEEP")) p->cons_sleep = std::max(0, std::min(2000, atoi(e)));
@@ -1000,6 +1004,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       // every load of a round in flight
       q.rpart = p->rpart;
       q.PPR_r = std::min(q.C, 16);
+      q.route_few = p->route_few ? 1 : 0;
     }
     if (front_umma_for(p, f.nt_front, f.budget) && !f.side && !q.rpart) {
       q.front_umma = 1;

@@ -1717,6 +1717,64 @@ __device__ __forceinline__ bool route_poll_logits(const Params& p, float* lgs, i
   return false;
 }
 
+// Few tokens (B * k <= 32, logits in shared memory): one warp a token
+// selects its experts over all of them, then warp 0 sorts the B * k (expert,
+// slot) pairs across its lanes (bitonic) and writes the tables itself: a
+// virtual expert per run of equal experts (at most B <= tg tokens), its
+// positions in slot order.  Two barriers instead of the general path's
+// slices, merge and CTA-wide scan, each of which costs several µs while the
+// weights stream.
+__device__ __forceinline__ void route_few(const Params& p, const float* bias, const float* lg_sm,
+                                          int* ids_s, int warp, int lane) {
+  const int K = p.topk, B = p.B, E = p.E;
+  if (warp < B) {
+    int sel_id;
+    float sel_w;
+    warp_topk<true>(lg_sm + (long long)warp * E, E, K, p.score_fn, bias, p.renorm, p.routed_scale,
+                    lane, sel_id, sel_w);
+    if (lane < K) {
+      p.ids[warp * K + lane] = sel_id;
+      p.wts[warp * K + lane] = sel_w;
+      ids_s[warp * K + lane] = sel_id;
+    }
+  }
+  named_sync(1, kConsumerThreads);
+  if (warp == 0) {
+    const int n = B * K;
+    // expert in the high bits, slot in the low 6; lanes past n sort last
+    uint32_t key = lane < n ? ((uint32_t)ids_s[lane] << 6) | (uint32_t)lane : 0xFFFFFFFFu;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, key, j);
+        const bool ascending = (lane & k) == 0, lower = (lane & j) == 0;
+        key = (lower == ascending) ? min(key, other) : max(key, other);
+      }
+    const int e = (int)(key >> 6), slot = (int)(key & 63u);
+    const int prev_e = __shfl_up_sync(0xffffffffu, e, 1);
+    const bool valid = lane < n;
+    const bool start = valid && (lane == 0 || prev_e != e);
+    const uint32_t starts = __ballot_sync(0xffffffffu, start);
+    const uint32_t upto = lane == 31 ? 0xFFFFFFFFu : ((2u << lane) - 1u);  // lanes 0..lane
+    if (valid) p.slots_sorted[lane] = slot;
+    if (start) {
+      const int v = __popc(starts & upto) - 1;
+      const uint32_t later = starts & ~upto;
+      const int next = later ? __ffs(later) - 1 : n;
+      VExpert ve;
+      ve.expert = e;
+      ve.start = lane;
+      ve.count = next - lane;
+      ve.pad = 0;
+      p.ve[v] = ve;
+      if (p.h_done) p.h_done[v] = 0;
+    }
+    if (lane == 0) *p.nve = __popc(starts);
+  }
+  named_sync(1, kConsumerThreads);  // (every table write precedes the release)
+}
+
 __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, float* bias_s,
                                           int* sm_flag, int tid, int warp, int lane, int pstride) {
   unsigned long long* tr = p.trace ? p.trace + (size_t)blockIdx.x * kTraceStride : nullptr;
@@ -1741,8 +1799,11 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
     named_sync(1, kConsumerThreads);
     if (!ok) return;
     if (tr && tid == 0) tr[4] = global_ns();
-    route_tokens(p, bias, scratch, lgs + p.B * p.E, ring_floats - bias_floats - p.B * p.E,
-                 sm_flag + 16, tid, warp, lane, lgs);  // ends with a barrier
+    if (p.B * p.topk <= 32 && p.route_few)
+      route_few(p, bias, lgs, reinterpret_cast<int*>(scratch), warp, lane);  // ends with a barrier
+    else
+      route_tokens(p, bias, scratch, lgs + p.B * p.E, ring_floats - bias_floats - p.B * p.E,
+                   sm_flag + 16, tid, warp, lane, lgs);  // ends with a barrier
     if (tid == 0) {
       if (tr) tr[5] = global_ns();
       st_release(p.route_ready, 1);
