@@ -1004,8 +1004,8 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
       // every load of a round in flight
       q.rpart = p->rpart;
       q.PPR_r = std::min(q.C, 16);
-      q.route_few = p->route_few ? 1 : 0;
     }
+    q.route_few = p->route_few ? 1 : 0;
     if (front_umma_for(p, f.nt_front, f.budget) && !f.side && !q.rpart) {
       q.front_umma = 1;
       q.wt = p->w_front_um;

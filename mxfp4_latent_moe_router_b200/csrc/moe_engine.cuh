@@ -1717,15 +1717,17 @@ __device__ __forceinline__ bool route_poll_logits(const Params& p, float* lgs, i
   return false;
 }
 
-// Few tokens (B * k <= 32, logits in shared memory): one warp a token
-// selects its experts over all of them, then warp 0 sorts the B * k (expert,
-// slot) pairs across its lanes (bitonic) and writes the tables itself: a
-// virtual expert per run of equal experts (at most B <= tg tokens), its
-// positions in slot order.  Two barriers instead of the general path's
-// slices, merge and CTA-wide scan, each of which costs several µs while the
-// weights stream.
+// Few tokens (B <= 8, B * k <= 64, logits in shared memory): one warp a
+// token selects its experts over all of them, then warp 0 sorts the B * k
+// (expert, slot) pairs (bitonic, two a lane: positions 2 lane and 2 lane + 1)
+// and writes the tables itself: a virtual expert per run of equal experts
+// (at most B <= tg tokens), its positions in slot order.  Two barriers
+// instead of the general path's slices, merge and CTA-wide scan, each of
+// which costs several µs while the weights stream.  es: 64 ints of shared
+// memory (the sorted experts, for the run lengths).
+constexpr int kRouteFewSlots = 64;
 __device__ __forceinline__ void route_few(const Params& p, const float* bias, const float* lg_sm,
-                                          int* ids_s, int warp, int lane) {
+                                          int* ids_s, int* es, int warp, int lane) {
   const int K = p.topk, B = p.B, E = p.E;
   if (warp < B) {
     int sel_id;
@@ -1741,36 +1743,68 @@ __device__ __forceinline__ void route_few(const Params& p, const float* bias, co
   named_sync(1, kConsumerThreads);
   if (warp == 0) {
     const int n = B * K;
-    // expert in the high bits, slot in the low 6; lanes past n sort last
-    uint32_t key = lane < n ? ((uint32_t)ids_s[lane] << 6) | (uint32_t)lane : 0xFFFFFFFFu;
+    // expert in the high bits, slot in the low 6; positions past n sort last
+    uint32_t key[2];
 #pragma unroll
-    for (int k = 2; k <= 32; k <<= 1)
+    for (int h = 0; h < 2; ++h) {
+      const int pos = 2 * lane + h;
+      key[h] = pos < n ? ((uint32_t)ids_s[pos] << 6) | (uint32_t)pos : 0xFFFFFFFFu;
+    }
+#pragma unroll
+    for (int k = 2; k <= kRouteFewSlots; k <<= 1) {
+      const bool ascending = ((2 * lane) & k) == 0;  // (bit k >= 2 is the lane's for both)
 #pragma unroll
       for (int j = k >> 1; j > 0; j >>= 1) {
-        const uint32_t other = __shfl_xor_sync(0xffffffffu, key, j);
-        const bool ascending = (lane & k) == 0, lower = (lane & j) == 0;
-        key = (lower == ascending) ? min(key, other) : max(key, other);
+        if (j == 1) {  // the lane's two positions
+          const uint32_t lo = min(key[0], key[1]), hi = max(key[0], key[1]);
+          key[0] = ascending ? lo : hi;
+          key[1] = ascending ? hi : lo;
+        } else {
+          const bool lower = (lane & (j >> 1)) == 0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, key[h], j >> 1);
+            key[h] = (lower == ascending) ? min(key[h], other) : max(key[h], other);
+          }
+        }
       }
-    const int e = (int)(key >> 6), slot = (int)(key & 63u);
-    const int prev_e = __shfl_up_sync(0xffffffffu, e, 1);
-    const bool valid = lane < n;
-    const bool start = valid && (lane == 0 || prev_e != e);
-    const uint32_t starts = __ballot_sync(0xffffffffu, start);
-    const uint32_t upto = lane == 31 ? 0xFFFFFFFFu : ((2u << lane) - 1u);  // lanes 0..lane
-    if (valid) p.slots_sorted[lane] = slot;
-    if (start) {
-      const int v = __popc(starts & upto) - 1;
-      const uint32_t later = starts & ~upto;
-      const int next = later ? __ffs(later) - 1 : n;
-      VExpert ve;
-      ve.expert = e;
-      ve.start = lane;
-      ve.count = next - lane;
-      ve.pad = 0;
-      p.ve[v] = ve;
-      if (p.h_done) p.h_done[v] = 0;
     }
-    if (lane == 0) *p.nve = __popc(starts);
+    const int e0 = (int)(key[0] >> 6), e1 = (int)(key[1] >> 6);
+    es[2 * lane] = e0;
+    es[2 * lane + 1] = e1;
+    const int prev1 = __shfl_up_sync(0xffffffffu, e1, 1);  // position 2 lane - 1
+    const bool st0 = 2 * lane < n && (lane == 0 || prev1 != e0);
+    const bool st1 = 2 * lane + 1 < n && e1 != e0;
+    // virtual expert index: run starts up to each position (warp prefix sum)
+    const int c = (int)st0 + (int)st1;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    const int excl = incl - c;
+    __syncwarp();  // es complete
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int pos = 2 * lane + h;
+      if (pos < n) p.slots_sorted[pos] = (int)(key[h] & 63u);
+      const bool st = h == 0 ? st0 : st1;
+      if (st) {
+        const int v = excl + (h == 0 ? 0 : (int)st0);
+        const int e = h == 0 ? e0 : e1;
+        int len = 1;
+        while (pos + len < n && es[pos + len] == e) ++len;  // (a run holds at most B tokens)
+        VExpert ve;
+        ve.expert = e;
+        ve.start = pos;
+        ve.count = len;
+        ve.pad = 0;
+        p.ve[v] = ve;
+        if (p.h_done) p.h_done[v] = 0;
+      }
+    }
+    if (lane == 31) *p.nve = incl;
   }
   named_sync(1, kConsumerThreads);  // (every table write precedes the release)
 }
@@ -1799,8 +1833,9 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
     named_sync(1, kConsumerThreads);
     if (!ok) return;
     if (tr && tid == 0) tr[4] = global_ns();
-    if (p.B * p.topk <= 32 && p.route_few)
-      route_few(p, bias, lgs, reinterpret_cast<int*>(scratch), warp, lane);  // ends with a barrier
+    if (p.B * p.topk <= kRouteFewSlots && p.route_few)
+      route_few(p, bias, lgs, reinterpret_cast<int*>(scratch),
+                reinterpret_cast<int*>(scratch) + kRouteFewSlots, warp, lane);  // ends with a barrier
     else
       route_tokens(p, bias, scratch, lgs + p.B * p.E, ring_floats - bias_floats - p.B * p.E,
                    sm_flag + 16, tid, warp, lane, lgs);  // ends with a barrier
@@ -1825,6 +1860,21 @@ __device__ __forceinline__ void route_cta(const Params& p, uint8_t* scratch, flo
   named_sync(1, kConsumerThreads);  // thread 0's acquire covers the others' logit reads
   if (!sm_flag[0]) return;
   if (tr && tid == 0) tr[4] = global_ns();
+  if (p.route_cta == 1 && p.B <= kConsumerWarps && p.B * p.topk <= kRouteFewSlots && p.route_few) {
+    // few tokens: their logits into the idle ring with every load in flight,
+    // then the one-warp table build
+    float* lgs = bias_s + bias_floats;
+    stage_floats(p.logits, p.B * p.E, lgs, tid);
+    named_sync(1, kConsumerThreads);
+    route_few(p, bias, lgs, reinterpret_cast<int*>(scratch), reinterpret_cast<int*>(scratch) + kRouteFewSlots,
+              warp, lane);  // ends with a barrier
+    if (tid == 0) {
+      if (tr) tr[5] = global_ns();
+      *p.router_done = 0;
+      st_release(p.route_ready, 1);
+    }
+    return;
+  }
   // this routing CTA's share of the tokens
   const int R = p.route_cta;
   const int r = (int)blockIdx.x - ((int)gridDim.x - R);
