@@ -158,13 +158,26 @@ typedef struct moe_plan_info {
  *                           (block-scaled e2m1 x e2m1 MMA, activations as four
  *                           e2m1 terms); fixes the packed weight order, so it
  *                           holds for the plan's life.  MOE_UMMA=0 also allows
- *                           MOE_FUSED, which keeps the warp-level MMA
+ *                           MOE_FUSED, which keeps the warp-level MMA, and
+ *                           keeps the front and tail on the warp-level MMA
+ *   MOE_UMMA_TAIL=0         the tail keeps the warp-level MMA (default: bf16
+ *                           tensor-core MMA when its activation comes from
+ *                           formed records; a second copy of its tiles)
+ *   MOE_UMMA_FRONT=0        the front keeps the warp-level MMA (default: bf16
+ *                           tensor-core MMA above 8 tokens, for plans of more
+ *                           than 8 tokens; a second copy of its tiles)
  *   MOE_EXPERT_CTAS_PER_SM=1  one CTA per SM for the expert kernels (default
  *                           2 at one token tile, and at two on the tensor cores)
  *   MOE_EXPERT_SMALL_MAX_B=n  largest B with 8-token virtual experts (16-token
  *                           ones on the tensor cores above B = 64; default
  *                           128; above it, 32-token groups)
  *   MOE_EXPERT_TG=8|16|32   tokens per virtual expert for every B
+ *   MOE_EXPERT_PPR=n        the expert kernels' split-K factor (default: the
+ *                           makespan model, chosen on the device)
+ *   MOE_ROUTE_TPC=n, MOE_ROUTE_MAX_CTAS=n  tokens per routing CTA and the
+ *                           most routing CTAs (defaults 8 and 16)
+ *   MOE_ROUTE_FEW=0         no one-warp selection and table build for B <= 8
+ *                           with B * k <= 64 (the general path instead)
  *   MOE_SIDE_LANE=0         no side lane, whatever shared_sms says
  *   MOE_TAIL_SPLIT=0        the tail's shared-expert part is not scheduled first
  *   MOE_Z_FLAG=0            expert gate/up waits for the whole front kernel
