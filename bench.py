@@ -300,6 +300,10 @@ def measure_workload(name, args, rank, local, dist, headline):
         p.load(dw, stream)
         del dw
         plans.append(p)
+    if args.next_layer_prefetch_mb > 0 and INSTANCES > 1:
+        # each instance is the next layer of the one before it
+        for k in range(INSTANCES):
+            plans[k].set_next_layer(plans[(k + 1) % INSTANCES], args.next_layer_prefetch_mb << 20)
     torch.cuda.synchronize()
     xs = [torch.from_numpy(synth.make_x(shape, step=s).view(np.int16)).cuda() for s in range(INPUT_POOL)]
     outs = [torch.empty_like(x) for x in xs]
@@ -527,6 +531,7 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": _workload_desc(shape), "tokens_per_step": B,
                        "weight_instances": args.instances,
+                       "next_layer_prefetch_mb": args.next_layer_prefetch_mb if args.instances > 1 else 0,
                        "l2": "inputs larger than L2: %d weight instances rotate, %.0f MB touched per step"
                              % (args.instances, head["step_bytes"] / 1e6),
                        "parallelism": "replicas" if ws > 1 else "single GPU"},
@@ -563,6 +568,9 @@ def main():
     ap.add_argument("--workload", default="b1", choices=["tiny", "b1", "b8", "b64", "b128"])
     ap.add_argument("--instances", type=int, default=4,
                     help="resident weight instances rotated per step (4 keeps every step out of L2)")
+    ap.add_argument("--next-layer-prefetch-mb", type=int, default=0,
+                    help="MB of the next instance's front weights each forward pulls into L2 "
+                         "(moe_set_next_layer; the instances stand for consecutive layers)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--shared-sms", type=int, default=0,

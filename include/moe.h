@@ -360,6 +360,29 @@ MOE_API moe_status moe_route_noalloc(const void *x, const void *router_w, const 
                                      int32_t top_k, int32_t score_fn, int32_t renormalize,
                                      float routed_scale, int32_t *ids, float *weights, void *stream);
 
+/*
+ * Cross-layer weight prefetch ("Hyper Optimizing Kimi K3 in vLLM", section
+ * 从算子之间找时间: fetch the next step's weights while HBM is under-used).
+ * From now on every forward of `p` also pulls the first `bytes` bytes of
+ * `next`'s front weights into L2: the router rows first, then the latent
+ * projection's, then the shared expert's gate/up rows (the order in which
+ * next's front kernel streams them).  The requests are issued by p's expert
+ * down kernel once each of its CTAs has issued its own stages, so they fill
+ * the HBM idle time of p's expert and tail phases; a forward of `next` that
+ * follows on the same GPU then reads those rows from L2.
+ *   next   a live plan on the same device (it may be p itself), or NULL
+ *   bytes  clamped to next's front weight size and rounded down to 16;
+ *          0 or next == NULL turns the prefetch off
+ * Results are unchanged: only where next's front kernel finds its weights.
+ * Destroying `next` turns the prefetch off on every plan that names it.  A
+ * captured CUDA graph keeps the pointer it was captured with: keep `next`
+ * alive while such a graph may run.
+ * Errors: MOE_ERR_INVALID_ARG for a p or next that is not a live plan,
+ * bytes < 0, or plans on different devices (p is then unchanged).
+ * Host-side only; thread-safe with respect to plan creation and destruction.
+ */
+MOE_API moe_status moe_set_next_layer(moe_plan p, moe_plan next, int64_t bytes);
+
 /* Release everything the plan owns.  NULL is ignored. */
 MOE_API void moe_plan_destroy(moe_plan p);
 

@@ -27,7 +27,7 @@ ABI_SYMBOLS = ["moe_plan_create", "moe_load_weights", "moe_forward", "moe_forwar
                "moe_last_routing", "moe_debug_fetch", "moe_sync_status", "moe_get_plan_info",
                "moe_plan_destroy", "moe_status_str", "moe_set_profiling", "moe_get_profile",
                "moe_route_noalloc", "moe_debug_trace", "moe_debug_geometry",
-               "moe_debug_expire_wait"]
+               "moe_debug_expire_wait", "moe_set_next_layer"]
 # launch slots: the four kernels a forward runs (the dense front kernel
 # streams the router, latent-projection and shared-expert gate/up rows and
 # runs top-k), then the single fused launch that MOE_FUSED=1 selects for
@@ -97,6 +97,7 @@ def load_library():
     lib.moe_debug_expire_wait.argtypes = [P, ctypes.c_int32, P]
     lib.moe_get_plan_info.argtypes = [P, ctypes.POINTER(moe_plan_info)]
     lib.moe_plan_destroy.argtypes = [P]
+    lib.moe_set_next_layer.argtypes = [P, P, ctypes.c_int64]
     lib.moe_plan_destroy.restype = None
     lib.moe_route_noalloc.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                       ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
@@ -226,6 +227,11 @@ def moe_debug_geometry(cfg: moe_config, num_sms: int, num_tokens: int) -> list:
     return [{f[0]: getattr(g, f[0]) for f in moe_geometry._fields_} for g in out]
 
 
+def moe_set_next_layer(plan: int, next_plan, nbytes: int) -> int:
+    """Cross-layer prefetch of next_plan's front weights (see include/moe.h)."""
+    return load_library().moe_set_next_layer(plan, next_plan, nbytes)
+
+
 def moe_plan_destroy(plan: int) -> None:
     if plan:
         load_library().moe_plan_destroy(plan)
@@ -295,6 +301,12 @@ class MoePlan:
 
     def sync_status(self) -> int:
         return moe_sync_status(self.handle)
+
+    def set_next_layer(self, nxt, nbytes: int):
+        """Pull nbytes of nxt's front weights into L2 during each forward
+        (nxt None: off)."""
+        st = moe_set_next_layer(self.handle, nxt.handle if nxt is not None else None, nbytes)
+        _check(st, "moe_set_next_layer")
 
     def info(self) -> moe_plan_info:
         return moe_get_plan_info(self.handle)

@@ -121,6 +121,11 @@ struct Params {
   int tg;             // tokens per group (EGU/EDN/TAIL)
   int KL;             // K extent of the chunked dimension (for ragged last chunk)
   int KS;             // TAIL: K extent of the shared part (I_s)
+  // EDN: the next layer's front weights, pulled into L2 once this CTA's own
+  // stages are issued (cross-layer prefetch); pf_bytes a multiple of 16, 0:
+  // none
+  const uint8_t* pf_src;
+  long long pf_bytes;
 
   // shared memory geometry (bytes)
   int nstages, stage_bytes, act_off, act_stride, scratch_off, stage_off;

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "../../include/moe.h"
@@ -90,6 +91,11 @@ struct moe_plan_s {
 
   std::vector<void*> allocs;
   size_t packed_bytes = 0, workspace_bytes = 0;
+
+  // cross-layer prefetch (moe_set_next_layer): the plan whose front weights
+  // each forward pulls into L2, and how many of their bytes
+  moe_plan_s* next_layer = nullptr;
+  long long next_bytes = 0;
 
   uint8_t* w_front = nullptr;
   uint8_t* w_egu = nullptr;
@@ -195,6 +201,11 @@ struct moe_plan_s {
   double prof_ms[kSlots] = {};
   int prof_count = 0;
 };
+
+// Live plans, so that destroying one clears every other plan's
+// cross-layer prefetch of it.
+std::mutex g_plans_mu;
+std::vector<moe_plan_s*> g_plans;
 
 // tokens per virtual expert for a forward of B tokens
 int expert_tg(const moe_plan_s* p, int B) {
@@ -811,6 +822,15 @@ moe_status create_impl(const moe_config* cfg, int device, moe_plan p) {
 
 void destroy_impl(moe_plan p) {
   if (!p) return;
+  {
+    std::lock_guard<std::mutex> lk(g_plans_mu);
+    g_plans.erase(std::remove(g_plans.begin(), g_plans.end(), p), g_plans.end());
+    for (moe_plan_s* o : g_plans)
+      if (o->next_layer == p) {
+        o->next_layer = nullptr;
+        o->next_bytes = 0;
+      }
+  }
   DeviceGuard g(p->device);
   cudaDeviceSynchronize();
   for (void* a : p->allocs) cudaFree(a);
@@ -1059,6 +1079,18 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     q.half_sm = f.expert_per_sm == 2 ? 1 : 0;
     q.piece_ctas = f.expert_grid;
     q.split_cost = split_cost_for(p, f.nt_e);
+    {
+      // the next layer's front weights (router rows first) into L2 while
+      // this layer's expert and tail phases leave HBM idle
+      std::lock_guard<std::mutex> lk(g_plans_mu);
+      if (p->next_layer && p->next_bytes > 0) {
+        // (the copy its front kernel streams at this batch size)
+        const moe_plan_s* n = p->next_layer;
+        const FwdGeom fn = fwd_geom(n, std::min(B, n->cfg.max_tokens));
+        q.pf_src = (front_umma_for(n, fn.nt_front, fn.budget) && !fn.side) ? n->w_front_um : n->w_front;
+        q.pf_bytes = p->next_bytes;
+      }
+    }
     TRY(launch_timed(p, KIND_EDN, KIND_EDN, f.nt_e, q, f.expert_grid, sm.total, s));
   }
   {
@@ -1153,11 +1185,32 @@ moe_status moe_plan_create(const moe_config* cfg, int device, moe_plan* out) {
     destroy_impl(p);
     return st;
   }
+  {
+    std::lock_guard<std::mutex> lk(g_plans_mu);
+    g_plans.push_back(p);
+  }
   *out = p;
   return MOE_OK;
 }
 
 void moe_plan_destroy(moe_plan p) { destroy_impl(p); }
+
+moe_status moe_set_next_layer(moe_plan p, moe_plan next, int64_t bytes) {
+  if (!p || bytes < 0) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_plans_mu);
+  if (std::find(g_plans.begin(), g_plans.end(), p) == g_plans.end()) return MOE_ERR_INVALID_ARG;
+  if (!next || bytes == 0) {
+    p->next_layer = nullptr;
+    p->next_bytes = 0;
+    return MOE_OK;
+  }
+  if (std::find(g_plans.begin(), g_plans.end(), next) == g_plans.end() || next->device != p->device)
+    return MOE_ERR_INVALID_ARG;
+  const long long have = (long long)next->g[KIND_FRONT].weight_bytes;
+  p->next_layer = next;
+  p->next_bytes = std::min<long long>(bytes, have) & ~15LL;
+  return MOE_OK;
+}
 
 moe_status moe_load_weights(moe_plan p, const moe_weights* w, void* stream) {
   if (!p || !w) return MOE_ERR_INVALID_ARG;

@@ -662,6 +662,15 @@ __device__ void producer(const Params& p, Ctl* ctl, uint8_t* stage_base, uint8_t
     if (lane == 0 && in_flight) grabbed = atomicAdd(&ctl->cursor, 1) + workers;
   }
   if (!waited && (prefetched > 0 || (!free_start && !ve_dep))) resolve();
+  // cross-layer prefetch: this CTA's share of the next layer's front weights
+  // into L2, 16 KB a request (no data lands in this CTA; the copies only warm
+  // L2 for the next forward's front kernel)
+  if (KIND == KIND_EDN && p.pf_bytes > 0) {
+    const long long per = (p.pf_bytes / gridDim.x + 16383) & ~16383LL;
+    const long long lo = (long long)blockIdx.x * per, hi = min(p.pf_bytes, lo + per);
+    for (long long o = lo + (long long)lane * 16384; o < hi; o += 32LL * 16384)
+      prefetch_l2(p.pf_src + o, (uint32_t)min(16384LL, hi - o));
+  }
   if (p.trace && lane == 0) {
     unsigned long long* tr = p.trace + (size_t)blockIdx.x * kTraceStride;
     tr[11] = (unsigned long long)pw;

@@ -57,6 +57,8 @@ def test_bad_config_rejected_on_host(lib):
 def test_null_plan_calls(lib):
     assert lib.moe_forward(None, None, 1, None, None) == 1
     assert lib.moe_sync_status(None) == 1
+    assert lib.moe_set_next_layer(None, None, 0) == 1
+    assert lib.moe_set_next_layer(None, None, 1 << 20) == 1
     lib.moe_plan_destroy(None)
 
 

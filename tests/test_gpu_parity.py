@@ -111,6 +111,40 @@ def test_tiny_single_token(tiny):
     full_check(blk, synth.make_x(shape))
 
 
+@pytest.mark.parametrize("B", [1, 13])
+def test_next_layer_prefetch(tiny, B):
+    """Two plans as consecutive layers, each pulling the other's front
+    weights into L2 during its forward: outputs bit-identical to the same
+    forwards without the prefetch, and within the oracle's bounds; bad
+    arguments are rejected and destroying the next plan turns it off."""
+    shape, w = tiny
+    w2 = synth.make_weights(shape, instance=1)
+    a = GpuBlock(shape, w, max_tokens=16)
+    b = GpuBlock(shape, w2, max_tokens=16)
+    xs = [synth.make_x(shape, tokens=B, step=40 + i) for i in range(4)]
+
+    def run_pair():
+        return [blk.run(x) for blk, x in zip([a, b, a, b], xs)]
+
+    plain = run_pair()
+    a.plan.set_next_layer(b.plan, 1 << 30)  # (clamped to b's front weights)
+    b.plan.set_next_layer(a.plan, 4096)
+    pref = run_pair()
+    for u, v in zip(plain, pref):
+        np.testing.assert_array_equal(u, v)
+    full_check(a, xs[0])
+    full_check(b, xs[1])
+    with pytest.raises(RuntimeError):
+        a.plan.set_next_layer(b.plan, -1)
+    b.plan.close()
+    np.testing.assert_array_equal(a.run(xs[2]), plain[2])
+    st = moe.moe_set_next_layer(a.plan.handle, 12345, 1 << 20)  # not a live plan
+    assert st == 1
+    a.plan.set_next_layer(None, 0)
+    a.plan.set_next_layer(a.plan, 1 << 20)  # its own weights: allowed
+    np.testing.assert_array_equal(a.run(xs[0]), plain[0])
+
+
 @pytest.mark.parametrize("B", [2, 13, 16])
 def test_tiny_ragged_batches(tiny, B):
     shape, w = tiny
