@@ -170,6 +170,9 @@ struct moe_plan_s {
   // split-K piece end in the split choice, whether kernels chain with
   // programmatic dependent launch, and whether small batches run fused
   int split_cost = 2;  // split-K piece-end price in stages (environment MOE_SPLIT_COST)
+  // fixed split-K factors of the front and tail kernels (environment
+  // MOE_FRONT_PPR, MOE_TAIL_PPR; 0: the makespan model's)
+  int front_ppr_fixed = 0, tail_ppr_fixed = 0;
   int max_stages = 5;  // ring depth cap (environment MOE_MAX_STAGES)
   int expert_per_sm_max = 2;     // environment MOE_EXPERT_CTAS_PER_SM
   int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
@@ -391,13 +394,20 @@ FwdGeom fwd_geom(const moe_plan_s* p, int B) {
 int rb_routed(const moe_plan_s* p) { return p->RB_router + p->RB_lat; }
 int rb_shared(const moe_plan_s* p) { return p->g[KIND_FRONT].RB - rb_routed(p); }
 
-// Front split-K factor: over every row block, or over one lane's.
+// Front split-K factor: over every row block, or over one lane's.  Its
+// piece-end price in the makespan model is twice the base (a little more at
+// 16 token tiles), as measured by sweeping the factor at the full-size
+// dimensions (us per step): B = 1 pieces of 8 chunks 83.0 against 14 85.5
+// (6: 84.6, 4: 89.1), B = 8 158.4 against 159.6, B = 128 7 pieces a row
+// block 347.5 against 4 350.6 (10: 374.4); B = 64 keeps 7.
 int front_ppr(const moe_plan_s* p, const FwdGeom& f, bool side_part) {
   const KindGeom& g = p->g[KIND_FRONT];
-  if (!f.side) return best_ppr(g.RB, g.C, f.front_workers, p->split_cost * (1 + std::max(1, f.nt_front) / 4));
+  if (p->front_ppr_fixed > 0) return std::min(p->front_ppr_fixed, g.C);
+  const int cost = 2 * p->split_cost + f.nt_front / 16;
+  if (!f.side) return best_ppr(g.RB, g.C, f.front_workers, cost);
   const int mats = side_part ? rb_shared(p) : rb_routed(p);
   const int ctas = side_part ? f.side_grid : f.front_workers;
-  return best_ppr(mats, g.C, ctas, p->split_cost * (1 + std::max(1, f.nt_front) / 4));
+  return best_ppr(mats, g.C, ctas, cost);
 }
 
 Params base_params(const moe_plan_s* p, int B) {
@@ -527,6 +537,25 @@ TailSplit tail_split_for(const moe_plan_s* p, int ppr, int B) {
   const int sh = std::max(1, std::min(C_sh, ppr - lat));
   return {lat, sh};
 }
+// The tail's split-K factor over `mats` row blocks (before the lane split).
+// Its piece-end price depends on how the activation reaches the stages, as
+// measured by sweeping the factor at the full-size dimensions (us per step):
+//   resident activation (few tokens): three times the base, B = 1 pieces of
+//     13 chunks (5 a row block) 81.8 against 8 85.5;
+//   formed records, one or two token tiles: half the base, B = 8 13 pieces
+//     a row block 156.9 against 8 159.6;
+//   formed records, more tiles: the token-tile scaled price plus one, 4
+//     pieces a row block at B = 64 (444.2 against 5 451.8; 3: 453.4) and
+//     at B = 128 (350.6; 3: 353.4).
+int tail_base_ppr(const moe_plan_s* p, int B, int mats, int ctas, int nt) {
+  const int C = p->g[KIND_TAIL].C;
+  if (p->tail_ppr_fixed > 0) return std::min(p->tail_ppr_fixed, C);
+  const bool resident = B * resident_stride(C * kDenseChunkK) <= kResidentMax;
+  const int cost = resident ? 3 * p->split_cost
+                   : nt <= 2 ? p->split_cost / 2
+                             : p->split_cost * (1 + nt / 4) + 1;
+  return best_ppr(mats, C, ctas, cost);
+}
 int tail_ppr(const moe_plan_s* p, int ppr, int B) {
   const TailSplit t = tail_split_for(p, ppr, B);
   return t.ppr_lat + t.ppr_sh;
@@ -559,7 +588,7 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      pieces = (size_t)passes * g.RB * tail_ppr(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, nt), B);
+      pieces = (size_t)passes * g.RB * tail_ppr(p, tail_base_ppr(p, B, g.RB * passes, f.tail_grid, nt), B);
     } else {
       nt = f.nt_e;
       // the split depends on the routing: take the largest over every
@@ -642,6 +671,8 @@ void plan_shape(moe_plan_s* p) {
 // (and by moe_debug_geometry, which reports what such a plan would launch).
 void read_env(moe_plan_s* p) {
   if (const char* e = getenv("MOE_SPLIT_COST")) p->split_cost = std::max(0, atoi(e));
+  if (const char* e = getenv("MOE_FRONT_PPR")) p->front_ppr_fixed = std::max(0, std::min(64, atoi(e)));
+  if (const char* e = getenv("MOE_TAIL_PPR")) p->tail_ppr_fixed = std::max(0, std::min(64, atoi(e)));
   if (const char* e = getenv("MOE_EXPERT_CTAS_PER_SM")) p->expert_per_sm_max = std::max(1, std::min(2, atoi(e)));
   if (const char* e = getenv("MOE_EXPERT_SMALL_MAX_B")) p->expert_small_max_b = std::max(0, atoi(e));
   if (const char* e = getenv("MOE_EXPERT_PPR")) p->expert_ppr_fixed = std::max(0, std::min(8, atoi(e)));
@@ -955,7 +986,7 @@ TailLaunch tail_launch(const moe_plan_s* p, const FwdGeom& f, int B, int part) {
   const int grid = part == 2 ? f.side_grid : f.tail_grid;
   // one split for both lanes: they share every row block's partial-sum slots
   // and its ticket count
-  const TailSplit ts = tail_split_for(p, ppr_for(p, g.RB * passes, g.C, f.tail_grid, f.nt_tail), B);
+  const TailSplit ts = tail_split_for(p, tail_base_ppr(p, B, g.RB * passes, f.tail_grid, f.nt_tail), B);
   l.ppr_lat = ts.ppr_lat;
   l.ppr_sh = ts.ppr_sh;
   l.ppr = ts.ppr_lat + ts.ppr_sh;
