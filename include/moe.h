@@ -174,6 +174,10 @@ typedef struct moe_plan_info {
  *   MOE_EXPERT_TG=8|16|32   tokens per virtual expert for every B
  *   MOE_EXPERT_PPR=n        the expert kernels' split-K factor (default: the
  *                           makespan model, chosen on the device)
+ *   MOE_FRONT_PPR=n, MOE_TAIL_PPR=n  fixed split-K factors (pieces a row block)
+ *                           of the front and tail kernels (default: the
+ *                           makespan model with the piece-end prices measured
+ *                           for each kernel and activation form)
  *   MOE_ROUTE_TPC=n, MOE_ROUTE_MAX_CTAS=n  tokens per routing CTA and the
  *                           most routing CTAs (defaults 8 and 16)
  *   MOE_ROUTE_FEW=0         no one-warp selection and table build for B <= 8
