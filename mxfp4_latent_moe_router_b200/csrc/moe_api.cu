@@ -585,6 +585,13 @@ size_t partial_floats(const moe_plan_s* p, int kind) {
       const int ppr = front_ppr(p, f, false);
       const int rb_hi = f.side ? rb_routed(p) : g.RB;
       pieces = (size_t)p->RB_router * router_ppr(ppr, g.C) + (size_t)(rb_hi - p->RB_router) * ppr;
+      if (p->use_fused && B <= kFusedMaxTokens) {
+        // the single launch: every row block, never a side lane
+        FwdGeom fg = f;
+        fg.side = false;
+        const int pf = front_ppr(p, fg, false);
+        pieces = std::max(pieces, (size_t)p->RB_router * router_ppr(pf, g.C) + (size_t)(g.RB - p->RB_router) * pf);
+      }
     } else if (kind == KIND_TAIL) {
       nt = f.nt_tail;
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
@@ -910,8 +917,11 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
     q.done = p->done;
     q.need_rb_edn = p->g[KIND_EDN].RB;
     q.need_rb_sh = p->g[KIND_FRONT].RB - p->RB_router - p->RB_lat;
+    // (split factors from the functions that size the partial-sum buffers)
     if (k == KIND_FRONT) {
-      q.PPR = ppr_for(p, q.RB, q.C, f.front_workers, 1);
+      FwdGeom fg = f;
+      fg.side = false;
+      q.PPR = front_ppr(p, fg, false);
       q.PPR_r = router_ppr(q.PPR, q.C);
       mp.n_front = p->RB_router * q.PPR_r + (q.RB - p->RB_router) * q.PPR;
     } else if (k == KIND_EGU || k == KIND_EDN) {
@@ -924,7 +934,7 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
         q.res_k = res_k;
       }
       const int passes = (B + p->tail_tg - 1) / p->tail_tg;
-      q.PPR = ppr_for(p, q.RB * passes, q.C, f.tail_grid, 1);
+      q.PPR = tail_base_ppr(p, B, q.RB * passes, f.tail_grid, 1);
     }
     mp.k[k] = q;
   }
