@@ -172,7 +172,8 @@ typedef struct moe_plan_info {
  *                           ones on the tensor cores above B = 64; default
  *                           128; above it, 32-token groups)
  *   MOE_EXPERT_TG=8|16|32   tokens per virtual expert for every B
- *   MOE_EXPERT_PPR=n        the expert kernels' split-K factor (default: the
+ *   MOE_EXPERT_PPR=n        the expert kernels' split-K factor (default 1, one
+ *                           piece a row block, measured fastest; 0: the
  *                           makespan model, chosen on the device)
  *   MOE_FRONT_PPR=n, MOE_TAIL_PPR=n  fixed split-K factors (pieces a row block)
  *                           of the front and tail kernels (default: the

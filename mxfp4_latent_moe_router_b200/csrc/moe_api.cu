@@ -177,7 +177,11 @@ struct moe_plan_s {
   int expert_per_sm_max = 2;     // environment MOE_EXPERT_CTAS_PER_SM
   int expert_small_max_b = 128;  // environment MOE_EXPERT_SMALL_MAX_B
   int expert_tg_fixed = 0;       // environment MOE_EXPERT_TG (8, 16 or 32; 0: by batch size)
-  int expert_ppr_fixed = 0;      // environment MOE_EXPERT_PPR (split-K factor; 0: makespan model)
+  // the expert kernels' split-K factor (environment MOE_EXPERT_PPR; 0: the
+  // makespan model).  One piece a row block measured fastest: b1 75.2 - 75.6
+  // us per step against 78.7 - 79.0 with the model, b8 152.2 - 152.6 against
+  // 156.5 - 156.9 (paired runs on two boxes)
+  int expert_ppr_fixed = 1;
   bool use_pdl = true;
   int fail_alloc_after = -1;     // environment MOE_FAIL_ALLOC_AFTER (tests only)
   int prod_sleep = 200, cons_sleep = 32;  // environment MOE_PROD_SLEEP / MOE_CONS_SLEEP (ns)
@@ -507,15 +511,9 @@ int ppr_for(const moe_plan_s* p, int mats, int C, int ctas, int nt) {
 // The expert kernels' split-K factor for `mats` row blocks (the device
 // computes the same from the routing's count of virtual experts), or the
 // fixed one of MOE_EXPERT_PPR (at most the chunk count).
-// The expert kernels' piece-end price: twice the dense kernels' (their
-// split-K sums also wait on the tensor-memory handover).  Measured at B = 1,
-// where the plain price split expert down's row blocks in 4: one piece a row
-// block 75.2 us per step against 78.7 (expert down 18.8 against 22.9 us).
-int expert_split_cost(const moe_plan_s* p, int nt) { return 2 * split_cost_for(p, nt); }
-
 int expert_ppr(const moe_plan_s* p, int mats, int C, int ctas, int nt) {
   if (p->expert_ppr_fixed > 0) return std::min(p->expert_ppr_fixed, C);
-  return best_ppr(mats, C, ctas, expert_split_cost(p, nt));
+  return ppr_for(p, mats, C, ctas, nt);
 }
 
 // Router row blocks are the first pieces handed out and the routing waits
@@ -945,7 +943,7 @@ moe_status enqueue_fused(moe_plan p, const Params& base, const FwdGeom& f, int B
       mp.n_front = p->RB_router * q.PPR_r + (q.RB - p->RB_router) * q.PPR;
     } else if (k == KIND_EGU || k == KIND_EDN) {
       q.piece_ctas = f.expert_grid;
-      q.split_cost = expert_split_cost(p, 1);
+      q.split_cost = split_cost_for(p, 1);
     } else {
       if (res_bytes) {
         q.res_off = kStageOff + table_bytes;
@@ -1099,7 +1097,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     set_kind(q, p, KIND_EGU, sm);
     q.half_sm = f.expert_per_sm == 2 ? 1 : 0;
     q.piece_ctas = f.expert_grid;
-    q.split_cost = expert_split_cost(p, f.nt_e);
+    q.split_cost = split_cost_for(p, f.nt_e);
     TRY(launch_timed(p, KIND_EGU, KIND_EGU, f.nt_e, q, f.expert_grid, sm.total, s));
   }
   if (f.side) {
@@ -1138,7 +1136,7 @@ moe_status enqueue_forward(moe_plan p, const void* x, int B, void* out, cudaStre
     set_kind(q, p, KIND_EDN, sm);
     q.half_sm = f.expert_per_sm == 2 ? 1 : 0;
     q.piece_ctas = f.expert_grid;
-    q.split_cost = expert_split_cost(p, f.nt_e);
+    q.split_cost = split_cost_for(p, f.nt_e);
     {
       // the next layer's front weights (router rows first) into L2 while
       // this layer's expert and tail phases leave HBM idle

@@ -343,6 +343,21 @@ def test_b1_full_size_warp_mma(full_weights, monkeypatch):
         blk.plan.close()
 
 
+@pytest.mark.parametrize("ppr", ["0", "4"])
+def test_b1_full_size_split_expert_pieces(full_weights, monkeypatch, ppr):
+    """The expert kernels' split-K path on the tensor cores (partial sums out
+    of tensor memory, tickets, the finalising sum): the makespan model's
+    factor (0) and 4 pieces a row block, against the oracle."""
+    shape = synth.SHAPES["b1"]
+    monkeypatch.setenv("MOE_EXPERT_PPR", ppr)
+    blk = GpuBlock(shape, full_weights, max_tokens=128)
+    try:
+        _, (mx, mn), near = full_check(blk, synth.make_x(shape, step=3))
+        print("b1 (expert pieces %s): max_rel %.3g mean_rel %.3g near-ties %s" % (ppr, mx, mn, near))
+    finally:
+        blk.plan.close()
+
+
 # sampled tokens for the whole-block check at B = 64 and 128 (every token's
 # routing is checked): spread over the batch, both ends included
 SAMPLES = {"b8": None,
